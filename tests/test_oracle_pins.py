@@ -1,0 +1,447 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a library
+routine (torch scaled_dot_product_attention / logsumexp in float64), a closed
+form, an invariant the method guarantees, or brute force on tiny inputs.  The
+set is chosen so that a plausible slip in the oracle (a dropped term, a wrong
+sign, the wrong GQA group, a transposed predictor, a mis-sized block) fails at
+least one of them.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_decoding_eta_b200 import synth
+from oracle import eta_oracle as O
+
+
+def f64(t):
+    return t.detach().to("cpu").double().numpy()
+
+
+def tiny(seed=0, B=2, Hq=4, Hkv=2, d=16, ctx=200, blk=16, q_scale=1.0, lengths=None,
+         n_clusters=4, seg=40, needles=0):
+    w = synth.Workload("tiny-test", B=B, Hq=Hq, Hkv=Hkv, d=d, ctx=ctx, blk=blk,
+                       n_clusters=n_clusters, seg=seg, needles=needles, q_scale=q_scale,
+                       seed=seed)
+    g = synth.generate(w, "cpu", lengths=lengths)
+    K, V, q = f64(g["K"]), f64(g["V"]), f64(g["q"])
+    L = g["lengths"].numpy().astype(np.int64)
+    return w, K, V, q, L, f64(g["W"])
+
+
+def sdpa_reference(q, K, V, L, scale):
+    """torch SDPA in float64 with GQA head h -> KV head h // G, per row lengths."""
+    B, Hq, d = q.shape
+    Hkv, Tm = K.shape[1], K.shape[2]
+    G = Hq // Hkv
+    Kt = torch.from_numpy(K).repeat_interleave(G, dim=1)
+    Vt = torch.from_numpy(V).repeat_interleave(G, dim=1)
+    qt = torch.from_numpy(q)[:, :, None, :]
+    mask = torch.arange(Tm)[None, :] < torch.from_numpy(L)[:, None]       # [B, Tm]
+    o = torch.nn.functional.scaled_dot_product_attention(
+        qt, Kt, Vt, attn_mask=mask[:, None, None, :], scale=scale)[:, :, 0, :]
+    s = torch.einsum("bhd,bhtd->bht", torch.from_numpy(q), Kt) * scale
+    s = s.masked_fill(~mask[:, None, :], -math.inf)
+    return o.numpy(), torch.logsumexp(s, dim=-1).numpy()
+
+
+# --------------------------------------------------------------------------
+# tau = -inf reduces to standard softmax attention (library routine)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("T", [0.0, 0.05])
+@pytest.mark.parametrize("prune", [O.PRUNE_SKIP, O.PRUNE_FLOOR])
+def test_tau_neg_inf_is_softmax_attention(T, prune):
+    w, K, V, q, L, W = tiny(seed=1, lengths=torch.tensor([200, 77]))
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk, V)
+    tau = np.full((w.B, w.Hq), -np.inf)
+    sc = O.screen(q, tau, meta, scale)
+    o, lse = O.decode(q, tau, K, V, L, sc["union_idx"], w.blk, scale, T, prune, meta)
+    o_ref, lse_ref = sdpa_reference(q, K, V, L, scale)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+    # every non-empty block is admitted, empty ones never
+    assert np.array_equal(sc["union"], meta["cnt"] > 0)
+
+
+def test_dense_decode_matches_library():
+    w, K, V, q, L, W = tiny(seed=2, lengths=torch.tensor([131, 200]))
+    scale = O.default_scale(w.d)
+    o, lse = O.dense_decode(q, K, V, L, scale)
+    o_ref, lse_ref = sdpa_reference(q, K, V, L, scale)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+
+
+def test_gqa_group_is_h_div_G():
+    # If head h used KV head h % Hkv instead of h // G, the library check fails:
+    # make the two KV heads very different so the mapping matters.
+    w, K, V, q, L, W = tiny(seed=3, Hq=4, Hkv=2)
+    V[:, 1] += 5.0
+    scale = O.default_scale(w.d)
+    o, _ = O.dense_decode(q, K, V, L, scale)
+    o_ref, _ = sdpa_reference(q, K, V, L, scale)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    assert o[:, 0].mean() < 2.5 < o[:, 3].mean()
+
+
+# --------------------------------------------------------------------------
+# tau above every score: hard gate sends every logit to 0 -> uniform mean
+# --------------------------------------------------------------------------
+def test_tau_above_scores_gives_uniform_mean():
+    w, K, V, q, L, W = tiny(seed=4, lengths=torch.tensor([200, 93]))
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk, V)
+    G = w.G
+    tau = np.zeros((w.B, w.Hq))
+    for b in range(w.B):
+        for h in range(w.Hq):
+            s = scale * K[b, h // G, :L[b]] @ q[b, h]
+            tau[b, h] = s.max() + 0.25
+            o, lse = O.dense_gated(q[b, h], tau[b, h], K[b, h // G], V[b, h // G], L[b], scale, 0.0)
+            np.testing.assert_allclose(o, V[b, h // G, :L[b]].mean(axis=0), atol=1e-12)
+            assert abs(lse - math.log(L[b])) < 1e-12
+    # FLOOR mode with pruning gives the same uniform mean over all valid keys
+    sc = O.screen(q, tau, meta, scale)
+    o, lse = O.decode(q, tau, K, V, L, sc["union_idx"], w.blk, scale, 0.0, O.PRUNE_FLOOR, meta)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            np.testing.assert_allclose(o[b, h], V[b, h // G, :L[b]].mean(axis=0), atol=1e-12)
+            assert abs(lse[b, h] - math.log(L[b])) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# exact geometric bound is sound: brute force over every key
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("q_scale", [1.0, 8.0])
+def test_exact_bound_dominates_every_key(q_scale):
+    w, K, V, q, L, W = tiny(seed=5, q_scale=q_scale, lengths=torch.tensor([200, 150]),
+                            needles=3)
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk)
+    G = w.G
+    for b in range(w.B):
+        for h in range(w.Hq):
+            ub = O.block_bounds(q[b, h], meta["cent"][b, h // G], meta["rmax"][b, h // G],
+                                meta["var"][b, h // G], scale)
+            for j in range(w.NB):
+                n = meta["cnt"][b, h // G, j]
+                if n == 0:
+                    continue
+                keys = K[b, h // G, j * w.blk: j * w.blk + n]
+                s = scale * keys @ q[b, h]
+                assert s.max() <= ub[j] * (1 + 1e-12) + 1e-12
+
+
+@pytest.mark.parametrize("density", [0.1, 0.38, 0.7])
+def test_no_key_above_tau_in_a_pruned_block(density):
+    w, K, V, q, L, W = tiny(seed=6, q_scale=8.0, needles=4)
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk)
+    G = w.G
+    tau = O.predict_tau(q, W, np.zeros(w.Hq))
+    ub = O.screen(q, tau, meta, scale)["bounds"]
+    tau = tau + O.offset_for_density(ub, tau, np.repeat(meta["cnt"] > 0, G, 1), density, G)
+    sc = O.screen(q, tau, meta, scale)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            s = scale * K[b, h // G, :L[b]] @ q[b, h]
+            for t in np.nonzero(s >= tau[b, h])[0]:
+                assert sc["admit"][b, h, t // w.blk]
+                assert sc["union"][b, h // G, t // w.blk]
+
+
+# --------------------------------------------------------------------------
+# pruning: FLOOR mode equals dense hard gating (exact bound)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("density", [0.05, 0.38, 0.9])
+def test_floor_prune_equals_dense_hard_gating(density):
+    w, K, V, q, L, W = tiny(seed=7, q_scale=8.0, needles=4, lengths=torch.tensor([200, 121]))
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk, V)
+    G = w.G
+    tau = O.predict_tau(q, W, np.zeros(w.Hq))
+    ub = O.screen(q, tau, meta, scale)["bounds"]
+    tau = tau + O.offset_for_density(ub, tau, np.repeat(meta["cnt"] > 0, G, 1), density, G)
+    sc = O.screen(q, tau, meta, scale)
+    o, lse = O.decode(q, tau, K, V, L, sc["union_idx"], w.blk, scale, 0.0, O.PRUNE_FLOOR, meta)
+    n_above = 0
+    for b in range(w.B):
+        for h in range(w.Hq):
+            od, ld = O.dense_gated(q[b, h], tau[b, h], K[b, h // G], V[b, h // G], L[b], scale, 0.0)
+            np.testing.assert_allclose(o[b, h], od, atol=1e-12)
+            assert abs(lse[b, h] - ld) < 1e-12
+            n_above += int((scale * K[b, h // G, :L[b]] @ q[b, h] >= tau[b, h]).sum())
+    if density < 0.5:
+        assert sc["union"].mean() < 1.0   # something really was pruned
+
+
+def test_floor_invariant_over_every_admissible_block_subset():
+    """Enumerate block subsets: any union that keeps every block holding a key
+    with s >= tau gives the dense hard-gated answer in FLOOR mode."""
+    w, K, V, q, L, W = tiny(seed=8, B=1, Hq=2, Hkv=1, d=8, ctx=64, blk=16, q_scale=6.0,
+                            seg=16)
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk, V)
+    s_all = scale * K[0, 0, :L[0]] @ q[0, 0]
+    tau = float(np.sort(s_all)[-2])          # two keys at or above tau
+    need = {t // w.blk for t in np.nonzero(s_all >= tau)[0]}
+    od, ld = O.dense_gated(q[0, 0], tau, K[0, 0], V[0, 0], L[0], scale, 0.0)
+    mr = {"cnt": meta["cnt"][0, 0], "vsum": meta["vsum"][0, 0]}
+    checked = 0
+    for r in range(w.NB + 1):
+        for S in itertools.combinations(range(w.NB), r):
+            o, lse = O.attend_blocks(q[0, 0], tau, K[0, 0], V[0, 0], L[0], list(S), w.blk,
+                                     scale, 0.0, O.PRUNE_FLOOR, mr)
+            if need <= set(S):
+                np.testing.assert_allclose(o, od, atol=1e-12)
+                assert abs(lse - ld) < 1e-12
+                checked += 1
+            elif len(need - set(S)):
+                # dropping a block that holds a key above tau changes the answer
+                assert not np.allclose(o, od, atol=1e-9) or abs(lse - ld) > 1e-9
+    assert checked >= 2
+
+
+def test_skip_prune_is_gated_softmax_over_union_keys():
+    w, K, V, q, L, W = tiny(seed=9, q_scale=8.0, lengths=torch.tensor([200, 170]))
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk)
+    G = w.G
+    tau = O.predict_tau(q, W, np.zeros(w.Hq)) + 0.3
+    sc = O.screen(q, tau, meta, scale)
+    T = 0.05
+    o, lse = O.decode(q, tau, K, V, L, sc["union_idx"], w.blk, scale, T, O.PRUNE_SKIP)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            g = h // G
+            keys = [t for t in range(L[b]) if sc["union"][b, g, t // w.blk]]
+            if not keys:
+                assert np.all(o[b, h] == 0) and lse[b, h] == -math.inf
+                continue
+            s = np.array([scale * float(K[b, g, t] @ q[b, h]) for t in keys])
+            gs = np.array([x / (1 + math.exp(-(x - tau[b, h]) / T)) for x in s])
+            p = np.exp(gs - gs.max())
+            ref = sum(p[i] * V[b, g, t] for i, t in enumerate(keys)) / p.sum()
+            np.testing.assert_allclose(o[b, h], ref, atol=1e-12)
+            assert abs(lse[b, h] - (gs.max() + math.log(p.sum()))) < 1e-12
+
+
+def test_empty_union_and_empty_row():
+    w, K, V, q, L, W = tiny(seed=10, lengths=torch.tensor([0, 50]))
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk, V)
+    tau = np.full((w.B, w.Hq), np.inf)
+    sc = O.screen(q, tau, meta, scale)
+    assert not sc["union"].any()
+    o, lse = O.decode(q, tau, K, V, L, sc["union_idx"], w.blk, scale, 0.0, O.PRUNE_SKIP)
+    assert np.all(o == 0) and np.all(lse == -np.inf)
+    o, lse = O.decode(q, tau, K, V, L, sc["union_idx"], w.blk, scale, 0.0, O.PRUNE_FLOOR, meta)
+    assert np.all(o[0] == 0) and np.all(lse[0] == -np.inf)       # no keys at all
+    for h in range(w.Hq):
+        np.testing.assert_allclose(o[1, h], V[1, h // w.G, :50].mean(0), atol=1e-12)
+        assert abs(lse[1, h] - math.log(50)) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# metadata closed forms
+# --------------------------------------------------------------------------
+def test_meta_identical_keys():
+    k = np.linspace(-1, 1, 8)
+    Ks = np.tile(k, (32, 1))
+    m = O.block_meta(Ks, 32, 16)
+    np.testing.assert_allclose(m["cent"], np.tile(k, (2, 1)), atol=1e-15)
+    assert np.all(m["rmax"] < 1e-15) and np.all(m["var"] < 1e-30)
+    assert list(m["cnt"]) == [16, 16]
+
+
+def test_meta_two_point_block_and_partial_tail():
+    rng = np.random.default_rng(0)
+    a, b = rng.normal(size=6), rng.normal(size=6)
+    Ks = np.zeros((12, 6))
+    Ks[0::2][:4] = a
+    Ks[1::2][:4] = b
+    Ks[8] = a
+    Ks[9] = b
+    V = rng.normal(size=(12, 6))
+    m = O.block_meta(Ks, 10, 8, V)        # blocks: [0,8) full, [8,10) partial, rows 10.. invalid
+    dist = np.linalg.norm(a - b)
+    for j in (0, 1):
+        np.testing.assert_allclose(m["cent"][j], (a + b) / 2, atol=1e-14)
+        assert abs(m["rmax"][j] - dist / 2) < 1e-14
+        assert abs(m["var"][j] - dist ** 2 / 4) < 1e-13
+    assert list(m["cnt"]) == [8, 2]
+    np.testing.assert_allclose(m["vsum"][1], V[8:10].sum(0), atol=1e-14)
+
+
+def test_meta_against_bruteforce_loops():
+    w, K, V, q, L, W = tiny(seed=11, lengths=torch.tensor([200, 37]))
+    meta = O.cache_meta(K, L, w.blk, V)
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            for j in range(w.NB):
+                rows = [t for t in range(j * w.blk, (j + 1) * w.blk) if t < L[b]]
+                assert meta["cnt"][b, g, j] == len(rows)
+                if not rows:
+                    continue
+                c = [sum(K[b, g, t, i] for t in rows) / len(rows) for i in range(w.d)]
+                d2 = [sum((K[b, g, t, i] - c[i]) ** 2 for i in range(w.d)) for t in rows]
+                np.testing.assert_allclose(meta["cent"][b, g, j], c, atol=1e-12)
+                assert abs(meta["rmax"][b, g, j] - math.sqrt(max(d2))) < 1e-12
+                assert abs(meta["var"][b, g, j] - sum(d2) / len(rows)) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# threshold predictor (Eq. 1)
+# --------------------------------------------------------------------------
+def test_predictor_one_hot_selects_coordinate():
+    B, Hq, d = 3, 4, 5
+    rng = np.random.default_rng(1)
+    q = rng.normal(size=(B, Hq, d))
+    bias = rng.normal(size=Hq)
+    for (h_src, k, h_dst) in [(0, 0, 0), (2, 3, 1), (3, 4, 3), (1, 2, 2)]:
+        W = np.zeros((Hq * d, Hq))
+        W[h_src * d + k, h_dst] = 1.0
+        tau = O.predict_tau(q, W, bias)
+        np.testing.assert_allclose(tau[:, h_dst], q[:, h_src, k] + bias[h_dst], atol=1e-15)
+        others = [h for h in range(Hq) if h != h_dst]
+        np.testing.assert_allclose(tau[:, others], np.broadcast_to(bias[others], (B, Hq - 1)))
+
+
+def test_const_tau_broadcast():
+    t = O.const_tau(3, np.array([0.5, -1.0]))
+    assert t.shape == (3, 2) and np.all(t[:, 0] == 0.5) and np.all(t[:, 1] == -1.0)
+
+
+# --------------------------------------------------------------------------
+# gate (Eq. 2-3)
+# --------------------------------------------------------------------------
+def test_gate_closed_forms_and_hard_limit():
+    tau, T = 0.7, 0.05
+    assert abs(O.gate(np.array([tau]), tau, T)[0] - tau / 2) < 1e-15
+    x = tau + T * math.log(3.0)           # sigmoid(ln 3) = 3/4
+    assert abs(O.gate(np.array([x]), tau, T)[0] - 0.75 * x) < 1e-14
+    x = tau - T * math.log(3.0)           # sigmoid(-ln 3) = 1/4
+    assert abs(O.gate(np.array([x]), tau, T)[0] - 0.25 * x) < 1e-14
+    s = np.linspace(-3, 3, 601)
+    s = s[np.abs(s - tau) > 1e-3]
+    np.testing.assert_allclose(O.gate(s, tau, 1e-6), O.gate(s, tau, 0.0), atol=1e-12)
+    hard = O.gate(np.array([tau - 1e-12, tau, tau + 1e-12]), tau, 0.0)
+    assert hard[0] == 0.0 and hard[1] == tau and hard[2] == tau + 1e-12
+    # overflow safety far from tau
+    assert np.all(np.isfinite(O.gate(np.array([-1e4, 1e4]), 0.0, 1e-3)))
+
+
+# --------------------------------------------------------------------------
+# screening structure
+# --------------------------------------------------------------------------
+def test_union_is_or_of_heads_and_G1_equals_head_mask():
+    w, K, V, q, L, W = tiny(seed=12)
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk)
+    tau = O.predict_tau(q, W, np.zeros(w.Hq)) + 0.2
+    sc = O.screen(q, tau, meta, scale)
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            heads = sc["admit"][b, g * w.G:(g + 1) * w.G]
+            assert np.array_equal(sc["union"][b, g], heads.any(0))
+            assert np.all(sc["union"][b, g] >= heads)
+            assert np.array_equal(sc["union_idx"][b][g], np.nonzero(heads.any(0))[0])
+    # G = 1
+    w1, K1, V1, q1, L1, W1 = tiny(seed=13, Hq=2, Hkv=2)
+    meta1 = O.cache_meta(K1, L1, w1.blk)
+    tau1 = O.predict_tau(q1, W1, np.zeros(2)) + 0.2
+    sc1 = O.screen(q1, tau1, meta1, O.default_scale(w1.d))
+    assert np.array_equal(sc1["union"], sc1["admit"])
+
+
+def test_block_permutation_permutes_masks():
+    w, K, V, q, L, W = tiny(seed=14, B=1, ctx=160, blk=16)
+    scale = O.default_scale(w.d)
+    perm = np.random.default_rng(3).permutation(w.NB)
+    Kp = K.reshape(w.B, w.Hkv, w.NB, w.blk, w.d)[:, :, perm].reshape(K.shape)
+    m, mp = O.cache_meta(K, L, w.blk), O.cache_meta(Kp, L, w.blk)
+    tau = O.predict_tau(q, W, np.zeros(w.Hq)) + 0.2
+    s, sp = O.screen(q, tau, m, scale), O.screen(q, tau, mp, scale)
+    np.testing.assert_allclose(sp["bounds"], s["bounds"][:, :, perm], atol=1e-12)
+    assert np.array_equal(sp["admit"], s["admit"][:, :, perm])
+
+
+def test_ragged_lengths_blocks_beyond_length_never_admitted():
+    w, K, V, q, L, W = tiny(seed=15, lengths=torch.tensor([200, 45]))
+    meta = O.cache_meta(K, L, w.blk)
+    assert meta["cnt"][1, 0, 2] == 45 - 32 and meta["cnt"][1, 0, 3] == 0
+    tau = np.full((w.B, w.Hq), -np.inf)
+    sc = O.screen(q, tau, meta, O.default_scale(w.d))
+    assert not sc["union"][1, :, 3:].any() and sc["union"][1, :, :3].all()
+
+
+def test_probabilistic_bound_properties():
+    w, K, V, q, L, W = tiny(seed=16, q_scale=4.0)
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk)
+    ex = O.screen(q, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_EXACT)["bounds"]
+    for z in (0.5, 1.0, 3.0, math.sqrt(w.d)):
+        pr = O.screen(q, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_PROB, z)["bounds"]
+        assert np.all(pr <= ex + 1e-12)
+        # for z <= sqrt(d) the min is inactive: var <= rmax^2 gives z sqrt(var/d) <= rmax
+        for b in range(w.B):
+            for h in range(w.Hq):
+                g = h // w.G
+                qh = q[b, h]
+                want = scale * (meta["cent"][b, g] @ qh + np.linalg.norm(qh) * z
+                                * np.sqrt(meta["var"][b, g] / w.d))
+                np.testing.assert_allclose(pr[b, h], want, atol=1e-12)
+    pr = O.screen(q, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_PROB, 1e9)["bounds"]
+    np.testing.assert_allclose(pr, ex, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# calibration rule
+# --------------------------------------------------------------------------
+def test_calibration_quantile_hits_density():
+    rng = np.random.default_rng(5)
+    n_q, Hq, NB = 64, 4, 97
+    bounds = rng.normal(size=(n_q, Hq, NB))
+    valid = rng.random((n_q, Hq, NB)) > 0.1
+    for dens in (0.16, 0.38, 0.51):
+        tau = O.calibrate_const_tau(bounds, valid, dens)
+        for h in range(Hq):
+            pool = bounds[:, h][valid[:, h]]
+            frac = (pool >= tau[h]).mean()
+            assert dens <= frac <= dens + 1.0 / pool.size + 1e-12
+
+
+# --------------------------------------------------------------------------
+# hand-derived worked example (tests/golden/hand_example_d2.json)
+# --------------------------------------------------------------------------
+def test_hand_derived_example():
+    import json
+    import os
+    ex = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                     "hand_example_d2.json")))
+    K = np.array(ex["K"])[None, None]
+    V = np.array(ex["V"])[None, None]
+    q = np.array(ex["q"])[None, None]
+    L = [4]
+    want = ex["expected"]
+    meta = O.cache_meta(K, L, ex["blk"], V)
+    np.testing.assert_allclose(meta["cent"][0, 0], want["cent"], atol=1e-15)
+    np.testing.assert_allclose(meta["rmax"][0, 0], want["rmax"], atol=1e-15)
+    np.testing.assert_allclose(meta["var"][0, 0], want["var"], atol=1e-15)
+    tau = np.array([[ex["tau"]]])
+    sc = O.screen(q, tau, meta, ex["scale"])
+    np.testing.assert_allclose(sc["bounds"][0, 0], want["bounds"], atol=1e-15)
+    assert list(sc["admit"][0, 0]) == want["admit"]
+    o, lse = O.decode(q, tau, K, V, L, sc["union_idx"], ex["blk"], ex["scale"], 0.0,
+                      O.PRUNE_SKIP)
+    np.testing.assert_allclose(o[0, 0], want["o_skip"], atol=1e-15)
+    assert abs(lse[0, 0] - want["lse_skip"]) < 1e-14
+    o, lse = O.decode(q, tau, K, V, L, sc["union_idx"], ex["blk"], ex["scale"], 0.0,
+                      O.PRUNE_FLOOR, meta)
+    np.testing.assert_allclose(o[0, 0], want["o_floor"], atol=1e-15)
+    assert abs(lse[0, 0] - want["lse_floor"]) < 1e-14

@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of the ETA block-sparse decode step on B200.
+
+One step = the whole hot path for one batch of decode queries of one layer:
+  eta_build_block_meta (tail block of every row: the cache grew by one token)
+  eta_predict_tau      (Eq. 1 threshold predictor)
+  eta_screen           (O(1) block screening, per-head masks, union compaction)
+  eta_decode           (gated split-KV attention over admitted blocks + LSE combine)
+
+Default workload: batch 64, 16 query / 4 KV heads, d = 128, 128K context, KV
+block 64, bf16 clustered-key cache (256 clusters, segments of 384-640 tokens),
+threshold bias calibrated for 16% union density, exact bound, hard gate.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the float64 CPU oracle
+on a bounded sample of the same workload instead (rank 0 only).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl eta|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_decoding_eta_b200 import synth  # noqa: E402
+
+METRIC = "decode attn steps/s and HBM GB/s on admitted KV bytes (% of B200 peak)"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+LAUNCHES_PER_STEP = 7   # meta tail 1 + tau 1 + screen 2 + decode 3 (plan, decode, combine)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_by_name(name: str) -> synth.Workload:
+    for w in synth.WORKLOADS.values():
+        if w.name == name or w.name.startswith(name):
+            return w
+    raise SystemExit(f"unknown workload {name}; choose from {list(synth.WORKLOADS)}")
+
+
+def density_offset(bounds: np.ndarray, tau0: np.ndarray, valid: np.ndarray, density: float,
+                   G: int, kind: str) -> float:
+    """Common threshold offset that admits the target fraction of (head, block)
+    pairs ("head") or (KV group, block) pairs ("union"): a quantile of the
+    margins bound - tau.  Workload calibration only (host numpy)."""
+    B, Hq, NB = bounds.shape
+    m = np.where(valid, bounds - tau0[:, :, None], -np.inf)
+    if kind == "union":
+        m = m.reshape(B, Hq // G, G, NB).max(axis=2)
+    v = m[np.isfinite(m)]
+    k = int(math.floor((1.0 - density) * v.size))
+    k = min(max(k, 0), v.size - 1)
+    return float(np.partition(v, k)[k])
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}",
+                                          f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def setup(w: synth.Workload, device, rank: int):
+    from long_context_decoding_eta_b200.api import EtaDecoder
+    g = synth.generate(w, device, seed=w.seed + 7919 * rank)
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, bound=w.bound, z=w.z,
+                     T=w.gate_T, keep_bounds=True)
+    dec.build_meta()
+    # workload calibration: bias so that tau hits the density target
+    if w.tau_mode == "const":
+        qc = synth.calibration_queries(w, g["mu"])
+        tau_const = dec.calibrate_const_tau(qc, w.density).to(device)
+        W = bias = None
+    else:
+        tau_const = None
+        W = g["W"]
+        dec.predict_tau(g["q"], W, None, None)
+        tau0 = dec.tau.clone()
+        dec.screen(g["q"], tau0, bounds=dec.bounds)
+        valid = (dec.cnt > 0).repeat_interleave(w.G, dim=1).cpu().numpy()
+        off = density_offset(dec.bounds.cpu().numpy(), tau0.cpu().numpy(), valid, w.density,
+                             w.G, w.density_kind)
+        bias = torch.full((w.Hq,), off, dtype=torch.float32, device=device)
+    dec.bounds = None
+    return g, dec, W, bias, tau_const
+
+
+def step_bytes(dec, w):
+    """Algorithmic HBM bytes of one step, from the step's own screening output."""
+    lengths = dec.lengths.to(torch.int64)
+    B, Hkv, NB, blk, d = dec.B, dec.Hkv, dec.NB, dec.blk, dec.d
+    cnt = dec.cnt.to(torch.int64)                          # [B, Hkv, NB] valid keys per block
+    idx = dec.union_idx.to(torch.int64)
+    ucnt = dec.union_cnt.to(torch.int64)
+    ar = torch.arange(NB, device=cnt.device)
+    take = ar[None, None, :] < ucnt[:, :, None]
+    keys = torch.where(take, torch.gather(cnt, 2, idx.clamp(0, NB - 1)), 0).sum()
+    adm_kv = int(keys) * d * 2 * 2                          # K + V, bf16
+    qbytes = B * w.Hq * d * 2
+    obytes = B * w.Hq * (d + 1) * 4
+    meta = B * Hkv * NB * (4 * d + 12)                      # cent + rmax + var + cnt read by screen
+    tail = B * Hkv * (blk * d * 2 + (4 * d + 12))           # tail block keys read + meta written
+    tau_bytes = w.Hq * d * w.Hq * 4 + B * w.Hq * 4
+    dens_union = float(ucnt.sum()) / max(1.0, float((cnt > 0).sum()))
+    dens_head = float(dec.head_cnt.to(torch.int64).sum()) / max(
+        1.0, float((cnt > 0).sum()) * (w.Hq // Hkv))
+    return dict(decode=adm_kv + qbytes + obytes, step=adm_kv + qbytes + obytes + meta + tail
+                + tau_bytes, admitted_kv=adm_kv, meta=meta, union_density=dens_union,
+                head_density=dens_head, dense_kv=int(lengths.sum()) * Hkv * d * 4)
+
+
+def run_eta(args, rank, world, device):
+    w = workload_by_name(args.workload)
+    g, dec, W, bias, tau_const = setup(w, device, rank)
+    q = g["q"]
+    stream = torch.cuda.current_stream()
+    # one step to measure densities / bytes, then check status
+    dec.step(q, W, bias, tau_const)
+    torch.cuda.synchronize()
+    dec.check_status()
+    by = step_bytes(dec, w)
+
+    def one_step(ev=None):
+        dec.append_update()
+        dec.predict_tau(q, W, bias, tau_const)
+        dec.screen(q)
+        if ev is not None:
+            ev[0].record(stream)
+        dec.decode(q)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(device.index if device.index is not None else 0) as clk:
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            one_step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    dec.check_status()
+    ms = t0.elapsed_time(t1)
+    dec_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # dense baseline on the same cache (same pipeline, every block, no gate)
+    for _ in range(3):
+        dec.dense_decode(q)
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nd = max(3, min(args.steps, 10))
+    d0.record(stream)
+    for _ in range(nd):
+        dec.dense_decode(q)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = d0.elapsed_time(d1) / nd
+
+    # end to end through the public API with host buffers
+    q_host = q.cpu().pin_memory()
+    o_host = torch.empty(dec.o.shape, dtype=torch.float32).pin_memory()
+    lse_host = torch.empty(dec.lse.shape, dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(q)
+
+    def e2e_step():
+        q_dev.copy_(q_host, non_blocking=True)
+        dec.step(q_dev, W, bias, tau_const)
+        o_host.copy_(dec.o, non_blocking=True)
+        lse_host.copy_(dec.lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    peak, peak_kind = peaks()
+    ms_step = ms / args.steps
+    achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC,
+        "value": world * args.steps / (ms * 1e-3),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "context": w.ctx, "blk": w.blk, "bound": w.bound, "gate_T": w.gate_T,
+            "tau_mode": w.tau_mode,
+            "density_target": f"{w.density:.2f} {w.density_kind}",
+            "union_density": round(by["union_density"], 4),
+            "head_density": round(by["head_density"], 4),
+            "l2": "no flush: admitted K/V per step and the screened metadata exceed the 126 MB L2",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "hbm_gbs": by["step"] / (ms_step * 1e-3) / 1e9,
+        "hbm_frac_of_nominal_8tbs": by["step"] / (ms_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
+        "bytes_per_step": {"admitted_kv": by["admitted_kv"], "metadata": by["meta"],
+                           "total": by["step"], "dense_kv": by["dense_kv"]},
+        "roofline": {"kernel": "eta_decode (plan + split-KV decode + combine)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                     "decode_ms": dec_ms, "traffic": None},
+        "dense_baseline": {"ms": dense_ms, "steps_per_s_decode_only": 1e3 / dense_ms,
+                           "gbs": by["dense_kv"] / (dense_ms * 1e-3) / 1e9,
+                           "speedup_of_eta_decode": dense_ms / dec_ms},
+        "e2e": {"value": world / (e2e_ms * 1e-3), "unit": "steps/s",
+                "h2d_bytes_per_step": q_host.numel() * 2,
+                "d2h_bytes_per_step": o_host.numel() * 4 + lse_host.numel() * 4},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, g, dec, W, bias, tau_const, rows=args.cpu_rows)
+    return res
+
+
+def oracle_sample_step(w, g, W, bias, tau_const, rows):
+    """Float64 oracle over a sample of batch rows (all heads of those rows).
+    Returns (seconds for one step of the sample, threads used)."""
+    from oracle import eta_oracle as O
+    sel = list(rows)
+    K64 = g["K"][sel].double().cpu().numpy()
+    V64 = g["V"][sel].double().cpu().numpy()
+    q64 = g["q"][sel].double().cpu().numpy()
+    L = g["lengths"][sel].cpu().numpy()
+    meta = O.cache_meta(K64, L, w.blk)           # prefill (not timed)
+    W64 = None if W is None else W.double().cpu().numpy()
+    b64 = None if bias is None else bias.double().cpu().numpy()
+    tc = None if tau_const is None else tau_const.double().cpu().numpy()
+    scale = 1.0 / math.sqrt(w.d)
+    t = time.perf_counter()
+    # tail-block metadata of every sampled (row, KV head)
+    for i in range(len(sel)):
+        j = (int(L[i]) - 1) // w.blk
+        for h in range(w.Hkv):
+            m = O.block_meta(K64[i, h, j * w.blk:(j + 1) * w.blk], int(L[i]) - j * w.blk, w.blk)
+            for k in ("cent", "rmax", "var", "cnt"):
+                meta[k][i, h, j] = m[k][0]
+    tau = O.predict_tau(q64, W64, b64) if tc is None else O.const_tau(len(sel), tc)
+    sc = O.screen(q64, tau, meta, scale, w.bound, w.z)
+    O.decode(q64, tau, K64, V64, L, sc["union_idx"], w.blk, scale, w.gate_T)
+    dt = time.perf_counter() - t
+    return dt, threads_used()
+
+
+def threads_used():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, g, dec, W, bias, tau_const, rows=2):
+    dt, cores = oracle_sample_step(w, g, W, bias, tau_const, range(rows))
+    per_step = dt * w.B / rows
+    return {"value": 1.0 / per_step, "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} of {w.B} batch rows (all {w.Hq} heads), float64 numpy oracle, "
+                      f"{dt:.2f} s measured, scaled by B/{rows}"}
+
+
+def run_reference(args, rank, world, device):
+    """The float64 CPU oracle as the reference arm, on a bounded sample per step.
+    The threshold bias is set by the oracle itself on the sampled rows, with the
+    same density rule as the eta arm; no CUDA kernel of this package runs."""
+    from oracle import eta_oracle as O
+    w = workload_by_name(args.workload)
+    g = synth.generate(w, device, seed=w.seed)
+    rows = list(range(args.cpu_rows))
+    K64 = g["K"][rows].double().cpu().numpy()
+    q64 = g["q"][rows].double().cpu().numpy()
+    L = g["lengths"][rows].cpu().numpy()
+    scale = 1.0 / math.sqrt(w.d)
+    meta = O.cache_meta(K64, L, w.blk)
+    W = bias = tau_const = None
+    if w.tau_mode == "const":
+        qc = synth.calibration_queries(w, g["mu"]).double().cpu().numpy()
+        n = qc.shape[0]
+        bounds = np.zeros((n, w.Hq, w.NB))
+        valid = np.zeros((n, w.Hq, w.NB), dtype=bool)
+        for i in range(n):
+            r = i % len(rows)
+            mrow = {k: v[r:r + 1] for k, v in meta.items()}
+            bounds[i] = O.screen(qc[i:i + 1], np.zeros((1, w.Hq)), mrow, scale, w.bound,
+                                 w.z)["bounds"][0]
+            valid[i] = np.repeat(meta["cnt"][r] > 0, w.G, axis=0)
+        tau_const = torch.from_numpy(O.calibrate_const_tau(bounds, valid, w.density))
+    else:
+        W = g["W"]
+        W64 = W.double().cpu().numpy()
+        tau0 = O.predict_tau(q64, W64, np.zeros(w.Hq))
+        ub = O.screen(q64, tau0, meta, scale, w.bound, w.z)["bounds"]
+        off = O.offset_for_density(ub, tau0, np.repeat(meta["cnt"] > 0, w.G, axis=1),
+                                   w.density, w.G, w.density_kind)
+        bias = torch.full((w.Hq,), off, dtype=torch.float64)
+    del K64
+    for _ in range(args.warmup):
+        oracle_sample_step(w, g, W, bias, tau_const, rows)
+    times = []
+    cores = 1
+    for _ in range(args.steps):
+        dt, cores = oracle_sample_step(w, g, W, bias, tau_const, rows)
+        times.append(dt * w.B / len(rows))
+    per = sum(times) / len(times)
+    v = 1.0 / per
+    return {
+        "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                   "context": w.ctx, "blk": w.blk},
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{len(rows)} of {w.B} batch rows per step (all heads), "
+                                   f"scaled by B/{len(rows)}"},
+        "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=synth.LONG128K.name)
+    ap.add_argument("--impl", default="eta", choices=["eta", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference" and rank != 0:
+        return 0
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1 and args.impl == "eta":
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=device)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, 1, device)
+        else:
+            res = run_eta(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1 and args.impl == "eta":
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,210 @@
+/*
+ * eta.h -- C ABI of the Elastic Threshold Attention (ETA) block-sparse decode step
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The method (arXiv 2609.20888, "Elastic Threshold Attention: Learned Contextual
+ * Sparsity for Long-Context Decoding"; abstract, and the evolve.pub review's FAQ,
+ * Summary and Methodology Assessment, Eq. 1-3): for each decode query, a threshold
+ * tau is predicted per query head (or frozen to a calibrated per-head constant);
+ * every KV block is screened in O(1) from cached per-block metadata against a
+ * score bound; blocks whose bound falls below tau are never loaded; the query
+ * heads of one KV group attend over the union of their admitted blocks with
+ * multiplicatively gated logits s' = s * sigmoid((s - tau) / T) (T -> 0: hard gate,
+ * a sub-threshold key keeps weight e^0 = 1).
+ *
+ * Conventions (all entry points):
+ *  - Every tensor argument is a caller-owned DEVICE pointer unless said otherwise.
+ *    The library never allocates, frees or retains memory.  Scratch comes from a
+ *    caller-provided workspace whose size the *_workspace_size query returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *    legacy default stream) and never synchronize the host.
+ *  - Host-side argument errors are returned immediately as ETA_ERR_* and nothing is
+ *    launched.  A launch failure returns ETA_ERR_CUDA.
+ *  - Errors found on the device (bounded waits that ran out, non-finite queries,
+ *    malformed block lists) are OR-ed into the caller's int32 word `dev_status`
+ *    (device memory, may be NULL to ignore them) as ETA_DEVSTAT_* bits; read it
+ *    after synchronizing the stream.  The caller zeroes it.
+ *  - bf16 tensors are passed as eta_bf16_t (the raw 16-bit pattern).
+ *  - Shapes: d in {64, 128}; blk in {64, 128}; G = Hq / Hkv in {1, 2, 4, 8};
+ *    T_max a multiple of blk; NB = T_max / blk blocks per (row, KV head);
+ *    NW = ceil(NB / 32) mask words.  Other shapes return ETA_ERR_UNSUPPORTED.
+ *  - Logit units: s = scale * (q . k), scale = 1/sqrt(d) when the scale argument is
+ *    0.  tau and every block bound are in these units.
+ */
+#ifndef ETA_H_
+#define ETA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t eta_bf16_t;
+
+typedef enum {
+  ETA_OK = 0,
+  ETA_ERR_INVALID_ARG = 1,     /* null pointer, negative size, misaligned pointer */
+  ETA_ERR_UNSUPPORTED = 2,     /* shape outside the supported set above */
+  ETA_ERR_WORKSPACE = 3,       /* workspace NULL or smaller than the query says */
+  ETA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
+  ETA_ERR_DEVICE_TIMEOUT = 5,  /* returned by eta_status_from_device() */
+  ETA_ERR_NONFINITE = 6        /* returned by eta_status_from_device() */
+} eta_status_t;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define ETA_DEVSTAT_TIMEOUT 0x1      /* a bounded pipeline wait gave up; outputs invalid */
+#define ETA_DEVSTAT_NONFINITE_Q 0x2  /* a query element was NaN or Inf */
+#define ETA_DEVSTAT_BAD_BLOCK 0x4    /* a block index out of range or an empty block */
+#define ETA_DEVSTAT_BAD_LENGTH 0x8   /* lengths[b] < 0 or > T_max (clamped) */
+
+typedef struct {
+  int32_t B;      /* batch rows (decode queries) */
+  int32_t Hq;     /* query heads */
+  int32_t Hkv;    /* KV heads; query head h reads KV head h / (Hq / Hkv) */
+  int32_t d;      /* head dimension */
+  int32_t blk;    /* KV block size in tokens */
+  int32_t T_max;  /* token capacity (stride) of the cache per (row, KV head) */
+} eta_dims_t;
+
+typedef enum { ETA_BOUND_EXACT = 0, ETA_BOUND_PROB = 1 } eta_bound_t;
+typedef enum { ETA_PRUNE_SKIP = 0, ETA_PRUNE_FLOOR = 1 } eta_prune_t;
+
+/* blk_begin value selecting the tail block (the one holding token lengths[b]-1)
+   of every row: the per-token append update. */
+#define ETA_TAIL_BLOCK (-1)
+
+/*
+ * eta_build_block_meta -- per-block key metadata (review Summary: "cached
+ * centroid/variance/max-norm metadata"; abstract: "cached geometric-probabilistic
+ * bounds").  For block j of (row b, KV head g) with n_j = clamp(lengths[b] - j*blk,
+ * 0, blk) valid keys k_t:
+ *   cent_j = (1/n_j) sum_t k_t                       (fp32)
+ *   rmax_j >= max_t ||k_t - cent_j||, measured against the stored fp32 cent_j and
+ *            rounded up so that the Cauchy-Schwarz bound stays sound in fp32
+ *   var_j  = (1/n_j) sum_t ||k_t - cent_j||^2
+ *   cnt_j  = n_j;  vsum_j = sum_t v_t (only when vsum != NULL)
+ * Empty blocks get zeros.
+ *
+ * K, V     bf16 [B, Hkv, T_max, d].  V may be NULL when vsum is NULL.
+ * lengths  int32 [B], valid tokens per row (keys t < lengths[b]).
+ * blk_begin, blk_end: recompute blocks [blk_begin, blk_end) of every row
+ *          (blk_end = -1: up to NB); blk_begin = ETA_TAIL_BLOCK: only the tail
+ *          block of each row (rows with lengths[b] = 0 are left untouched).
+ * cent     fp32 [B, Hkv, d, NB]  (dimension-major per row, for coalesced screening)
+ * rmax,var fp32 [B, Hkv, NB];  cnt int32 [B, Hkv, NB]
+ * vsum     fp32 [B, Hkv, NB, d] or NULL (needed only by ETA_PRUNE_FLOOR)
+ */
+eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_bf16_t* K,
+                                  const eta_bf16_t* V, const int32_t* lengths,
+                                  int32_t blk_begin, int32_t blk_end, float* cent,
+                                  float* rmax, float* var, int32_t* cnt, float* vsum,
+                                  void* stream);
+
+/*
+ * eta_predict_tau -- per-query, per-head threshold (review Methodology Assessment,
+ * Eq. 1: tau = qbar W_tau + b_tau on the concatenated post-RoPE queries; abstract:
+ * frozen per-head constants after calibration).
+ *   predictor mode (tau_const == NULL):
+ *     tau[b, h] = sum_{i < Hq*d} qbar[b, i] * W[i, h] + bias[h],  qbar[b] = concat_h q[b, h]
+ *   constant mode (tau_const != NULL): tau[b, h] = tau_const[h]; W and bias ignored.
+ * q     bf16 [B, Hq, d];  W fp32 [Hq*d, Hq] row-major;  bias fp32 [Hq] or NULL (= 0)
+ * tau_const fp32 [Hq] or NULL;  tau (out) fp32 [B, Hq]
+ * dev_status: ETA_DEVSTAT_NONFINITE_Q if q holds NaN/Inf (predictor mode).
+ */
+eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const float* W,
+                             const float* bias, const float* tau_const, float* tau,
+                             int32_t* dev_status, void* stream);
+
+/*
+ * eta_screen -- O(1)-per-block screening with hard pruning (review FAQ: blocks whose
+ * best possible score falls below the threshold are skipped; abstract: screening
+ * "in O(1) time using cached geometric-probabilistic bounds"; co-admission across
+ * the query heads of a KV group).
+ *   UB[b,h,j] = scale * (q.cent_j + ||q|| * R_j),  q = q[b,h], g = h / G
+ *     ETA_BOUND_EXACT: R_j = rmax_j                      (Cauchy-Schwarz, sound)
+ *     ETA_BOUND_PROB:  R_j = min(rmax_j, z * sqrt(var_j / d))
+ *   admit[b,h,j] = cnt_j > 0 && UB[b,h,j] >= tau[b,h]
+ *   union[b,g,j] = OR over the G query heads of group g
+ * Outputs:
+ *   head_mask  uint32 [B, Hq, NW]: bit (j % 32) of word j / 32 = admit[b,h,j]
+ *   union_idx  int32  [B, Hkv, NB]: admitted-union block indices, ascending; the
+ *              first union_cnt[b,g] entries are valid, the rest untouched
+ *   union_cnt  int32  [B, Hkv]
+ *   bounds_out fp32   [B, Hq, NB] or NULL (calibration, near-tie logging)
+ *   head_cnt   int32  [B, Hq] or NULL: popcount of the head's admit mask
+ * ws/ws_bytes: scratch of at least eta_screen_workspace_size(dims) bytes.
+ */
+size_t eta_screen_workspace_size(const eta_dims_t* dims);
+eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
+                        const float* cent, const float* rmax, const float* var,
+                        const int32_t* cnt, eta_bound_t bound, float z, float scale,
+                        uint32_t* head_mask, int32_t* union_idx, int32_t* union_cnt,
+                        float* bounds_out, int32_t* head_cnt, void* ws, size_t ws_bytes,
+                        int32_t* dev_status, void* stream);
+
+/*
+ * eta_decode -- gated attention over the admitted-union blocks only (review
+ * Methodology Assessment, Eq. 2-3 with beta = 1/T; review FAQ: a sub-threshold
+ * logit goes to zero, weight e^0 = 1; abstract: co-admitted tokens are absorbed).
+ * Each query head h of group g attends over every valid key t of the blocks
+ * union_idx[b,g,0..union_cnt[b,g]) with its own tau[b,h]:
+ *   s_t  = scale * q[b,h] . k_t
+ *   s'_t = s_t * sigmoid((s_t - tau) / T)      (T > 0)
+ *   s'_t = s_t if s_t >= tau else 0            (T == 0, hard gate)
+ *   o[b,h] = sum_t e^{s'_t} v_t / sum_t e^{s'_t},   lse[b,h] = log sum_t e^{s'_t}
+ * ETA_PRUNE_SKIP: pruned blocks are absent from the softmax; an empty union gives
+ *   o = 0, lse = -inf.
+ * ETA_PRUNE_FLOOR: every valid key of a pruned block enters with logit 0 (its
+ *   hard-gated value), using cnt and vsum from eta_build_block_meta (both required).
+ * Split-KV over the admitted list (every CTA streams an equal share of admitted
+ * blocks, TMA bulk copies into shared memory), fp32 online softmax, LSE combine.
+ * K, V bf16 [B, Hkv, T_max, d], 16-byte aligned.  o fp32 [B, Hq, d], lse fp32 [B, Hq].
+ * ws/ws_bytes: scratch of at least eta_decode_workspace_size(dims) bytes (for the
+ * current device).  dev_status bits: TIMEOUT, NONFINITE_Q, BAD_BLOCK, BAD_LENGTH.
+ */
+size_t eta_decode_workspace_size(const eta_dims_t* dims);
+eta_status_t eta_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
+                        const eta_bf16_t* K, const eta_bf16_t* V, const int32_t* lengths,
+                        const int32_t* union_idx, const int32_t* union_cnt, float T,
+                        float scale, eta_prune_t prune, const float* vsum,
+                        const int32_t* cnt, float* o, float* lse, void* ws,
+                        size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * eta_dense_decode -- the dense baseline the speedups are measured against (the
+ * pages compare with FlashAttention-2 decode): standard softmax decode attention
+ * over every valid key, no threshold, no gate, same split-KV pipeline as eta_decode.
+ * Workspace: eta_decode_workspace_size(dims).
+ */
+eta_status_t eta_dense_decode(const eta_dims_t* dims, const eta_bf16_t* q,
+                              const eta_bf16_t* K, const eta_bf16_t* V,
+                              const int32_t* lengths, float scale, float* o, float* lse,
+                              void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * eta_calibrate_const_tau -- offline calibration of frozen per-head thresholds
+ * (abstract: "an offline calibration algorithm ... that freezes per-head constant
+ * thresholds").  HOST pointers.  The pages do not print the algorithm; the rule
+ * implemented: for each head h, pool bounds[i, h, j] over the n_q calibration
+ * queries and the blocks with valid[i, h, j] != 0, sort ascending, and return the
+ * element at index floor((1 - density) * N), so that admit-iff-bound>=tau admits
+ * at least the target fraction of the pooled (query, block) pairs.
+ * bounds fp32 [n_q, Hq, NB] (eta_screen's bounds_out), valid uint8 [n_q, Hq, NB],
+ * tau_out fp32 [Hq].  Returns ETA_ERR_INVALID_ARG if a head has no valid entry.
+ */
+eta_status_t eta_calibrate_const_tau(const float* bounds, const uint8_t* valid,
+                                     int32_t n_q, int32_t Hq, int32_t NB, float density,
+                                     float* tau_out);
+
+/* Maps a device status word (read back by the caller) to a status code. */
+eta_status_t eta_status_from_device(int32_t dev_status);
+
+/* Human-readable name of a status code (static storage). */
+const char* eta_status_string(eta_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ETA_H_ */

@@ -1,0 +1,169 @@
+"""ctypes binding of libeta.so: the C ABI declared in include/eta.h, one Python
+function per entry point with the same name.  Argument marshalling only: torch
+tensors are turned into device pointers, and every non-OK status raises.
+
+The library must be built (python -m long_context_decoding_eta_b200.build); there
+is no fallback of any kind when it is missing.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libeta.so")
+
+ETA_OK = 0
+STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape",
+                3: "workspace missing or too small", 4: "CUDA error",
+                5: "device wait timed out", 6: "non-finite query"}
+BOUND = {"exact": 0, "prob": 1}
+PRUNE = {"skip": 0, "floor": 1}
+TAIL_BLOCK = -1
+DEVSTAT_TIMEOUT, DEVSTAT_NONFINITE_Q, DEVSTAT_BAD_BLOCK, DEVSTAT_BAD_LENGTH = 1, 2, 4, 8
+
+EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size",
+           "eta_screen", "eta_decode_workspace_size", "eta_decode", "eta_dense_decode",
+           "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string")
+
+
+class EtaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {code} ({STATUS_NAMES.get(code, '?')})")
+        self.code = code
+
+
+class Dims(C.Structure):
+    _fields_ = [("B", C.c_int32), ("Hq", C.c_int32), ("Hkv", C.c_int32), ("d", C.c_int32),
+                ("blk", C.c_int32), ("T_max", C.c_int32)]
+
+    @classmethod
+    def of(cls, B, Hq, Hkv, d, blk, T_max):
+        return cls(int(B), int(Hq), int(Hkv), int(d), int(blk), int(T_max))
+
+    def __repr__(self):
+        return (f"Dims(B={self.B}, Hq={self.Hq}, Hkv={self.Hkv}, d={self.d}, blk={self.blk}, "
+                f"T_max={self.T_max})")
+
+
+_lib: Optional[C.CDLL] = None
+P = C.c_void_p
+I32 = C.c_int32
+F32 = C.c_float
+DIMS = C.POINTER(Dims)
+
+
+def lib() -> C.CDLL:
+    """Loads libeta.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m long_context_decoding_eta_b200.build`")
+    L = C.CDLL(LIB_PATH)
+    L.eta_build_block_meta.argtypes = [DIMS, P, P, P, I32, I32, P, P, P, P, P, P]
+    L.eta_predict_tau.argtypes = [DIMS, P, P, P, P, P, P, P]
+    L.eta_screen_workspace_size.argtypes = [DIMS]
+    L.eta_screen_workspace_size.restype = C.c_size_t
+    L.eta_screen.argtypes = [DIMS, P, P, P, P, P, P, I32, F32, F32, P, P, P, P, P, P,
+                             C.c_size_t, P, P]
+    L.eta_decode_workspace_size.argtypes = [DIMS]
+    L.eta_decode_workspace_size.restype = C.c_size_t
+    L.eta_decode.argtypes = [DIMS, P, P, P, P, P, P, P, F32, F32, I32, P, P, P, P, P,
+                             C.c_size_t, P, P]
+    L.eta_dense_decode.argtypes = [DIMS, P, P, P, P, F32, P, P, P, C.c_size_t, P, P]
+    L.eta_calibrate_const_tau.argtypes = [P, P, I32, I32, I32, F32, P]
+    L.eta_status_from_device.argtypes = [I32]
+    L.eta_status_string.argtypes = [I32]
+    L.eta_status_string.restype = C.c_char_p
+    for name in ("eta_build_block_meta", "eta_predict_tau", "eta_screen", "eta_decode",
+                 "eta_dense_decode", "eta_calibrate_const_tau", "eta_status_from_device"):
+        getattr(L, name).restype = I32
+    _lib = L
+    return L
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> Optional[C.c_void_p]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, code: int):
+    if code != ETA_OK:
+        raise EtaError(fn, code)
+
+
+def eta_build_block_meta(dims: Dims, K, V, lengths, blk_begin, blk_end, cent, rmax, var, cnt,
+                         vsum=None, stream=None):
+    _check("eta_build_block_meta", lib().eta_build_block_meta(
+        C.byref(dims), _p(K), _p(V), _p(lengths), int(blk_begin), int(blk_end), _p(cent),
+        _p(rmax), _p(var), _p(cnt), _p(vsum), _stream(stream)))
+
+
+def eta_predict_tau(dims: Dims, q, W, bias, tau_const, tau, dev_status=None, stream=None):
+    _check("eta_predict_tau", lib().eta_predict_tau(
+        C.byref(dims), _p(q), _p(W), _p(bias), _p(tau_const), _p(tau), _p(dev_status),
+        _stream(stream)))
+
+
+def eta_screen_workspace_size(dims: Dims) -> int:
+    return int(lib().eta_screen_workspace_size(C.byref(dims)))
+
+
+def eta_screen(dims: Dims, q, tau, cent, rmax, var, cnt, bound, z, scale, head_mask,
+               union_idx, union_cnt, bounds_out, head_cnt, ws, dev_status=None, stream=None):
+    _check("eta_screen", lib().eta_screen(
+        C.byref(dims), _p(q), _p(tau), _p(cent), _p(rmax), _p(var), _p(cnt),
+        BOUND[bound] if isinstance(bound, str) else int(bound), float(z), float(scale),
+        _p(head_mask), _p(union_idx), _p(union_cnt), _p(bounds_out), _p(head_cnt), _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _p(dev_status), _stream(stream)))
+
+
+def eta_decode_workspace_size(dims: Dims) -> int:
+    return int(lib().eta_decode_workspace_size(C.byref(dims)))
+
+
+def eta_decode(dims: Dims, q, tau, K, V, lengths, union_idx, union_cnt, T, scale, prune,
+               vsum, cnt, o, lse, ws, dev_status=None, stream=None):
+    _check("eta_decode", lib().eta_decode(
+        C.byref(dims), _p(q), _p(tau), _p(K), _p(V), _p(lengths), _p(union_idx),
+        _p(union_cnt), float(T), float(scale),
+        PRUNE[prune] if isinstance(prune, str) else int(prune), _p(vsum), _p(cnt), _p(o),
+        _p(lse), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _p(dev_status),
+        _stream(stream)))
+
+
+def eta_dense_decode(dims: Dims, q, K, V, lengths, scale, o, lse, ws, dev_status=None,
+                     stream=None):
+    _check("eta_dense_decode", lib().eta_dense_decode(
+        C.byref(dims), _p(q), _p(K), _p(V), _p(lengths), float(scale), _p(o), _p(lse), _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _p(dev_status), _stream(stream)))
+
+
+def eta_calibrate_const_tau(bounds: torch.Tensor, valid: torch.Tensor, density: float):
+    """Host call: bounds fp32 [n_q, Hq, NB] and valid bool/uint8 of the same shape
+    (CPU tensors).  Returns tau fp32 [Hq] (CPU)."""
+    b = bounds.detach().to("cpu", torch.float32).contiguous()
+    v = valid.detach().to("cpu", torch.uint8).contiguous()
+    n_q, Hq, NB = b.shape
+    out = torch.empty(Hq, dtype=torch.float32)
+    _check("eta_calibrate_const_tau", lib().eta_calibrate_const_tau(
+        _p(b), _p(v), n_q, Hq, NB, float(density), _p(out)))
+    return out
+
+
+def eta_status_from_device(word: int) -> int:
+    return int(lib().eta_status_from_device(int(word)))
+
+
+def eta_status_string(code: int) -> str:
+    return lib().eta_status_string(int(code)).decode()

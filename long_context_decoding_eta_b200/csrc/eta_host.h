@@ -1,0 +1,48 @@
+// Host-side helpers shared by the C-ABI entry points: argument checks, device
+// properties, launch-error mapping.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/eta.h"
+
+namespace eta {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int num_blocks(const eta_dims_t* d) { return d->T_max / d->blk; }
+inline int num_words(const eta_dims_t* d) { return (num_blocks(d) + 31) / 32; }
+
+// Common shape validation.  Returns ETA_OK or the error to report.
+inline eta_status_t check_dims(const eta_dims_t* d) {
+  if (!d) return ETA_ERR_INVALID_ARG;
+  if (d->B <= 0 || d->Hq <= 0 || d->Hkv <= 0 || d->d <= 0 || d->blk <= 0 || d->T_max <= 0)
+    return ETA_ERR_INVALID_ARG;
+  if (d->Hq % d->Hkv != 0) return ETA_ERR_INVALID_ARG;
+  const int G = d->Hq / d->Hkv;
+  if (!(G == 1 || G == 2 || G == 4 || G == 8)) return ETA_ERR_UNSUPPORTED;
+  if (!(d->d == 64 || d->d == 128)) return ETA_ERR_UNSUPPORTED;
+  if (!(d->blk == 64 || d->blk == 128)) return ETA_ERR_UNSUPPORTED;
+  if (d->T_max % d->blk != 0) return ETA_ERR_UNSUPPORTED;
+  if ((int64_t)d->B * d->Hkv > 65535) return ETA_ERR_UNSUPPORTED;   // grid.y limit
+  if (num_blocks(d) > 65536) return ETA_ERR_UNSUPPORTED;
+  if (d->Hq > 256) return ETA_ERR_UNSUPPORTED;
+  return ETA_OK;
+}
+
+inline eta_status_t launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+inline int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace eta

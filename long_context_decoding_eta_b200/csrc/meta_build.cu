@@ -1,0 +1,152 @@
+// Per-KV-block metadata (centroid, max deviation radius, variance, count, V sum).
+//
+// "Cached centroid/variance/max-norm metadata" (evolve.pub review of arXiv
+// 2609.20888, Summary); "cached geometric-probabilistic bounds" (abstract).
+// One warp per block; every lane owns d/32 consecutive dimensions, so each key
+// row is one coalesced 128/256-byte warp load.  Blocks live in L2 between the two
+// passes over their keys (16-32 KB each).
+#include "eta_common.cuh"
+#include "eta_host.h"
+
+namespace eta {
+
+// 1 + 2^-20: covers the relative rounding error of the fp32 distance
+// computation below (<= ~6 ulp on the sqrt), so rmax never under-states the
+// true maximum distance to the stored fp32 centroid.
+constexpr float kRadiusInflate = 1.00000095367431640625f;
+constexpr int kMetaWarps = 8;
+
+template <int DPL>
+ETA_DEV void load_row(const eta_bf16_t* p, float (&x)[DPL]) {
+  if constexpr (DPL == 4) {
+    uint2 w = *reinterpret_cast<const uint2*>(p);
+    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+  } else {
+    uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+    x[0] = bf16_lo(w); x[1] = bf16_hi(w);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kMetaWarps * 32)
+meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restrict__ K,
+                  const eta_bf16_t* __restrict__ V, const int32_t* __restrict__ lengths,
+                  int blk_begin, int nblk, int tail, float* __restrict__ cent,
+                  float* __restrict__ rmax, float* __restrict__ var, int32_t* __restrict__ cnt,
+                  float* __restrict__ vsum, int32_t* status) {
+  constexpr int DPL = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y;                 // (row, KV head) = b * Hkv + g
+  const int b = r / Hkv;
+  int len = lengths[b];
+  if (len < 0 || len > T_max) {
+    if (lane == 0 && warp == 0 && blockIdx.x == 0) set_status(status, ETA_DEVSTAT_BAD_LENGTH);
+    len = min(max(len, 0), T_max);
+  }
+  int j;
+  if (tail) {
+    if (blockIdx.x != 0 || warp != 0 || len == 0) return;
+    j = (len - 1) / blk;
+  } else {
+    const int jj = blockIdx.x * kMetaWarps + warp;
+    if (jj >= nblk) return;
+    j = blk_begin + jj;
+  }
+  const int n = min(max(len - j * blk, 0), blk);
+  const size_t rowj = (size_t)r * NB + j;
+  const eta_bf16_t* kb = K + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
+
+  float c[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) c[i] = 0.f;
+  // pass 1: centroid (sequential fp32 sum over the keys, then one division)
+#pragma unroll 8
+  for (int t = 0; t < n; ++t) {
+    float x[DPL];
+    load_row<DPL>(kb + (size_t)t * D, x);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) c[i] += x[i];
+  }
+  if (n > 0) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) c[i] = c[i] / (float)n;
+  }
+  // pass 2: squared distances to the stored fp32 centroid
+  float r2max = 0.f, s2 = 0.f;
+#pragma unroll 4
+  for (int t = 0; t < n; ++t) {
+    float x[DPL];
+    load_row<DPL>(kb + (size_t)t * D, x);
+    float p = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const float dv = x[i] - c[i];
+      p = fmaf(dv, dv, p);
+    }
+    p = warp_sum(p);          // butterfly: bit-identical in every lane
+    r2max = fmaxf(r2max, p);
+    s2 += p;
+  }
+  float* cr = cent + (size_t)r * D * NB + j;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) cr[(size_t)(lane * DPL + i) * NB] = c[i];
+  if (lane == 0) {
+    rmax[rowj] = n > 0 ? __fmul_ru(__fsqrt_ru(r2max), kRadiusInflate) : 0.f;
+    var[rowj] = n > 0 ? s2 / (float)n : 0.f;
+    cnt[rowj] = n;
+  }
+  if (vsum) {
+    const eta_bf16_t* vb = V + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
+    float a[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) a[i] = 0.f;
+#pragma unroll 8
+    for (int t = 0; t < n; ++t) {
+      float x[DPL];
+      load_row<DPL>(vb + (size_t)t * D, x);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) a[i] += x[i];
+    }
+    float* vr = vsum + rowj * D + lane * DPL;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) vr[i] = a[i];
+  }
+}
+
+}  // namespace eta
+
+using namespace eta;
+
+extern "C" eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_bf16_t* K,
+                                             const eta_bf16_t* V, const int32_t* lengths,
+                                             int32_t blk_begin, int32_t blk_end, float* cent,
+                                             float* rmax, float* var, int32_t* cnt, float* vsum,
+                                             void* stream) {
+  eta_status_t st = check_dims(dims);
+  if (st != ETA_OK) return st;
+  if (!K || !lengths || !cent || !rmax || !var || !cnt) return ETA_ERR_INVALID_ARG;
+  if (vsum && !V) return ETA_ERR_INVALID_ARG;
+  if (!aligned16(K) || (V && !aligned16(V))) return ETA_ERR_INVALID_ARG;
+  const int NB = num_blocks(dims);
+  const int R = dims->B * dims->Hkv;
+  const bool tail = blk_begin == ETA_TAIL_BLOCK;
+  int nblk = 0;
+  if (!tail) {
+    if (blk_end < 0) blk_end = NB;
+    if (blk_begin < 0 || blk_begin > blk_end || blk_end > NB) return ETA_ERR_INVALID_ARG;
+    nblk = blk_end - blk_begin;
+    if (nblk == 0) return ETA_OK;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dim3 grid(tail ? 1 : (nblk + kMetaWarps - 1) / kMetaWarps, R);
+  dim3 block(tail ? 32 : kMetaWarps * 32);
+  if (dims->d == 128)
+    meta_build_kernel<128><<<grid, block, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB, K, V,
+                                                   lengths, blk_begin, nblk, tail, cent, rmax,
+                                                   var, cnt, vsum, nullptr);
+  else
+    meta_build_kernel<64><<<grid, block, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB, K, V,
+                                                  lengths, blk_begin, nblk, tail, cent, rmax,
+                                                  var, cnt, vsum, nullptr);
+  return launch_status();
+}

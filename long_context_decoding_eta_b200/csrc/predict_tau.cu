@@ -1,0 +1,84 @@
+// Threshold per (query, head): the linear predictor on the concatenated post-RoPE
+// query heads (evolve.pub review of arXiv 2609.20888, Methodology Assessment,
+// Eq. 1: tau = qbar W_tau + b_tau) or a frozen per-head constant (abstract: offline
+// calibration "freezes per-head constant thresholds").
+//
+// A GEMV per batch row: one CTA per row streams W (Hq*d x Hq fp32, 128 KB at
+// Hq = 16, d = 128; L2-resident across rows) with every thread owning rows of W,
+// then a fixed-order block reduction, so results are deterministic.
+#include "eta_common.cuh"
+#include "eta_host.h"
+
+namespace eta {
+
+constexpr int kTauThreads = 256;
+constexpr int kTauHeadsPerPass = 16;
+
+__global__ void __launch_bounds__(kTauThreads)
+predict_tau_kernel(int Hq, int D, const eta_bf16_t* __restrict__ q, const float* __restrict__ W,
+                   const float* __restrict__ bias, float* __restrict__ tau, int32_t* status) {
+  __shared__ float red[kTauThreads / 32][kTauHeadsPerPass];
+  const int b = blockIdx.x;
+  const int n = Hq * D;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const eta_bf16_t* qb = q + (size_t)b * n;
+  bool bad = false;
+  for (int h0 = 0; h0 < Hq; h0 += kTauHeadsPerPass) {
+    const int hc = min(kTauHeadsPerPass, Hq - h0);
+    float acc[kTauHeadsPerPass];
+#pragma unroll
+    for (int k = 0; k < kTauHeadsPerPass; ++k) acc[k] = 0.f;
+    for (int i = threadIdx.x; i < n; i += kTauThreads) {
+      const float x = bf16_to_f(qb[i]);
+      bad |= !isfinite(x);
+      const float* wr = W + (size_t)i * Hq + h0;
+#pragma unroll
+      for (int k = 0; k < kTauHeadsPerPass; ++k)
+        if (k < hc) acc[k] = fmaf(x, __ldg(wr + k), acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < kTauHeadsPerPass; ++k) {
+      const float v = warp_sum(acc[k]);
+      if (lane == 0) red[warp][k] = v;
+    }
+    __syncthreads();
+    if (threadIdx.x < hc) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < kTauThreads / 32; ++w) s += red[w][threadIdx.x];
+      const int h = h0 + threadIdx.x;
+      tau[(size_t)b * Hq + h] = s + (bias ? bias[h] : 0.f);
+    }
+    __syncthreads();
+  }
+  if (bad) set_status(status, ETA_DEVSTAT_NONFINITE_Q);
+}
+
+__global__ void const_tau_kernel(int total, int Hq, const float* __restrict__ tau_const,
+                                 float* __restrict__ tau) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < total) tau[i] = tau_const[i % Hq];
+}
+
+}  // namespace eta
+
+using namespace eta;
+
+extern "C" eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q,
+                                        const float* W, const float* bias,
+                                        const float* tau_const, float* tau, int32_t* dev_status,
+                                        void* stream) {
+  eta_status_t st = check_dims(dims);
+  if (st != ETA_OK) return st;
+  if (!tau) return ETA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (tau_const) {
+    const int total = dims->B * dims->Hq;
+    const_tau_kernel<<<(total + 255) / 256, 256, 0, s>>>(total, dims->Hq, tau_const, tau);
+    return launch_status();
+  }
+  if (!q || !W) return ETA_ERR_INVALID_ARG;
+  predict_tau_kernel<<<dims->B, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau,
+                                                      dev_status);
+  return launch_status();
+}

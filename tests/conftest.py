@@ -20,3 +20,11 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """Builds libeta.so in-tree once per session (nvcc cross-compiles without a GPU)."""
+    from long_context_decoding_eta_b200 import build
+    build.build()
+    yield

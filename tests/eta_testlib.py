@@ -1,0 +1,168 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI,
+run the float64 oracle on the same seeded inputs, and compare with the stated
+tolerances (admit masks bit-exact except near-ties; o max-abs 1e-2 and
+mean-abs 1e-3; lse abs 1e-3)."""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+import torch
+
+from oracle import eta_oracle as O
+
+NEAR_TIE_REL = 1e-5        # |UB - tau| <= 1e-5 * max(1, |tau|) may disagree
+O_MAX_ABS = 1e-2
+O_MEAN_ABS = 1e-3
+LSE_ABS = 1e-3
+
+
+def f64(t):
+    return t.detach().to("cpu").double().numpy()
+
+
+def unpack_mask(words: torch.Tensor, NB: int) -> np.ndarray:
+    """uint32 words [..., NW] (stored as int32) -> bool [..., NB]."""
+    w = words.detach().cpu().numpy().astype(np.int64) & 0xFFFFFFFF
+    bits = (w[..., :, None] >> np.arange(32)) & 1
+    return bits.reshape(*w.shape[:-1], -1)[..., :NB].astype(bool)
+
+
+def run_cuda(dec, q, W=None, bias=None, tau_const=None, tau=None) -> Dict[str, np.ndarray]:
+    """Full CUDA path on an EtaDecoder whose metadata is built: tau, screen, decode."""
+    if tau is None:
+        dec.predict_tau(q, W, bias, tau_const)
+    else:
+        dec.tau.copy_(tau)
+    dec.screen(q)
+    dec.decode(q)
+    torch.cuda.synchronize()
+    dec.check_status()
+    out = dict(tau=f64(dec.tau), head_mask=unpack_mask(dec.head_mask, dec.NB),
+               union_idx=dec.union_idx.cpu().numpy(), union_cnt=dec.union_cnt.cpu().numpy(),
+               head_cnt=dec.head_cnt.cpu().numpy(), o=f64(dec.o), lse=f64(dec.lse))
+    if dec.bounds is not None:
+        out["bounds"] = f64(dec.bounds)
+    return out
+
+
+def gpu_meta(dec) -> Dict[str, np.ndarray]:
+    m = dict(cent=f64(dec.cent.transpose(2, 3)), rmax=f64(dec.rmax), var=f64(dec.var),
+             cnt=dec.cnt.cpu().numpy().astype(np.int64))
+    if dec.vsum is not None:
+        m["vsum"] = f64(dec.vsum)
+    return m
+
+
+def check_meta(gm: Dict[str, np.ndarray], om: Dict[str, np.ndarray], rows=None):
+    sel = (lambda a: a) if rows is None else (lambda a: a[rows])
+    assert np.array_equal(sel(gm["cnt"]), om["cnt"])
+    np.testing.assert_allclose(sel(gm["cent"]), om["cent"], rtol=0, atol=2e-6)
+    g_r, o_r = sel(gm["rmax"]), om["rmax"]
+    # sound (never below the true radius, beyond fp32 centroid rounding) and tight
+    assert np.all(g_r >= o_r * (1 - 1e-6) - 1e-6), float((o_r - g_r).max())
+    assert np.all(g_r <= o_r * (1 + 1e-5) + 1e-6), float((g_r - o_r).max())
+    np.testing.assert_allclose(sel(gm["var"]), om["var"], rtol=2e-5, atol=1e-6)
+    if "vsum" in gm and "vsum" in om:
+        np.testing.assert_allclose(sel(gm["vsum"]), om["vsum"], rtol=0, atol=2e-4)
+
+
+@dataclass
+class ParityReport:
+    n_blocks: int = 0
+    mask_mismatch: int = 0
+    near_ties: int = 0
+    groups_skipped: List = field(default_factory=list)
+    heads_compared: int = 0
+    o_max_abs: float = 0.0
+    o_mean_abs: float = 0.0
+    lse_max_abs: float = 0.0
+
+
+def compare_step(gpu: Dict[str, np.ndarray], ref_tau: np.ndarray, ref_sc, ref_o, ref_lse,
+                 q64, K64, V64, L, blk: int, scale: float, T: float, G: int,
+                 rows: Optional[Sequence[int]] = None, tau_atol: float = 2e-5) -> ParityReport:
+    """Compares the CUDA step with the oracle step on the rows `rows` of the batch
+    (all rows if None; the oracle arrays hold only those rows)."""
+    rows = list(range(gpu["o"].shape[0])) if rows is None else list(rows)
+    rep = ParityReport()
+    np.testing.assert_allclose(gpu["tau"][rows], ref_tau, rtol=0, atol=tau_atol)
+    ub, tau = ref_sc["bounds"], ref_tau
+    gmask = gpu["head_mask"][rows]
+    omask = ref_sc["admit"]
+    near = np.abs(ub - tau[:, :, None]) <= NEAR_TIE_REL * np.maximum(1.0, np.abs(tau))[:, :, None]
+    mism = gmask != omask
+    rep.n_blocks = int(omask.size)
+    rep.mask_mismatch = int(mism.sum())
+    rep.near_ties = int((mism & near).sum())
+    assert not np.any(mism & ~near), f"{int((mism & ~near).sum())} admit bits differ off near-ties"
+    B, Hq, NB = omask.shape
+    Hkv = Hq // G
+    # GPU union list must be the ascending OR of its own head masks, exactly
+    gunion = gmask.reshape(B, Hkv, G, NB).any(axis=2)
+    for bi, b in enumerate(rows):
+        for g in range(Hkv):
+            want = np.nonzero(gunion[bi, g])[0]
+            c = int(gpu["union_cnt"][b, g])
+            assert c == want.size
+            assert np.array_equal(gpu["union_idx"][b, g, :c], want)
+    assert np.array_equal(gpu["head_cnt"][rows], gmask.sum(axis=2))
+    # outputs: compare heads whose group union agrees and whose gate has no near-tie
+    errs = []
+    lerr = []
+    for bi, b in enumerate(rows):
+        for h in range(Hq):
+            g = h // G
+            if not np.array_equal(gunion[bi, g], ref_sc["union"][bi, g]):
+                rep.groups_skipped.append((b, h, "union near-tie"))
+                continue
+            if T == 0.0:
+                idx = O.block_keys(ref_sc["union_idx"][bi][g], int(L[bi]), blk)
+                s = scale * (K64[bi, g][idx] @ q64[bi, h])
+                if np.any(np.abs(s - tau[bi, h]) <= NEAR_TIE_REL * max(1.0, abs(tau[bi, h]))):
+                    rep.groups_skipped.append((b, h, "gate near-tie"))
+                    continue
+            e = np.abs(gpu["o"][b, h] - ref_o[bi, h])
+            errs.append(e)
+            gl, rl = gpu["lse"][b, h], ref_lse[bi, h]
+            if math.isinf(rl):
+                assert math.isinf(gl) and gl < 0
+                lerr.append(0.0)
+            else:
+                lerr.append(abs(gl - rl))
+            rep.heads_compared += 1
+    if errs:
+        e = np.stack(errs)
+        rep.o_max_abs = float(e.max())
+        rep.o_mean_abs = float(e.mean())
+        rep.lse_max_abs = float(max(lerr))
+    assert rep.heads_compared > 0
+    assert rep.o_max_abs <= O_MAX_ABS, rep
+    assert rep.o_mean_abs <= O_MEAN_ABS, rep
+    assert rep.lse_max_abs <= LSE_ABS, rep
+    return rep
+
+
+def oracle_step(K64, V64, q64, L, W64, bias, blk, scale, T, bound="exact", z=3.0,
+                prune="skip", tau_const=None):
+    meta = O.cache_meta(K64, L, blk, V64 if prune == "floor" else None)
+    if tau_const is None:
+        tau = O.predict_tau(q64, W64, bias)
+    else:
+        tau = O.const_tau(q64.shape[0], tau_const)
+    sc = O.screen(q64, tau, meta, scale, bound, z)
+    o, lse = O.decode(q64, tau, K64, V64, L, sc["union_idx"], blk, scale, T, prune, meta)
+    return meta, tau, sc, o, lse
+
+
+def density_bias(K64, q64, L, W64, blk, scale, G, density, kind, bound="exact", z=3.0):
+    """Per-head bias that makes the predictor hit a density target on the given
+    rows (oracle arithmetic only): bias_h = offset such that tau = qW + bias admits
+    the target fraction of (head, block) or (group, block) pairs."""
+    meta = O.cache_meta(K64, L, blk)
+    tau0 = O.predict_tau(q64, W64, np.zeros(q64.shape[1]))
+    ub = O.screen(q64, tau0, meta, scale, bound, z)["bounds"]
+    valid = np.repeat(meta["cnt"] > 0, G, axis=1)
+    return O.offset_for_density(ub, tau0, valid, density, G, kind)

@@ -1,0 +1,82 @@
+"""The C-ABI library loads and exports every entry point include/eta.h declares;
+host-only entry points (calibration, status helpers, argument validation) work
+without a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_decoding_eta_b200 import _lib as L
+from oracle import eta_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "eta.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(eta_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = L.lib()
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L.EXPORTS)
+
+
+def test_header_declares_the_four_method_calls():
+    names = declared_functions()
+    for n in ("eta_build_block_meta", "eta_predict_tau", "eta_screen", "eta_decode"):
+        assert n in names
+
+
+def test_status_strings():
+    assert L.eta_status_string(0) == "ok"
+    assert L.eta_status_string(3).startswith("workspace")
+    assert L.eta_status_from_device(0) == 0
+    assert L.eta_status_from_device(L.DEVSTAT_TIMEOUT) == 5
+    assert L.eta_status_from_device(L.DEVSTAT_NONFINITE_Q) == 6
+    assert L.eta_status_from_device(L.DEVSTAT_BAD_BLOCK) == 1
+
+
+@pytest.mark.parametrize("density", [0.16, 0.38, 0.51, 1.0])
+def test_host_calibration_matches_oracle_quantile(density):
+    rng = np.random.default_rng(0)
+    bounds = rng.normal(size=(64, 4, 50)).astype(np.float32)
+    valid = rng.random((64, 4, 50)) > 0.05
+    tau = L.eta_calibrate_const_tau(torch.from_numpy(bounds), torch.from_numpy(valid), density)
+    ref = O.calibrate_const_tau(bounds.astype(np.float64), valid, density)
+    np.testing.assert_array_equal(tau.numpy().astype(np.float64), ref)
+
+
+def test_calibration_rejects_empty_head():
+    b = torch.zeros(2, 2, 3)
+    v = torch.zeros(2, 2, 3, dtype=torch.bool)
+    v[:, 0] = True
+    with pytest.raises(L.EtaError):
+        L.eta_calibrate_const_tau(b, v, 0.5)
+
+
+def test_argument_validation_without_gpu():
+    lib = L.lib()
+    dims = L.Dims.of(2, 16, 4, 128, 64, 4096)
+    # null q -> invalid argument, nothing launched
+    r = lib.eta_decode(ctypes.byref(dims), None, None, None, None, None, None, None, 0.0, 0.0,
+                       0, None, None, None, None, None, 0, None, None)
+    assert r == 1
+    bad = L.Dims.of(2, 16, 4, 96, 64, 4096)            # d = 96 unsupported
+    r = lib.eta_screen(ctypes.byref(bad), *([None] * 6), 0, 0.0, 0.0, *([None] * 6), 0, None,
+                       None)
+    assert r == 2
+    odd = L.Dims.of(2, 16, 4, 128, 64, 4000)           # T_max not a multiple of blk
+    assert lib.eta_build_block_meta(ctypes.byref(odd), *([None] * 3), 0, -1, *([None] * 6)) == 2
+    g3 = L.Dims.of(2, 12, 4, 128, 64, 4096)            # G = 3 unsupported
+    assert lib.eta_predict_tau(ctypes.byref(g3), *([None] * 7)) == 2
+    assert L.eta_screen_workspace_size(dims) == 256       # 2*4 rows x 2 words, 256-aligned
+    assert L.eta_screen_workspace_size(bad) == 0

@@ -1,0 +1,216 @@
+"""CUDA path (through the C ABI) against the float64 oracle on the same seeded
+inputs.  Masks bit-exact except logged near-ties; o within max-abs 1e-2 and
+mean-abs 1e-3; lse within 1e-3."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_decoding_eta_b200 import synth
+from long_context_decoding_eta_b200._lib import EtaError
+from long_context_decoding_eta_b200.api import EtaDecoder
+from oracle import eta_oracle as O
+
+from eta_testlib import (check_meta, compare_step, density_bias, f64, gpu_meta, oracle_step,
+                         run_cuda, unpack_mask)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def make(w, lengths=None, seed=None):
+    g = synth.generate(w, "cpu", seed=seed, lengths=lengths)
+    return g
+
+
+def to_dev(g):
+    return {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in g.items()}
+
+
+def full_parity(w, *, lengths=None, prune="skip", T=None, bound=None, z=None, density=None,
+                kind=None, seed=None, tau_const=None):
+    T = w.gate_T if T is None else T
+    bound = w.bound if bound is None else bound
+    z = w.z if z is None else z
+    density = w.density if density is None else density
+    kind = w.density_kind if kind is None else kind
+    g = make(w, lengths, seed)
+    K64, V64, q64, W64 = f64(g["K"]), f64(g["V"]), f64(g["q"]), f64(g["W"])
+    L = g["lengths"].numpy().astype(np.int64)
+    scale = 1.0 / math.sqrt(w.d)
+    bias = np.full(w.Hq, density_bias(K64, q64, L, W64, w.blk, scale, w.G, density, kind,
+                                      bound, z))
+    gd = to_dev(g)
+    dec = EtaDecoder(gd["K"], gd["V"], gd["lengths"], w.Hq, w.blk, bound=bound, z=z, T=T,
+                     prune=prune, keep_bounds=True)
+    dec.build_meta()
+    bias_t = torch.tensor(bias, dtype=torch.float32, device=DEV)
+    tc = None if tau_const is None else torch.tensor(tau_const, dtype=torch.float32, device=DEV)
+    gpu = run_cuda(dec, gd["q"], gd["W"], bias_t, tc)
+    meta, tau, sc, o, lse = oracle_step(K64, V64, q64, L, W64, bias, w.blk, scale, T, bound, z,
+                                        prune, tau_const)
+    check_meta(gpu_meta(dec), meta)
+    rep = compare_step(gpu, tau, sc, o, lse, q64, K64, V64, L, w.blk, scale, T, w.G)
+    return rep, gpu, sc
+
+
+def test_tiny_workload_end_to_end():
+    rep, gpu, sc = full_parity(synth.TINY)
+    dens = sc["admit"].mean()
+    assert 0.3 < dens < 0.46, dens
+    print(rep)
+
+
+def test_mid_workload_needles_soft_gate():
+    rep, gpu, sc = full_parity(synth.MID)
+    print(rep)
+
+
+@pytest.mark.parametrize("T", [0.0, 0.05])
+@pytest.mark.parametrize("prune", ["skip", "floor"])
+def test_sharp_variant_keys_above_tau(T, prune):
+    w = synth.MID.with_(B=4, ctx=8192, q_scale=8.0, needles=16, density=0.3,
+                        density_kind="head", seed=77)
+    rep, gpu, sc = full_parity(w, T=T, prune=prune)
+    print(rep)
+
+
+def test_ragged_lengths_empty_and_single_token_rows():
+    w = synth.MID.with_(B=6, ctx=4096, needles=0, seed=78)
+    lengths = torch.tensor([4096, 0, 1, 4031, 65, 2000], dtype=torch.int32)
+    for prune in ("skip", "floor"):
+        rep, gpu, sc = full_parity(w, lengths=lengths, prune=prune, T=0.0, density=0.5)
+        # the empty row: SKIP gives o = 0, lse = -inf; FLOOR too (no keys at all)
+        assert np.all(gpu["o"][1] == 0) and np.all(np.isneginf(gpu["lse"][1]))
+
+
+@pytest.mark.parametrize("d,G,blk", [(64, 1, 64), (64, 8, 128), (128, 2, 128), (128, 8, 64),
+                                     (128, 4, 128)])
+def test_shapes(d, G, blk):
+    w = synth.Workload("shape", B=3, Hq=2 * G, Hkv=2, d=d, ctx=3000, blk=blk, n_clusters=16,
+                       seg=200, needles=2, gate_T=0.0, density=0.4, density_kind="head",
+                       seed=100 + d + G + blk)
+    lengths = torch.tensor([3000, 2777, 1234], dtype=torch.int32)
+    rep, gpu, sc = full_parity(w, lengths=lengths)
+
+
+def test_probabilistic_bound_blk128():
+    w = synth.EXTREME512K.with_(B=2, ctx=16384, seed=79)
+    rep, gpu, sc = full_parity(w, bound="prob", z=3.0)
+    rep2, gpu2, sc2 = full_parity(w, bound="exact")
+    # same inputs, same metadata: the probabilistic bound is never looser
+    assert np.all(gpu["bounds"] <= gpu2["bounds"] + 1e-6)
+
+
+def test_const_tau_mode():
+    w = synth.MID.with_(B=2, ctx=8192, seed=80)
+    rep, gpu, sc = full_parity(w, tau_const=np.linspace(1.6, 2.2, w.Hq))
+    assert np.allclose(gpu["tau"], np.linspace(1.6, 2.2, w.Hq)[None, :], atol=1e-6)
+
+
+def test_tau_neg_inf_is_dense_attention_and_dense_kernel():
+    w = synth.MID.with_(B=3, ctx=5000, needles=0, seed=81)
+    g = to_dev(make(w, lengths=torch.tensor([5000, 4097, 64], dtype=torch.int32)))
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, T=0.0)
+    dec.build_meta()
+    tau = torch.full((w.B, w.Hq), -math.inf, device=DEV)
+    gpu = run_cuda(dec, g["q"], tau=tau)
+    o_d, lse_d = [t.clone() for t in dec.dense_decode(g["q"])]
+    torch.cuda.synchronize()
+    dec.check_status()
+    K64, V64, q64 = f64(g["K"]), f64(g["V"]), f64(g["q"])
+    L = g["lengths"].cpu().numpy()
+    o_ref, lse_ref = O.dense_decode(q64, K64, V64, L, 1.0 / math.sqrt(w.d))
+    for o, lse in ((gpu["o"], gpu["lse"]), (f64(o_d), f64(lse_d))):
+        err = np.abs(o - o_ref)
+        assert err.max() <= 1e-2 and err.mean() <= 1e-3
+        assert np.abs(lse - lse_ref).max() <= 1e-3
+    np.testing.assert_allclose(gpu["o"], f64(o_d), atol=1e-5)
+
+
+def test_tau_above_every_score_gives_uniform_mean():
+    w = synth.MID.with_(B=2, ctx=4096, needles=0, seed=82)
+    g = to_dev(make(w))
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, T=0.0, prune="floor")
+    dec.build_meta()
+    tau = torch.full((w.B, w.Hq), 1e3, device=DEV)   # above every bound too: all pruned
+    gpu = run_cuda(dec, g["q"], tau=tau)
+    assert gpu["union_cnt"].sum() == 0
+    V64 = f64(g["V"])
+    for b in range(w.B):
+        for h in range(w.Hq):
+            np.testing.assert_allclose(gpu["o"][b, h], V64[b, h // w.G, :4096].mean(0),
+                                       atol=1e-5)
+            assert abs(gpu["lse"][b, h] - math.log(4096)) < 1e-5
+
+
+def test_tail_append_update_matches_rebuild():
+    w = synth.MID.with_(B=3, ctx=4096, needles=0, seed=83)
+    lengths = torch.tensor([4000, 4095, 100], dtype=torch.int32)
+    g = to_dev(make(w, lengths=lengths))
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, prune="floor")
+    dec.build_meta()
+    # append one token per row and update only the tail blocks
+    for b in range(w.B):
+        t = int(dec.lengths[b])
+        dec.K[b, :, t] = torch.randn(w.Hkv, w.d, device=DEV).to(torch.bfloat16)
+        dec.V[b, :, t] = torch.randn(w.Hkv, w.d, device=DEV).to(torch.bfloat16)
+    dec.lengths += 1
+    dec.append_update()
+    inc = {k: v.clone() for k, v in gpu_meta(dec).items()}
+    dec.build_meta()
+    full = gpu_meta(dec)
+    for k in full:
+        assert np.array_equal(inc[k], full[k]), k
+    o_meta = O.cache_meta(f64(dec.K), dec.lengths.cpu().numpy(), w.blk, f64(dec.V))
+    check_meta(full, o_meta)
+
+
+def test_status_nonfinite_query_and_bad_arguments():
+    w = synth.TINY.with_(seed=84)
+    g = to_dev(make(w))
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk)
+    dec.build_meta()
+    q = g["q"].clone()
+    q[0, 1, 3] = float("nan")
+    dec.predict_tau(q, g["W"], None, None)
+    torch.cuda.synchronize()
+    with pytest.raises(EtaError):
+        dec.check_status()
+    # host-side validation: workspace too small, null pointer
+    from long_context_decoding_eta_b200 import _lib as L
+    small = torch.empty(16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(EtaError) as ei:
+        L.eta_decode(dec.dims, g["q"], dec.tau, dec.K, dec.V, dec.lengths, dec.union_idx,
+                     dec.union_cnt, 0.0, 0.0, "skip", None, None, dec.o, dec.lse, small)
+    assert ei.value.code == 3
+    with pytest.raises(EtaError) as ei:
+        L.eta_decode(dec.dims, None, dec.tau, dec.K, dec.V, dec.lengths, dec.union_idx,
+                     dec.union_cnt, 0.0, 0.0, "skip", None, None, dec.o, dec.lse, dec.ws_decode)
+    assert ei.value.code == 1
+
+
+def test_calibration_matches_oracle_rule():
+    w = synth.MID.with_(B=4, ctx=8192, needles=0, seed=85)
+    g = make(w)
+    gd = to_dev(g)
+    dec = EtaDecoder(gd["K"], gd["V"], gd["lengths"], w.Hq, w.blk, keep_bounds=True)
+    dec.build_meta()
+    qc = synth.calibration_queries(w, g["mu"], n=16)
+    tau_gpu = dec.calibrate_const_tau(qc, 0.38).numpy()
+    # oracle: bounds of the same calibration queries on oracle metadata
+    K64 = f64(g["K"])
+    L = g["lengths"].numpy()
+    meta = O.cache_meta(K64, L, w.blk)
+    q64 = f64(qc)
+    rows = np.arange(16) % w.B
+    scale = 1.0 / math.sqrt(w.d)
+    bounds = np.zeros((16, w.Hq, w.NB))
+    valid = np.zeros((16, w.Hq, w.NB), dtype=bool)
+    for i in range(16):
+        mrow = {k: v[rows[i]:rows[i] + 1] for k, v in meta.items()}
+        bounds[i] = O.screen(q64[i:i + 1], np.zeros((1, w.Hq)), mrow, scale)["bounds"][0]
+        valid[i] = np.repeat(meta["cnt"][rows[i]] > 0, w.G, axis=0)
+    tau_ref = O.calibrate_const_tau(bounds, valid, 0.38)
+    np.testing.assert_allclose(tau_gpu, tau_ref, rtol=0, atol=2e-5)

@@ -49,10 +49,10 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def workload_by_name(name: str) -> synth.Workload:
+def workload_by_name(name: str, B: int = 0) -> synth.Workload:
     for w in synth.WORKLOADS.values():
         if w.name == name or w.name.startswith(name):
-            return w
+            return w.with_(B=B, name=w.name.replace(f"b{w.B}-", f"b{B}-", 1)) if B else w
     raise SystemExit(f"unknown workload {name}; choose from {list(synth.WORKLOADS)}")
 
 
@@ -175,7 +175,7 @@ def step_bytes(dec, w):
 
 
 def run_eta(args, rank, world, device):
-    w = workload_by_name(args.workload)
+    w = workload_by_name(args.workload, args.B)
     g, dec, W, bias, tau_const = setup(w, device, rank)
     q = g["q"]
     stream = torch.cuda.current_stream()
@@ -204,6 +204,15 @@ def run_eta(args, rank, world, device):
            for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with Clocks(device.index if device.index is not None else 0) as clk:
+        # keep the same load running for at least ~1 s so the 100 ms clock
+        # sampler sees the GPU under this step, then time exactly `steps` steps
+        t_soak = time.perf_counter()
+        while time.perf_counter() - t_soak < args.clock_soak_s:
+            for _ in range(8):
+                one_step()
+            torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(args.steps):
@@ -360,7 +369,7 @@ def run_reference(args, rank, world, device):
     The threshold bias is set by the oracle itself on the sampled rows, with the
     same density rule as the eta arm; no CUDA kernel of this package runs."""
     from oracle import eta_oracle as O
-    w = workload_by_name(args.workload)
+    w = workload_by_name(args.workload, args.B)
     g = synth.generate(w, device, seed=w.seed)
     rows = list(range(args.cpu_rows))
     K64 = g["K"][rows].double().cpu().numpy()
@@ -424,6 +433,9 @@ def main():
     ap.add_argument("--impl", default="eta", choices=["eta", "reference"])
     ap.add_argument("--cpu-rows", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-soak-s", type=float, default=1.0,
+                    help="untimed steps run under the clock sampler before the timed region")
+    ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -158,7 +158,7 @@ def test_tail_append_update_matches_rebuild():
         dec.V[b, :, t] = torch.randn(w.Hkv, w.d, device=DEV).to(torch.bfloat16)
     dec.lengths += 1
     dec.append_update()
-    inc = {k: v.clone() for k, v in gpu_meta(dec).items()}
+    inc = {k: v.copy() for k, v in gpu_meta(dec).items()}
     dec.build_meta()
     full = gpu_meta(dec)
     for k in full:

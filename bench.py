@@ -175,6 +175,8 @@ def step_bytes(dec, w):
 
 
 def run_eta(args, rank, world, device):
+    from long_context_decoding_eta_b200 import _lib
+    _lib.eta_set_decode_engine(args.engine)
     w = workload_by_name(args.workload, args.B)
     g, dec, W, bias, tau_const = setup(w, device, rank)
     q = g["q"]
@@ -288,7 +290,7 @@ def run_eta(args, rank, world, device):
         "config": {
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
             "context": w.ctx, "blk": w.blk, "bound": w.bound, "gate_T": w.gate_T,
-            "tau_mode": w.tau_mode,
+            "tau_mode": w.tau_mode, "engine": args.engine,
             "density_target": f"{w.density:.2f} {w.density_kind}",
             "union_density": round(by["union_density"], 4),
             "head_density": round(by["head_density"], 4),
@@ -436,6 +438,8 @@ def main():
     ap.add_argument("--clock-soak-s", type=float, default=1.0,
                     help="untimed steps run under the clock sampler before the timed region")
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
+    ap.add_argument("--engine", default="auto", choices=["auto", "tcgen05", "fma"],
+                    help="decode engine of libeta.so")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

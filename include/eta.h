@@ -184,6 +184,20 @@ eta_status_t eta_dense_decode(const eta_dims_t* dims, const eta_bf16_t* q,
                               void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * Decode engine (process-wide; both compute the same function, both are tested
+ * against the float64 oracle):
+ *   ETA_ENGINE_TCGEN05 -- q.k and p.v on the tensor cores (tcgen05.mma, TMEM
+ *                         accumulators, TMA tensor copies with 128-byte swizzle);
+ *                         d = 128 only (other d fall back to the FMA engine)
+ *   ETA_ENGINE_FMA     -- q.k and p.v on the CUDA cores in fp32 (1-D TMA bulk copies)
+ *   ETA_ENGINE_AUTO    -- the default: the engine this library measures fastest
+ * eta_set_decode_engine returns ETA_ERR_INVALID_ARG for an unknown value.
+ */
+typedef enum { ETA_ENGINE_AUTO = 0, ETA_ENGINE_TCGEN05 = 1, ETA_ENGINE_FMA = 2 } eta_engine_t;
+eta_status_t eta_set_decode_engine(eta_engine_t engine);
+eta_engine_t eta_get_decode_engine(void);
+
+/*
  * eta_calibrate_const_tau -- offline calibration of frozen per-head thresholds
  * (abstract: "an offline calibration algorithm ... that freezes per-head constant
  * thresholds").  HOST pointers.  The pages do not print the algorithm; the rule

@@ -27,7 +27,9 @@ DEVSTAT_TIMEOUT, DEVSTAT_NONFINITE_Q, DEVSTAT_BAD_BLOCK, DEVSTAT_BAD_LENGTH = 1,
 
 EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size",
            "eta_screen", "eta_decode_workspace_size", "eta_decode", "eta_dense_decode",
-           "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string")
+           "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string",
+           "eta_set_decode_engine", "eta_get_decode_engine")
+ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 
 
 class EtaError(RuntimeError):
@@ -80,6 +82,10 @@ def lib() -> C.CDLL:
     L.eta_status_from_device.argtypes = [I32]
     L.eta_status_string.argtypes = [I32]
     L.eta_status_string.restype = C.c_char_p
+    L.eta_set_decode_engine.argtypes = [I32]
+    L.eta_set_decode_engine.restype = I32
+    L.eta_get_decode_engine.argtypes = []
+    L.eta_get_decode_engine.restype = I32
     for name in ("eta_build_block_meta", "eta_predict_tau", "eta_screen", "eta_decode",
                  "eta_dense_decode", "eta_calibrate_const_tau", "eta_status_from_device"):
         getattr(L, name).restype = I32
@@ -167,3 +173,14 @@ def eta_status_from_device(word: int) -> int:
 
 def eta_status_string(code: int) -> str:
     return lib().eta_status_string(int(code)).decode()
+
+
+def eta_set_decode_engine(engine) -> None:
+    """engine: "auto" | "tcgen05" | "fma" (or the integer value)."""
+    _check("eta_set_decode_engine", lib().eta_set_decode_engine(
+        ENGINE[engine] if isinstance(engine, str) else int(engine)))
+
+
+def eta_get_decode_engine() -> str:
+    v = int(lib().eta_get_decode_engine())
+    return {k: n for n, k in ENGINE.items()}.get(v, str(v))

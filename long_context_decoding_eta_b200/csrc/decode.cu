@@ -18,8 +18,12 @@
 //                  and write one partial (m, l, o) slot.
 //   combine_kernel log-sum-exp merge of the partial slots of each (row, head), plus the
 //                  floor term of pruned blocks in FLOOR mode.
+#include <cudaTypedefs.h>
 #include <math.h>
 
+#include <atomic>
+
+#include "decode_tc.cuh"
 #include "eta_common.cuh"
 #include "eta_host.h"
 
@@ -547,6 +551,81 @@ inline eta_status_t launch_combine(const eta_dims_t* dims, const CombineParams& 
   return ETA_ERR_UNSUPPORTED;
 }
 
+// ---------------------------------------------------------------- tcgen05 engine host side
+std::atomic<int> g_engine{ETA_ENGINE_AUTO};
+
+inline bool use_tc(const eta_dims_t* d) {
+  const int e = g_engine.load();
+  if (e == ETA_ENGINE_FMA) return false;
+  // TMA row coordinates are 32-bit
+  const bool fits = (uint64_t)d->B * d->Hkv * d->T_max < (1ull << 31);
+  // AUTO and TCGEN05: the tensor-core engine wherever it applies (measured ~1.6x the
+  // FMA engine's bandwidth on the 128K / B = 64 workload)
+  return d->d == 128 && fits;
+}
+
+using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+inline EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D view [rows, 128] of a bf16 tensor, box 64 columns x box_rows rows, 128-byte swizzle.
+inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {128, rows};
+  cuuint64_t gstride[1] = {128 * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int G, bool DENSE>
+eta_status_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq,
+                         const tc::TcParams& prm, int P, cudaStream_t s) {
+  auto kern = tc::decode_tc_kernel<G, DENSE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES) !=
+      cudaSuccess)
+    return ETA_ERR_CUDA;
+  kern<<<P, tc::NT, tc::SMEM_BYTES, s>>>(mk, mv, mq, prm);
+  return launch_status();
+}
+
+template <bool DENSE>
+eta_status_t launch_tc(const eta_dims_t* dims, const DecodeParams& d, const eta_bf16_t* q,
+                       const eta_bf16_t* K, const eta_bf16_t* V, int P, cudaStream_t s) {
+  CUtensorMap mk, mv, mq;
+  const uint64_t kv_rows = (uint64_t)dims->B * dims->Hkv * dims->T_max;
+  if (!make_map(&mk, K, kv_rows, 64) || !make_map(&mv, V, kv_rows, 64) ||
+      !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16))
+    return ETA_ERR_CUDA;
+  tc::TcParams prm;
+  prm.Hq = d.Hq; prm.Hkv = d.Hkv; prm.T_max = d.T_max; prm.NB = d.NB; prm.blk = d.blk;
+  prm.scale = d.scale; prm.invT = d.invT; prm.tau = d.tau; prm.lengths = d.lengths;
+  prm.union_idx = d.union_idx; prm.row_off = d.row_off; prm.cta_row = d.cta_row;
+  prm.plan = d.plan; prm.part_o = d.part_o; prm.part_ml = d.part_ml; prm.status = d.status;
+  switch (dims->Hq / dims->Hkv) {
+    case 1: return launch_tc_t<1, DENSE>(mk, mv, mq, prm, P, s);
+    case 2: return launch_tc_t<2, DENSE>(mk, mv, mq, prm, P, s);
+    case 4: return launch_tc_t<4, DENSE>(mk, mv, mq, prm, P, s);
+    case 8: return launch_tc_t<8, DENSE>(mk, mv, mq, prm, P, s);
+  }
+  return ETA_ERR_UNSUPPORTED;
+}
+
 template <bool DENSE>
 eta_status_t run_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                         const eta_bf16_t* K, const eta_bf16_t* V, const int32_t* lengths,
@@ -590,7 +669,9 @@ eta_status_t run_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float
   prm.q = q; prm.tau = tau; prm.K = K; prm.V = V; prm.lengths = lengths;
   prm.union_idx = union_idx; prm.row_off = row_off; prm.cta_row = cta_row; prm.plan = plan;
   prm.part_o = part_o; prm.part_ml = part_ml; prm.status = dev_status;
-  if ((st = launch_decode<DENSE>(dims, prm, P, s)) != ETA_OK) return st;
+  st = use_tc(dims) ? launch_tc<DENSE>(dims, prm, q, K, V, P, s)
+                    : launch_decode<DENSE>(dims, prm, P, s);
+  if (st != ETA_OK) return st;
 
   CombineParams cp;
   cp.Hq = dims->Hq; cp.Hkv = dims->Hkv; cp.NB = NB; cp.blk = dims->blk; cp.T_max = dims->T_max;
@@ -603,6 +684,17 @@ eta_status_t run_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float
 }  // namespace eta
 
 using namespace eta;
+
+extern "C" eta_status_t eta_set_decode_engine(eta_engine_t engine) {
+  if (engine != ETA_ENGINE_AUTO && engine != ETA_ENGINE_TCGEN05 && engine != ETA_ENGINE_FMA)
+    return ETA_ERR_INVALID_ARG;
+  g_engine.store((int)engine);
+  return ETA_OK;
+}
+
+extern "C" eta_engine_t eta_get_decode_engine(void) {
+  return static_cast<eta_engine_t>(g_engine.load());
+}
 
 extern "C" size_t eta_decode_workspace_size(const eta_dims_t* dims) {
   if (check_dims(dims) != ETA_OK) return 0;

@@ -80,3 +80,12 @@ def test_argument_validation_without_gpu():
     assert lib.eta_predict_tau(ctypes.byref(g3), *([None] * 7)) == 2
     assert L.eta_screen_workspace_size(dims) == 256       # 2*4 rows x 2 words, 256-aligned
     assert L.eta_screen_workspace_size(bad) == 0
+
+
+def test_engine_selection_host_only():
+    assert L.eta_get_decode_engine() == "auto"
+    L.eta_set_decode_engine("fma")
+    assert L.eta_get_decode_engine() == "fma"
+    L.eta_set_decode_engine("auto")
+    with pytest.raises(L.EtaError):
+        L.eta_set_decode_engine(7)

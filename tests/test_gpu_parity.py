@@ -19,6 +19,15 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+@pytest.fixture(autouse=True, params=["fma", "tcgen05"])
+def engine(request):
+    """Every parity test runs on both decode engines."""
+    from long_context_decoding_eta_b200 import _lib as L
+    L.eta_set_decode_engine(request.param)
+    yield request.param
+    L.eta_set_decode_engine("auto")
+
+
 def make(w, lengths=None, seed=None):
     g = synth.generate(w, "cpu", seed=seed, lengths=lengths)
     return g

@@ -173,6 +173,36 @@ eta_status_t eta_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float
                         size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * eta_decode_static -- eta_decode for callers that cannot allocate device memory.
+ * (No counterpart in the paper: this is a packaging choice of this library.)
+ * Some callers cannot give the library any scratch memory -- for instance a
+ * serving loop whose device memory is entirely taken by its own pool once it has
+ * started, or code that must not call cudaMalloc on the decode path because
+ * cudaMalloc can synchronize the device and stall other streams.  This entry
+ * point computes exactly what eta_decode computes, with the same arguments minus
+ * the workspace: its scratch is a fixed 4 MiB array in device memory that the
+ * library defines statically, so every GPU that loads the library holds those
+ * 4 MiB until the process exits.  It calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *  - Limit: returns ETA_ERR_WORKSPACE when eta_decode_workspace_size(dims) would
+ *    exceed eta_decode_static_max_workspace() (4 MiB; enough for B * Hkv up to
+ *    about 900 pairs at G = 4, d = 128 on a 148-SM GPU).
+ *  - Set-up: the first call made on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current).  Make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents; nothing
+ *    in it needs to start at zero.  Calls that overlap on the GPU (other streams,
+ *    other host threads) race on it: serialize them.
+ */
+eta_status_t eta_decode_static(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
+                               const eta_bf16_t* K, const eta_bf16_t* V,
+                               const int32_t* lengths, const int32_t* union_idx,
+                               const int32_t* union_cnt, float T, float scale,
+                               eta_prune_t prune, const float* vsum, const int32_t* cnt,
+                               float* o, float* lse, int32_t* dev_status, void* stream);
+size_t eta_decode_static_max_workspace(void);
+
+/*
  * eta_dense_decode -- the dense baseline the speedups are measured against (the
  * pages compare with FlashAttention-2 decode): standard softmax decode attention
  * over every valid key, no threshold, no gate, same split-KV pipeline as eta_decode.

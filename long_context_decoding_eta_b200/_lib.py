@@ -28,7 +28,8 @@ DEVSTAT_TIMEOUT, DEVSTAT_NONFINITE_Q, DEVSTAT_BAD_BLOCK, DEVSTAT_BAD_LENGTH = 1,
 EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size",
            "eta_screen", "eta_decode_workspace_size", "eta_decode", "eta_dense_decode",
            "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string",
-           "eta_set_decode_engine", "eta_get_decode_engine")
+           "eta_set_decode_engine", "eta_get_decode_engine", "eta_decode_static",
+           "eta_decode_static_max_workspace")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 
 
@@ -82,6 +83,11 @@ def lib() -> C.CDLL:
     L.eta_status_from_device.argtypes = [I32]
     L.eta_status_string.argtypes = [I32]
     L.eta_status_string.restype = C.c_char_p
+    L.eta_decode_static.argtypes = [DIMS, P, P, P, P, P, P, P, F32, F32, I32, P, P, P, P, P,
+                                    P]
+    L.eta_decode_static.restype = I32
+    L.eta_decode_static_max_workspace.argtypes = []
+    L.eta_decode_static_max_workspace.restype = C.c_size_t
     L.eta_set_decode_engine.argtypes = [I32]
     L.eta_set_decode_engine.restype = I32
     L.eta_get_decode_engine.argtypes = []
@@ -146,6 +152,21 @@ def eta_decode(dims: Dims, q, tau, K, V, lengths, union_idx, union_cnt, T, scale
         PRUNE[prune] if isinstance(prune, str) else int(prune), _p(vsum), _p(cnt), _p(o),
         _p(lse), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(), _p(dev_status),
         _stream(stream)))
+
+
+def eta_decode_static(dims: Dims, q, tau, K, V, lengths, union_idx, union_cnt, T, scale,
+                      prune, vsum, cnt, o, lse, dev_status=None, stream=None):
+    """eta_decode without a workspace argument: the library's fixed device scratch
+    is used instead (for callers that cannot allocate device memory)."""
+    _check("eta_decode_static", lib().eta_decode_static(
+        C.byref(dims), _p(q), _p(tau), _p(K), _p(V), _p(lengths), _p(union_idx),
+        _p(union_cnt), float(T), float(scale),
+        PRUNE[prune] if isinstance(prune, str) else int(prune), _p(vsum), _p(cnt), _p(o),
+        _p(lse), _p(dev_status), _stream(stream)))
+
+
+def eta_decode_static_max_workspace() -> int:
+    return int(lib().eta_decode_static_max_workspace())
 
 
 def eta_dense_decode(dims: Dims, q, K, V, lengths, scale, o, lse, ws, dev_status=None,

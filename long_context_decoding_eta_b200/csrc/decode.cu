@@ -721,3 +721,57 @@ extern "C" eta_status_t eta_dense_decode(const eta_dims_t* dims, const eta_bf16_
                           ETA_PRUNE_SKIP, nullptr, nullptr, o, lse, ws, ws_bytes, dev_status,
                           stream);
 }
+
+// ---------------------------------------------------------------- decode without a workspace
+//
+// Some callers cannot hand the library any device memory for scratch: a serving
+// loop whose device memory is entirely owned by its own pool once it has started,
+// or code that must not call cudaMalloc on the decode path because cudaMalloc can
+// synchronize the device and stall every other stream.  eta_decode_static serves
+// them: it runs exactly the eta_decode pipeline, but its scratch (the plan, the
+// prefix sums and the per-CTA partial results) lives in the fixed array below,
+// which every GPU that loads this library holds until the process exits.
+namespace eta {
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;   // 4 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch per device, looked up once per device (with
+// that device current) on the first call made on it.
+constexpr int kMaxDevices = 64;
+static std::atomic<void*> g_static_scratch_ptr[kMaxDevices];
+
+inline eta_status_t static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ETA_ERR_CUDA;
+  void* ptr = g_static_scratch_ptr[dev].load();
+  if (!ptr) {
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return ETA_ERR_CUDA;
+    g_static_scratch_ptr[dev].store(ptr);
+  }
+  *out = ptr;
+  return ETA_OK;
+}
+
+}  // namespace eta
+
+extern "C" size_t eta_decode_static_max_workspace(void) { return eta::kStaticScratchBytes; }
+
+extern "C" eta_status_t eta_decode_static(const eta_dims_t* dims, const eta_bf16_t* q,
+                                          const float* tau, const eta_bf16_t* K,
+                                          const eta_bf16_t* V, const int32_t* lengths,
+                                          const int32_t* union_idx, const int32_t* union_cnt,
+                                          float T, float scale, eta_prune_t prune,
+                                          const float* vsum, const int32_t* cnt, float* o,
+                                          float* lse, int32_t* dev_status, void* stream) {
+  eta_status_t st = check_dims(dims);
+  if (st != ETA_OK) return st;
+  const size_t need = ws_layout(dims, decode_grid()).total;
+  if (need > kStaticScratchBytes) return ETA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if ((st = static_scratch(&ws)) != ETA_OK) return st;
+  // Nothing in the scratch has to start at zero: every call's plan kernel rewrites
+  // all the bookkeeping the later kernels of the same call read.
+  return run_decode<false>(dims, q, tau, K, V, lengths, union_idx, union_cnt, T, scale, prune,
+                           vsum, cnt, o, lse, ws, kStaticScratchBytes, dev_status, stream);
+}

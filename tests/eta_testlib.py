@@ -48,11 +48,12 @@ def run_cuda(dec, q, W=None, bias=None, tau_const=None, tau=None) -> Dict[str, n
     return out
 
 
-def gpu_meta(dec) -> Dict[str, np.ndarray]:
-    m = dict(cent=f64(dec.cent.transpose(2, 3)), rmax=f64(dec.rmax), var=f64(dec.var),
-             cnt=dec.cnt.cpu().numpy().astype(np.int64))
+def gpu_meta(dec, rows=None) -> Dict[str, np.ndarray]:
+    sel = (lambda t: t) if rows is None else (lambda t: t[rows])
+    m = dict(cent=f64(sel(dec.cent).transpose(2, 3)), rmax=f64(sel(dec.rmax)),
+             var=f64(sel(dec.var)), cnt=sel(dec.cnt).cpu().numpy().astype(np.int64))
     if dec.vsum is not None:
-        m["vsum"] = f64(dec.vsum)
+        m["vsum"] = f64(sel(dec.vsum))
     return m
 
 

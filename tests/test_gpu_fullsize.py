@@ -1,0 +1,134 @@
+"""Full-size workloads, in the launch configuration the benchmark times (whole
+batch on the GPU, default engine), checked against the float64 oracle on sampled
+batch rows (the oracle computes those rows one by one), plus properties that hold
+at any size for every row."""
+import gc
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_decoding_eta_b200 import _lib as L
+from long_context_decoding_eta_b200 import synth
+from long_context_decoding_eta_b200.api import EtaDecoder
+from oracle import eta_oracle as O
+
+from eta_testlib import check_meta, compare_step, f64, gpu_meta, run_cuda, unpack_mask
+
+pytestmark = pytest.mark.gpu
+
+
+def rows_f64(t, rows):
+    return t[rows].double().cpu().numpy()
+
+
+def sampled_oracle_bias(w, g, rows, scale):
+    """Threshold offset from the oracle on the sampled rows (density target of the
+    workload), so that no input of the comparison comes from the CUDA path."""
+    K64 = rows_f64(g["K"], rows)
+    q64 = rows_f64(g["q"], rows)
+    L64 = g["lengths"][rows].cpu().numpy()
+    meta = O.cache_meta(K64, L64, w.blk)
+    W64 = g["W"].double().cpu().numpy()
+    tau0 = O.predict_tau(q64, W64, np.zeros(w.Hq))
+    ub = O.screen(q64, tau0, meta, scale, w.bound, w.z)["bounds"]
+    valid = np.repeat(meta["cnt"] > 0, w.G, axis=1)
+    return O.offset_for_density(ub, tau0, valid, w.density, w.G, w.density_kind)
+
+
+def whole_batch_properties(dec, gpu, w):
+    """Checks that hold for every row at any size."""
+    G, NB = w.G, dec.NB
+    hm = gpu["head_mask"]                                   # [B, Hq, NB]
+    cnt = dec.cnt.cpu().numpy()
+    assert not np.any(hm & ~np.repeat(cnt > 0, G, axis=1)), "empty block admitted"
+    un = hm.reshape(w.B, w.Hkv, G, NB).any(axis=2)
+    assert np.array_equal(gpu["union_cnt"], un.sum(axis=2))
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            c = gpu["union_cnt"][b, g]
+            assert np.array_equal(gpu["union_idx"][b, g, :c], np.nonzero(un[b, g])[0])
+    assert np.all(np.isfinite(gpu["o"]))
+    return un.mean()
+
+
+def run_fullsize(w, rows, tau_const=None, engine="auto"):
+    L.eta_set_decode_engine(engine)
+    scale = 1.0 / math.sqrt(w.d)
+    g = synth.generate(w, "cuda")
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, bound=w.bound, z=w.z,
+                     T=w.gate_T, keep_bounds=True)
+    dec.build_meta()
+    if tau_const is None:
+        bias = sampled_oracle_bias(w, g, rows, scale)
+        gpu = run_cuda(dec, g["q"], g["W"], torch.full((w.Hq,), bias, device="cuda"))
+        b64 = np.full(w.Hq, bias)
+    else:
+        gpu = run_cuda(dec, g["q"], tau_const=torch.tensor(tau_const, dtype=torch.float32,
+                                                            device="cuda"))
+        b64 = None
+    union_density = whole_batch_properties(dec, gpu, w)
+    # oracle on the sampled rows
+    K64, V64, q64 = rows_f64(g["K"], rows), rows_f64(g["V"], rows), rows_f64(g["q"], rows)
+    L64 = g["lengths"][rows].cpu().numpy()
+    meta = O.cache_meta(K64, L64, w.blk)
+    if tau_const is None:
+        tau = O.predict_tau(q64, g["W"].double().cpu().numpy(), b64)
+    else:
+        tau = O.const_tau(len(rows), np.asarray(tau_const, dtype=np.float64))
+    sc = O.screen(q64, tau, meta, scale, w.bound, w.z)
+    o, lse = O.decode(q64, tau, K64, V64, L64, sc["union_idx"], w.blk, scale, w.gate_T)
+    check_meta(gpu_meta(dec, rows), meta)
+    rep = compare_step(gpu, tau, sc, o, lse, q64, K64, V64, L64, w.blk, scale, w.gate_T, w.G,
+                       rows=rows)
+    del dec, g
+    gc.collect()
+    torch.cuda.empty_cache()
+    L.eta_set_decode_engine("auto")
+    return rep, union_density
+
+
+@pytest.mark.parametrize("engine", ["auto", "fma"])
+def test_long_128k_b64_union16(engine):
+    w = synth.LONG128K
+    rep, dens = run_fullsize(w, rows=[0, 37, 63], engine=engine)
+    # the density target is set on the 3 sampled rows only; across the batch it
+    # varies with the rows' thresholds: require real pruning and real admission
+    assert 0.01 < dens < 0.6, dens
+    print(rep, dens)
+
+
+def test_extreme_512k_b64_prob_bound_blk128():
+    w = synth.EXTREME512K
+    rep, dens = run_fullsize(w, rows=[5, 60])
+    assert 0.01 < dens < 0.6, dens
+    print(rep, dens)
+
+
+def test_calibrated_256k_const_tau():
+    # per-head constants from the calibration rule on the oracle, with the
+    # calibration queries paired with the sampled rows (the full-batch pairing
+    # would need the oracle's metadata of all 64 rows)
+    w = synth.CALIB256K
+    rows = [3, 42]
+    scale = 1.0 / math.sqrt(w.d)
+    g = synth.generate(w, "cuda")
+    K64 = rows_f64(g["K"], rows)
+    L64 = g["lengths"][rows].cpu().numpy()
+    meta = O.cache_meta(K64, L64, w.blk)
+    qc = synth.calibration_queries(w, g["mu"]).double().cpu().numpy()
+    n = qc.shape[0]
+    bounds = np.zeros((n, w.Hq, w.NB))
+    valid = np.zeros((n, w.Hq, w.NB), dtype=bool)
+    for i in range(n):
+        r = i % len(rows)
+        mrow = {k: v[r:r + 1] for k, v in meta.items()}
+        bounds[i] = O.screen(qc[i:i + 1], np.zeros((1, w.Hq)), mrow, scale)["bounds"][0]
+        valid[i] = np.repeat(meta["cnt"][r] > 0, w.G, axis=0)
+    tau_const = O.calibrate_const_tau(bounds, valid, w.density)
+    del g, K64
+    gc.collect()
+    torch.cuda.empty_cache()
+    rep, dens = run_fullsize(w, rows=rows, tau_const=tau_const)
+    print(rep, dens)

@@ -2,9 +2,10 @@
 //
 // "Cached centroid/variance/max-norm metadata" (evolve.pub review of arXiv
 // 2609.20888, Summary); "cached geometric-probabilistic bounds" (abstract).
-// One warp per block; every lane owns d/32 consecutive dimensions, so each key
-// row is one coalesced 128/256-byte warp load.  Blocks live in L2 between the two
-// passes over their keys (16-32 KB each).
+// Full build: one warp per block; every lane owns d/32 consecutive dimensions, so
+// each key row is one coalesced 128/256-byte warp load.  Blocks live in L2 between
+// the two passes over their keys (16-32 KB each).  Tail refresh (the per-token
+// append): one CTA per block, keys split over its 8 warps.
 #include "eta_common.cuh"
 #include "eta_host.h"
 
@@ -56,16 +57,29 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
   const size_t rowj = (size_t)r * NB + j;
   const eta_bf16_t* kb = K + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
 
+  // The keys are summed in kMetaWarps consecutive chunks of ceil(blk / kMetaWarps)
+  // keys, each chunk sequentially from zero, and the chunk sums in order: exactly
+  // the order of meta_tail_kernel, so a tail refresh and a full rebuild of the same
+  // block give bit-identical metadata.
+  const int per = (blk + kMetaWarps - 1) / kMetaWarps;
   float c[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) c[i] = 0.f;
-  // pass 1: centroid (sequential fp32 sum over the keys, then one division)
-#pragma unroll 8
-  for (int t = 0; t < n; ++t) {
-    float x[DPL];
-    load_row<DPL>(kb + (size_t)t * D, x);
+  // pass 1: centroid
+  for (int w = 0; w < kMetaWarps; ++w) {
+    const int lo = min(w * per, n), hi = min(lo + per, n);
+    float pc[DPL];
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) c[i] += x[i];
+    for (int i = 0; i < DPL; ++i) pc[i] = 0.f;
+#pragma unroll 4
+    for (int t = lo; t < hi; ++t) {
+      float x[DPL];
+      load_row<DPL>(kb + (size_t)t * D, x);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) pc[i] += x[i];
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) c[i] += pc[i];
   }
   if (n > 0) {
 #pragma unroll
@@ -73,19 +87,24 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
   }
   // pass 2: squared distances to the stored fp32 centroid
   float r2max = 0.f, s2 = 0.f;
+  for (int w = 0; w < kMetaWarps; ++w) {
+    const int lo = min(w * per, n), hi = min(lo + per, n);
+    float ps = 0.f;
 #pragma unroll 4
-  for (int t = 0; t < n; ++t) {
-    float x[DPL];
-    load_row<DPL>(kb + (size_t)t * D, x);
-    float p = 0.f;
+    for (int t = lo; t < hi; ++t) {
+      float x[DPL];
+      load_row<DPL>(kb + (size_t)t * D, x);
+      float p = 0.f;
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) {
-      const float dv = x[i] - c[i];
-      p = fmaf(dv, dv, p);
+      for (int i = 0; i < DPL; ++i) {
+        const float dv = x[i] - c[i];
+        p = fmaf(dv, dv, p);
+      }
+      p = warp_sum(p);          // butterfly: bit-identical in every lane
+      r2max = fmaxf(r2max, p);
+      ps += p;
     }
-    p = warp_sum(p);          // butterfly: bit-identical in every lane
-    r2max = fmaxf(r2max, p);
-    s2 += p;
+    s2 += ps;
   }
   float* cr = cent + (size_t)r * D * NB + j;
 #pragma unroll
@@ -100,16 +119,132 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
     float a[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) a[i] = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < n; ++t) {
+    for (int w = 0; w < kMetaWarps; ++w) {
+      const int lo = min(w * per, n), hi = min(lo + per, n);
+      float pa[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) pa[i] = 0.f;
+#pragma unroll 4
+      for (int t = lo; t < hi; ++t) {
+        float x[DPL];
+        load_row<DPL>(vb + (size_t)t * D, x);
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) pa[i] += x[i];
+      }
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) a[i] += pa[i];
+    }
+    float* vr = vsum + rowj * D + lane * DPL;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) vr[i] = a[i];
+  }
+}
+
+// Tail-block refresh (one block per (row, KV head) after a token is appended):
+// the same arithmetic as meta_build_kernel (sequential fp32 sum over the keys in
+// token order, one division, butterfly distance sums), but the block's keys are
+// split over the 8 warps of a CTA so the latency chain is blk/8 keys instead of blk.
+// The chunk sums are combined in warp order, the same order meta_build_kernel
+// uses, so both kernels give bit-identical metadata for the same block.
+template <int D>
+__global__ void __launch_bounds__(kMetaWarps * 32)
+meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restrict__ K,
+                 const eta_bf16_t* __restrict__ V, const int32_t* __restrict__ lengths,
+                 float* __restrict__ cent, float* __restrict__ rmax, float* __restrict__ var,
+                 int32_t* __restrict__ cnt, float* __restrict__ vsum) {
+  constexpr int DPL = D / 32;
+  __shared__ float part[kMetaWarps][D];
+  __shared__ float red_max[kMetaWarps], red_sum[kMetaWarps];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x, b = r / Hkv;
+  const int len = min(max(lengths[b], 0), T_max);
+  if (len == 0) return;                      // uniform over the CTA
+  const int j = (len - 1) / blk;
+  const int n = min(len - j * blk, blk);
+  const int per = (blk + kMetaWarps - 1) / kMetaWarps;
+  const int t_lo = min(warp * per, n), t_hi = min(t_lo + per, n);
+  const size_t rowj = (size_t)r * NB + j;
+  const eta_bf16_t* kb = K + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
+
+  float c[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) c[i] = 0.f;
+  for (int t = t_lo; t < t_hi; ++t) {
+    float x[DPL];
+    load_row<DPL>(kb + (size_t)t * D, x);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) c[i] += x[i];
+  }
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) part[warp][lane * DPL + i] = c[i];
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMetaWarps; ++w) s += part[w][lane * DPL + i];
+    c[i] = s / (float)n;
+  }
+  float r2max = 0.f, s2 = 0.f;
+  for (int t = t_lo; t < t_hi; ++t) {
+    float x[DPL];
+    load_row<DPL>(kb + (size_t)t * D, x);
+    float pd = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const float dv = x[i] - c[i];
+      pd = fmaf(dv, dv, pd);
+    }
+    pd = warp_sum(pd);
+    r2max = fmaxf(r2max, pd);
+    s2 += pd;
+  }
+  if (lane == 0) {
+    red_max[warp] = r2max;
+    red_sum[warp] = s2;
+  }
+  if (warp == 0) {
+    float* cr = cent + (size_t)r * D * NB + j;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) cr[(size_t)(lane * DPL + i) * NB] = c[i];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f, sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMetaWarps; ++w) {
+      m = fmaxf(m, red_max[w]);
+      sum += red_sum[w];
+    }
+    rmax[rowj] = __fmul_ru(__fsqrt_ru(m), kRadiusInflate);
+    var[rowj] = sum / (float)n;
+    cnt[rowj] = n;
+  }
+  if (vsum) {
+    __syncthreads();
+    const eta_bf16_t* vb = V + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
+    float a[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) a[i] = 0.f;
+    for (int t = t_lo; t < t_hi; ++t) {
       float x[DPL];
       load_row<DPL>(vb + (size_t)t * D, x);
 #pragma unroll
       for (int i = 0; i < DPL; ++i) a[i] += x[i];
     }
-    float* vr = vsum + rowj * D + lane * DPL;
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) vr[i] = a[i];
+    for (int i = 0; i < DPL; ++i) part[warp][lane * DPL + i] = a[i];
+    __syncthreads();
+    if (warp == 0) {
+      float* vr = vsum + rowj * D + lane * DPL;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        float s = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMetaWarps; ++w) s += part[w][lane * DPL + i];
+        vr[i] = s;
+      }
+    }
   }
 }
 
@@ -138,8 +273,19 @@ extern "C" eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_b
     if (nblk == 0) return ETA_OK;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dim3 grid(tail ? 1 : (nblk + kMetaWarps - 1) / kMetaWarps, R);
-  dim3 block(tail ? 32 : kMetaWarps * 32);
+  if (tail) {
+    if (dims->d == 128)
+      meta_tail_kernel<128><<<R, kMetaWarps * 32, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB,
+                                                          K, V, lengths, cent, rmax, var, cnt,
+                                                          vsum);
+    else
+      meta_tail_kernel<64><<<R, kMetaWarps * 32, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB,
+                                                         K, V, lengths, cent, rmax, var, cnt,
+                                                         vsum);
+    return launch_status();
+  }
+  dim3 grid((nblk + kMetaWarps - 1) / kMetaWarps, R);
+  dim3 block(kMetaWarps * 32);
   if (dims->d == 128)
     meta_build_kernel<128><<<grid, block, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB, K, V,
                                                    lengths, blk_begin, nblk, tail, cent, rmax,

@@ -3,55 +3,56 @@
 // Eq. 1: tau = qbar W_tau + b_tau) or a frozen per-head constant (abstract: offline
 // calibration "freezes per-head constant thresholds").
 //
-// A GEMV per batch row: one CTA per row streams W (Hq*d x Hq fp32, 128 KB at
-// Hq = 16, d = 128; L2-resident across rows) with every thread owning rows of W,
-// then a fixed-order block reduction, so results are deterministic.
+// A GEMV per batch row, split by KV group: W (Hq*d x Hq fp32, 128 KB at Hq = 16,
+// d = 128) stays L2-resident across rows; every thread owns rows of W, then a
+// fixed-order block reduction, so results are deterministic.
 #include "eta_common.cuh"
 #include "eta_host.h"
 
 namespace eta {
 
 constexpr int kTauThreads = 256;
-constexpr int kTauHeadsPerPass = 16;
 
+// One CTA per (batch row, KV group): the G outputs of the group, each thread
+// owning every 256th element of qbar; W's G columns of the group are read as one
+// 16/32-byte piece per row of W.  2 * Hkv * B CTAs keep the GEMV latency short.
+template <int G>
 __global__ void __launch_bounds__(kTauThreads)
-predict_tau_kernel(int Hq, int D, const eta_bf16_t* __restrict__ q, const float* __restrict__ W,
-                   const float* __restrict__ bias, float* __restrict__ tau, int32_t* status) {
-  __shared__ float red[kTauThreads / 32][kTauHeadsPerPass];
-  const int b = blockIdx.x;
+predict_tau_group_kernel(int Hq, int D, const eta_bf16_t* __restrict__ q,
+                         const float* __restrict__ W, const float* __restrict__ bias,
+                         float* __restrict__ tau, int32_t* status) {
+  __shared__ float red[kTauThreads / 32][G];
+  const int b = blockIdx.x, g = blockIdx.y;
   const int n = Hq * D;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const eta_bf16_t* qb = q + (size_t)b * n;
+  const int h0 = g * G;
+  float acc[G];
+#pragma unroll
+  for (int k = 0; k < G; ++k) acc[k] = 0.f;
   bool bad = false;
-  for (int h0 = 0; h0 < Hq; h0 += kTauHeadsPerPass) {
-    const int hc = min(kTauHeadsPerPass, Hq - h0);
-    float acc[kTauHeadsPerPass];
+#pragma unroll 4
+  for (int i = threadIdx.x; i < n; i += kTauThreads) {
+    const float x = bf16_to_f(qb[i]);
+    bad |= !isfinite(x);
+    const float* wr = W + (size_t)i * Hq + h0;
 #pragma unroll
-    for (int k = 0; k < kTauHeadsPerPass; ++k) acc[k] = 0.f;
-    for (int i = threadIdx.x; i < n; i += kTauThreads) {
-      const float x = bf16_to_f(qb[i]);
-      bad |= !isfinite(x);
-      const float* wr = W + (size_t)i * Hq + h0;
-#pragma unroll
-      for (int k = 0; k < kTauHeadsPerPass; ++k)
-        if (k < hc) acc[k] = fmaf(x, __ldg(wr + k), acc[k]);
-    }
-#pragma unroll
-    for (int k = 0; k < kTauHeadsPerPass; ++k) {
-      const float v = warp_sum(acc[k]);
-      if (lane == 0) red[warp][k] = v;
-    }
-    __syncthreads();
-    if (threadIdx.x < hc) {
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < kTauThreads / 32; ++w) s += red[w][threadIdx.x];
-      const int h = h0 + threadIdx.x;
-      tau[(size_t)b * Hq + h] = s + (bias ? bias[h] : 0.f);
-    }
-    __syncthreads();
+    for (int k = 0; k < G; ++k) acc[k] = fmaf(x, __ldg(wr + k), acc[k]);
   }
-  if (bad) set_status(status, ETA_DEVSTAT_NONFINITE_Q);
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    const float v = warp_sum(acc[k]);
+    if (lane == 0) red[warp][k] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < G) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kTauThreads / 32; ++w) s += red[w][threadIdx.x];
+    const int h = h0 + threadIdx.x;
+    tau[(size_t)b * Hq + h] = s + (bias ? bias[h] : 0.f);
+  }
+  if (bad && g == 0) set_status(status, ETA_DEVSTAT_NONFINITE_Q);
 }
 
 __global__ void const_tau_kernel(int total, int Hq, const float* __restrict__ tau_const,
@@ -78,7 +79,13 @@ extern "C" eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t
     return launch_status();
   }
   if (!q || !W) return ETA_ERR_INVALID_ARG;
-  predict_tau_kernel<<<dims->B, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau,
-                                                      dev_status);
+  const dim3 grid(dims->B, dims->Hkv);
+  switch (dims->Hq / dims->Hkv) {
+    case 1: predict_tau_group_kernel<1><<<grid, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau, dev_status); break;
+    case 2: predict_tau_group_kernel<2><<<grid, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau, dev_status); break;
+    case 4: predict_tau_group_kernel<4><<<grid, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau, dev_status); break;
+    case 8: predict_tau_group_kernel<8><<<grid, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau, dev_status); break;
+    default: return ETA_ERR_UNSUPPORTED;
+  }
   return launch_status();
 }

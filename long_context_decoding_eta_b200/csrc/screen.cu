@@ -80,6 +80,120 @@ screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
   if (lane == 0) union_words[(size_t)r * NW + w] = uni;
 }
 
+// Vector form for NB % 4 == 0: lane l of a warp owns the 4 consecutive blocks
+// 4l..4l+3 of a 128-block group, so each of the d loads of a lane is one 16-byte
+// load and a warp moves 512 bytes per dimension.  A warp's four 32-bit admit words
+// per head are assembled from the lanes' 4-bit nibbles with an OR butterfly over
+// groups of 8 lanes.  Each warp walks kGroupsPerWarp groups so that the per-CTA
+// prologue (the group's queries in shared memory, their norms) is amortized.
+constexpr int kGroupsPerWarp = 1;
+constexpr int kScreen4Warps = 4;
+
+template <int D, int G>
+__global__ void __launch_bounds__(kScreen4Warps * 32)
+screen4_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
+               const float* __restrict__ tau, const float* __restrict__ cent,
+               const float* __restrict__ rmax, const float* __restrict__ var,
+               const int32_t* __restrict__ cnt, int bound, float z, float scale,
+               uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
+               float* __restrict__ bounds_out) {
+  __shared__ __align__(16) float qs[D * G];
+  __shared__ float qn[G], ts[G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.y, b = r / Hkv, g = r % Hkv;
+  const size_t qhead0 = (size_t)b * Hq + (size_t)g * G;
+
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int h = i / D, k = i % D;
+    qs[k * G + h] = bf16_to_f(q[(qhead0 + h) * D + k]);
+  }
+  __syncthreads();
+  for (int h = warp; h < G; h += kScreen4Warps) {
+    float s = 0.f;
+    for (int k = lane; k < D; k += 32) s = fmaf(qs[k * G + h], qs[k * G + h], s);
+    s = warp_sum(s);
+    if (lane == 0) {
+      qn[h] = sqrtf(s);
+      ts[h] = tau[qhead0 + h];
+    }
+  }
+  __syncthreads();
+
+  const int ngroups = (NB + 127) / 128;
+  for (int it = 0; it < kGroupsPerWarp; ++it) {
+    const int grp = (blockIdx.x * kScreen4Warps + warp) * kGroupsPerWarp + it;
+    if (grp >= ngroups) return;
+    const int j0 = grp * 128 + lane * 4;
+    const bool vj = j0 < NB;                       // NB % 4 == 0: all 4 valid or none
+    const float4* cp = reinterpret_cast<const float4*>(cent + (size_t)r * D * NB + (vj ? j0 : 0));
+    const size_t rowq = (size_t)NB / 4;            // float4 stride between dimensions
+    float acc[4][G];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[k][h] = 0.f;
+    // batches of kLoadBatch independent 16-byte loads in flight per lane
+    constexpr int kLoadBatch = 16;
+#pragma unroll 1
+    for (int d0 = 0; d0 < D; d0 += kLoadBatch) {
+      float4 cb[kLoadBatch];
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u)
+        cb[u] = vj ? __ldg(cp + (size_t)(d0 + u) * rowq) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < kLoadBatch; ++u) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float qv = qs[(d0 + u) * G + h];
+          acc[0][h] = fmaf(qv, cb[u].x, acc[0][h]);
+          acc[1][h] = fmaf(qv, cb[u].y, acc[1][h]);
+          acc[2][h] = fmaf(qv, cb[u].z, acc[2][h]);
+          acc[3][h] = fmaf(qv, cb[u].w, acc[3][h]);
+        }
+      }
+    }
+    const size_t rj = (size_t)r * NB + j0;
+    float rad[4] = {0.f, 0.f, 0.f, 0.f};
+    int n[4] = {0, 0, 0, 0};
+    if (vj) {
+      const float4 rr = __ldg(reinterpret_cast<const float4*>(rmax + rj));
+      const int4 cc = __ldg(reinterpret_cast<const int4*>(cnt + rj));
+      rad[0] = rr.x; rad[1] = rr.y; rad[2] = rr.z; rad[3] = rr.w;
+      n[0] = cc.x; n[1] = cc.y; n[2] = cc.z; n[3] = cc.w;
+      if (bound == ETA_BOUND_PROB) {
+        const float4 vv = __ldg(reinterpret_cast<const float4*>(var + rj));
+        rad[0] = fminf(rad[0], z * sqrtf(vv.x / (float)D));
+        rad[1] = fminf(rad[1], z * sqrtf(vv.y / (float)D));
+        rad[2] = fminf(rad[2], z * sqrtf(vv.z / (float)D));
+        rad[3] = fminf(rad[3], z * sqrtf(vv.w / (float)D));
+      }
+    }
+    uint32_t uni = 0;
+    const int wsel = lane >> 3;                    // word of the group this lane's nibble lands in
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      uint32_t nib = 0;
+      float ubv[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        ubv[k] = scale * fmaf(qn[h], rad[k], acc[k][h]);
+        if (vj && n[k] > 0 && ubv[k] >= ts[h]) nib |= 1u << k;
+      }
+      if (bounds_out && vj)
+        *reinterpret_cast<float4*>(bounds_out + (qhead0 + h) * NB + j0) =
+            make_float4(ubv[0], ubv[1], ubv[2], ubv[3]);
+      uint32_t word = nib << (4 * (lane & 7));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      word |= __shfl_xor_sync(0xffffffffu, word, 4);
+      // lanes 8w..8w+7 now hold word w of the group
+      if ((lane & 7) == 0 && grp * 4 + wsel < NW) head_mask[(qhead0 + h) * NW + grp * 4 + wsel] = word;
+      uni |= word;
+    }
+    if ((lane & 7) == 0 && grp * 4 + wsel < NW) union_words[(size_t)r * NW + grp * 4 + wsel] = uni;
+  }
+}
+
 __global__ void __launch_bounds__(kCompactThreads)
 compact_kernel(int Hq, int Hkv, int G, int NB, int NW, const uint32_t* __restrict__ union_words,
                const uint32_t* __restrict__ head_mask, int32_t* __restrict__ union_idx,
@@ -154,6 +268,27 @@ static void launch_screen(int G, dim3 grid, cudaStream_t s, int Hq, int Hkv, int
 #undef ETA_SCREEN_CASE
 }
 
+template <int D>
+static void launch_screen4(int G, dim3 grid, cudaStream_t s, int Hq, int Hkv, int NB, int NW,
+                           const eta_bf16_t* q, const float* tau, const float* cent,
+                           const float* rmax, const float* var, const int32_t* cnt, int bound,
+                           float z, float scale, uint32_t* head_mask, uint32_t* uw,
+                           float* bounds_out) {
+  const dim3 block(kScreen4Warps * 32);
+#define ETA_SCREEN4_CASE(GG)                                                                  \
+  case GG:                                                                                    \
+    screen4_kernel<D, GG><<<grid, block, 0, s>>>(Hq, Hkv, NB, NW, q, tau, cent, rmax, var, cnt, \
+                                                 bound, z, scale, head_mask, uw, bounds_out); \
+    break;
+  switch (G) {
+    ETA_SCREEN4_CASE(1)
+    ETA_SCREEN4_CASE(2)
+    ETA_SCREEN4_CASE(4)
+    ETA_SCREEN4_CASE(8)
+  }
+#undef ETA_SCREEN4_CASE
+}
+
 }  // namespace eta
 
 using namespace eta;
@@ -182,13 +317,27 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   const int R = dims->B * dims->Hkv, G = dims->Hq / dims->Hkv;
   uint32_t* uw = static_cast<uint32_t*>(ws);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dim3 grid((NW + kScreenWarps - 1) / kScreenWarps, R);
-  if (dims->d == 128)
-    launch_screen<128>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
-                       (int)bound, z, scale, head_mask, uw, bounds_out);
-  else
-    launch_screen<64>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
-                      (int)bound, z, scale, head_mask, uw, bounds_out);
+  const bool vec = (NB % 4 == 0) && aligned16(cent) && aligned16(rmax) && aligned16(cnt) &&
+                   (!var || aligned16(var)) && (!bounds_out || aligned16(bounds_out));
+  if (vec) {
+    const int ngroups = (NB + 127) / 128;
+    const int per_cta = kScreen4Warps * kGroupsPerWarp;
+    dim3 grid((ngroups + per_cta - 1) / per_cta, R);
+    if (dims->d == 128)
+      launch_screen4<128>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
+                          (int)bound, z, scale, head_mask, uw, bounds_out);
+    else
+      launch_screen4<64>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
+                         (int)bound, z, scale, head_mask, uw, bounds_out);
+  } else {
+    dim3 grid((NW + kScreenWarps - 1) / kScreenWarps, R);
+    if (dims->d == 128)
+      launch_screen<128>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
+                         (int)bound, z, scale, head_mask, uw, bounds_out);
+    else
+      launch_screen<64>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
+                        (int)bound, z, scale, head_mask, uw, bounds_out);
+  }
   st = launch_status();
   if (st != ETA_OK) return st;
   compact_kernel<<<R, kCompactThreads, 0, s>>>(dims->Hq, dims->Hkv, G, NB, NW, uw, head_mask,

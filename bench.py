@@ -71,6 +71,23 @@ def density_offset(bounds: np.ndarray, tau0: np.ndarray, valid: np.ndarray, dens
     return float(np.partition(v, k)[k])
 
 
+def reduce_max(x: float, device) -> float:
+    """Max over ranks of a per-rank figure (the job time of the independent,
+    weak-scaled replicas).  Identity when not running distributed."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, steps: int, max_ms: float) -> float:
+    """Whole-job steps/s: every rank runs `steps` full-batch steps of its own
+    replica; the job takes the slowest rank's time."""
+    return world * steps / (max_ms * 1e-3)
+
+
 class Clocks:
     """Samples SM clocks and throttle reasons with nvidia-smi during a region."""
 
@@ -224,12 +241,8 @@ def run_eta(args, rank, world, device):
     if world > 1:
         torch.distributed.barrier()
     dec.check_status()
-    ms = t0.elapsed_time(t1)
+    ms = reduce_max(t0.elapsed_time(t1), device)
     dec_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
 
     # dense baseline on the same cache (same pipeline, every block, no gate)
     for _ in range(3):
@@ -265,18 +278,14 @@ def run_eta(args, rank, world, device):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, device)
 
     peak, peak_kind = peaks()
     ms_step = ms / args.steps
     achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
     res = {
         "metric": METRIC,
-        "value": world * args.steps / (ms * 1e-3),
+        "value": job_throughput(world, args.steps, ms),
         "unit": "steps/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -309,7 +318,7 @@ def run_eta(args, rank, world, device):
         "dense_baseline": {"ms": dense_ms, "steps_per_s_decode_only": 1e3 / dense_ms,
                            "gbs": by["dense_kv"] / (dense_ms * 1e-3) / 1e9,
                            "speedup_of_eta_decode": dense_ms / dec_ms},
-        "e2e": {"value": world / (e2e_ms * 1e-3), "unit": "steps/s",
+        "e2e": {"value": job_throughput(world, 1, e2e_ms), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host.numel() * 2,
                 "d2h_bytes_per_step": o_host.numel() * 4 + lse_host.numel() * 4},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,

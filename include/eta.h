@@ -242,6 +242,18 @@ eta_status_t eta_calibrate_const_tau(const float* bounds, const uint8_t* valid,
                                      int32_t n_q, int32_t Hq, int32_t NB, float density,
                                      float* tau_out);
 
+/*
+ * eta_selftest_wait_timeout -- diagnostic of the failure detection (no counterpart
+ * in the paper).  Launches one small kernel that waits, with the same bounded wait
+ * the decode kernels use, on an mbarrier that nothing arrives on and on the int32
+ * flag *never_set (device memory, may be NULL; the caller keeps it 0).  After
+ * wait_limit polls each wait gives up and ETA_DEVSTAT_TIMEOUT is OR-ed into
+ * *dev_status (device memory); the context stays usable.
+ * wait_limit in [1, 2^24], else ETA_ERR_INVALID_ARG.
+ */
+eta_status_t eta_selftest_wait_timeout(uint32_t wait_limit, const int32_t* never_set,
+                                       int32_t* dev_status, void* stream);
+
 /* Maps a device status word (read back by the caller) to a status code. */
 eta_status_t eta_status_from_device(int32_t dev_status);
 

@@ -29,7 +29,7 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_screen", "eta_decode_workspace_size", "eta_decode", "eta_dense_decode",
            "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string",
            "eta_set_decode_engine", "eta_get_decode_engine", "eta_decode_static",
-           "eta_decode_static_max_workspace")
+           "eta_decode_static_max_workspace", "eta_selftest_wait_timeout")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 
 
@@ -88,6 +88,8 @@ def lib() -> C.CDLL:
     L.eta_decode_static.restype = I32
     L.eta_decode_static_max_workspace.argtypes = []
     L.eta_decode_static_max_workspace.restype = C.c_size_t
+    L.eta_selftest_wait_timeout.argtypes = [C.c_uint32, P, P, P]
+    L.eta_selftest_wait_timeout.restype = I32
     L.eta_set_decode_engine.argtypes = [I32]
     L.eta_set_decode_engine.restype = I32
     L.eta_get_decode_engine.argtypes = []
@@ -205,3 +207,9 @@ def eta_set_decode_engine(engine) -> None:
 def eta_get_decode_engine() -> str:
     v = int(lib().eta_get_decode_engine())
     return {k: n for n, k in ENGINE.items()}.get(v, str(v))
+
+
+def eta_selftest_wait_timeout(wait_limit: int, never_set, dev_status, stream=None) -> None:
+    """Runs the bounded-wait diagnostic kernel (see include/eta.h)."""
+    _check("eta_selftest_wait_timeout", lib().eta_selftest_wait_timeout(
+        int(wait_limit), _p(never_set), _p(dev_status), _stream(stream)))

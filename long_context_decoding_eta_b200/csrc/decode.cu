@@ -104,6 +104,7 @@ ETA_DEV float transpose_reduce32(float (&v)[32], int lane) {
 
 template <int D, int G, bool DENSE, int NCW, int NSTAGES>
 __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_kernel(const DecodeParams p) {
+  ETA_PDL_ENTRY();
   using C = DecodeCfg<D, G, NCW, NSTAGES>;
   constexpr int DPL = C::DPL, KG = C::KG;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -345,6 +346,7 @@ __global__ void __launch_bounds__(kPlanThreads)
 plan_kernel(int R, int Hkv, int NB, int blk, int T_max, const int32_t* __restrict__ union_cnt,
             const int32_t* __restrict__ lengths, int P, int32_t* __restrict__ row_off,
             int32_t* __restrict__ cta_row, int32_t* __restrict__ plan, int32_t* status) {
+  ETA_PDL_ENTRY();
   __shared__ int wsum[kPlanThreads / 32];
   __shared__ int s_chunk;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -421,6 +423,7 @@ struct CombineParams {
 
 template <int D, int G>
 __global__ void __launch_bounds__(D) combine_kernel(const CombineParams p) {
+  ETA_PDL_ENTRY();
   __shared__ uint32_t adm[65536 / 32];
   __shared__ int s_nfloor;
   const int r = blockIdx.x, b = r / p.Hkv, g = r % p.Hkv;
@@ -521,8 +524,7 @@ eta_status_t launch_decode_t(const eta_dims_t* dims, const DecodeParams& prm, in
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return ETA_ERR_CUDA;
-  kern<<<P, C::NT, C::SMEM, s>>>(prm);
-  return launch_status();
+  return launch_k(kern, dim3(P), dim3(C::NT), C::SMEM, s, prm);
 }
 
 template <bool DENSE>
@@ -541,10 +543,8 @@ inline eta_status_t launch_combine(const eta_dims_t* dims, const CombineParams& 
                                    cudaStream_t s) {
   const int G = dims->Hq / dims->Hkv, R = dims->B * dims->Hkv;
 #define ETA_CMB_CASE(DD, GG)                                              \
-  if (dims->d == DD && G == GG) {                                         \
-    combine_kernel<DD, GG><<<R, DD, 0, s>>>(cp);                          \
-    return launch_status();                                               \
-  }
+  if (dims->d == DD && G == GG)                                           \
+    return launch_k(combine_kernel<DD, GG>, dim3(R), dim3(DD), 0, s, cp);
   ETA_CMB_CASE(128, 1) ETA_CMB_CASE(128, 2) ETA_CMB_CASE(128, 4) ETA_CMB_CASE(128, 8)
   ETA_CMB_CASE(64, 1) ETA_CMB_CASE(64, 2) ETA_CMB_CASE(64, 4) ETA_CMB_CASE(64, 8)
 #undef ETA_CMB_CASE
@@ -600,8 +600,7 @@ eta_status_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUt
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES) !=
       cudaSuccess)
     return ETA_ERR_CUDA;
-  kern<<<P, tc::NT, tc::SMEM_BYTES, s>>>(mk, mv, mq, prm);
-  return launch_status();
+  return launch_k(kern, dim3(P), dim3(tc::NT), tc::SMEM_BYTES, s, mk, mv, mq, prm);
 }
 
 template <bool DENSE>
@@ -656,10 +655,9 @@ eta_status_t run_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float
   const int R = dims->B * dims->Hkv, NB = num_blocks(dims);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  plan_kernel<DENSE><<<1, kPlanThreads, 0, s>>>(R, dims->Hkv, NB, dims->blk, dims->T_max,
-                                                union_cnt, lengths, P, row_off, cta_row, plan,
-                                                dev_status);
-  if ((st = launch_status()) != ETA_OK) return st;
+  st = launch_k(plan_kernel<DENSE>, dim3(1), dim3(kPlanThreads), 0, s, R, dims->Hkv, NB,
+                dims->blk, dims->T_max, union_cnt, lengths, P, row_off, cta_row, plan, dev_status);
+  if (st != ETA_OK) return st;
 
   DecodeParams prm;
   prm.Hq = dims->Hq; prm.Hkv = dims->Hkv; prm.T_max = dims->T_max; prm.NB = NB;

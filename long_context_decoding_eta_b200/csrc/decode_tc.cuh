@@ -150,6 +150,7 @@ template <int G, bool DENSE>
 __global__ void __launch_bounds__(NT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const TcParams p) {
+  ETA_PDL_ENTRY();
   static_assert(G >= 1 && G <= 8, "G");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(

@@ -16,6 +16,19 @@ namespace eta {
 // legitimate wait (seconds) while still ending a lost wait.
 constexpr uint32_t kWaitLimit = 1u << 22;
 
+// Programmatic dependent launch: every kernel of the library is launched with
+// programmatic stream serialization allowed, waits for the grid before it in the
+// stream (completion and memory flush) before touching any global memory, and
+// then lets the grid after it start launching.  Only launch latency overlaps;
+// the data dependencies stay exactly those of plain stream order.
+ETA_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+ETA_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+#define ETA_PDL_ENTRY() \
+  do {                  \
+    eta::pdl_wait();    \
+    eta::pdl_trigger(); \
+  } while (0)
+
 ETA_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 ETA_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 ETA_DEV float bf16_to_f(uint16_t h) { return __uint_as_float(((uint32_t)h) << 16); }
@@ -58,14 +71,18 @@ ETA_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for phase `parity` of `bar`.  Returns false when the limit ran out
-// or when *abort became non-zero (another thread of the CTA gave up).
-ETA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+// Bounded wait for phase `parity` of `bar`.  Returns false when `limit` polls ran
+// out or when *abort became non-zero (another thread of the CTA gave up).
+ETA_DEV bool mbar_wait_n(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
   }
   return false;
+}
+
+ETA_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_n(bar, parity, abort, kWaitLimit);
 }
 
 // 1-D bulk copy (TMA engine) of `bytes` from global to this CTA's shared memory,

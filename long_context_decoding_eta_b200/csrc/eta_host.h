@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/eta.h"
 
 namespace eta {
@@ -29,6 +31,26 @@ inline eta_status_t check_dims(const eta_dims_t* d) {
   if (num_blocks(d) > 65536) return ETA_ERR_UNSUPPORTED;
   if (d->Hq > 256) return ETA_ERR_UNSUPPORTED;
   return ETA_OK;
+}
+
+// Launches `kern` on `s` with programmatic stream serialization allowed (see
+// ETA_PDL_ENTRY in eta_common.cuh).
+template <typename... KArgs, typename... Args>
+inline eta_status_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) == cudaSuccess
+             ? ETA_OK
+             : ETA_ERR_CUDA;
 }
 
 inline eta_status_t launch_status() {

@@ -35,6 +35,7 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
                   int blk_begin, int nblk, int tail, float* __restrict__ cent,
                   float* __restrict__ rmax, float* __restrict__ var, int32_t* __restrict__ cnt,
                   float* __restrict__ vsum, int32_t* status) {
+  ETA_PDL_ENTRY();
   constexpr int DPL = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.y;                 // (row, KV head) = b * Hkv + g
@@ -152,6 +153,7 @@ meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restri
                  const eta_bf16_t* __restrict__ V, const int32_t* __restrict__ lengths,
                  float* __restrict__ cent, float* __restrict__ rmax, float* __restrict__ var,
                  int32_t* __restrict__ cnt, float* __restrict__ vsum) {
+  ETA_PDL_ENTRY();
   constexpr int DPL = D / 32;
   __shared__ float part[kMetaWarps][D];
   __shared__ float red_max[kMetaWarps], red_sum[kMetaWarps];
@@ -274,25 +276,13 @@ extern "C" eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_b
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (tail) {
-    if (dims->d == 128)
-      meta_tail_kernel<128><<<R, kMetaWarps * 32, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB,
-                                                          K, V, lengths, cent, rmax, var, cnt,
-                                                          vsum);
-    else
-      meta_tail_kernel<64><<<R, kMetaWarps * 32, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB,
-                                                         K, V, lengths, cent, rmax, var, cnt,
-                                                         vsum);
-    return launch_status();
+    auto kern = dims->d == 128 ? meta_tail_kernel<128> : meta_tail_kernel<64>;
+    return launch_k(kern, dim3(R), dim3(kMetaWarps * 32), 0, s, dims->Hkv, dims->T_max,
+                    dims->blk, NB, K, V, lengths, cent, rmax, var, cnt, vsum);
   }
   dim3 grid((nblk + kMetaWarps - 1) / kMetaWarps, R);
-  dim3 block(kMetaWarps * 32);
-  if (dims->d == 128)
-    meta_build_kernel<128><<<grid, block, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB, K, V,
-                                                   lengths, blk_begin, nblk, tail, cent, rmax,
-                                                   var, cnt, vsum, nullptr);
-  else
-    meta_build_kernel<64><<<grid, block, 0, s>>>(dims->Hkv, dims->T_max, dims->blk, NB, K, V,
-                                                  lengths, blk_begin, nblk, tail, cent, rmax,
-                                                  var, cnt, vsum, nullptr);
-  return launch_status();
+  auto kern = dims->d == 128 ? meta_build_kernel<128> : meta_build_kernel<64>;
+  return launch_k(kern, grid, dim3(kMetaWarps * 32), 0, s, dims->Hkv, dims->T_max, dims->blk,
+                  NB, K, V, lengths, blk_begin, nblk, 0, cent, rmax, var, cnt, vsum,
+                  (int32_t*)nullptr);
 }

@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(kTauThreads)
 predict_tau_group_kernel(int Hq, int D, const eta_bf16_t* __restrict__ q,
                          const float* __restrict__ W, const float* __restrict__ bias,
                          float* __restrict__ tau, int32_t* status) {
+  ETA_PDL_ENTRY();
   __shared__ float red[kTauThreads / 32][G];
   const int b = blockIdx.x, g = blockIdx.y;
   const int n = Hq * D;
@@ -57,6 +58,7 @@ predict_tau_group_kernel(int Hq, int D, const eta_bf16_t* __restrict__ q,
 
 __global__ void const_tau_kernel(int total, int Hq, const float* __restrict__ tau_const,
                                  float* __restrict__ tau) {
+  ETA_PDL_ENTRY();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < total) tau[i] = tau_const[i % Hq];
 }
@@ -75,17 +77,19 @@ extern "C" eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (tau_const) {
     const int total = dims->B * dims->Hq;
-    const_tau_kernel<<<(total + 255) / 256, 256, 0, s>>>(total, dims->Hq, tau_const, tau);
-    return launch_status();
+    return launch_k(const_tau_kernel, dim3((total + 255) / 256), dim3(256), 0, s, total,
+                    dims->Hq, tau_const, tau);
   }
   if (!q || !W) return ETA_ERR_INVALID_ARG;
   const dim3 grid(dims->B, dims->Hkv);
+  void (*kern)(int, int, const eta_bf16_t*, const float*, const float*, float*, int32_t*) = nullptr;
   switch (dims->Hq / dims->Hkv) {
-    case 1: predict_tau_group_kernel<1><<<grid, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau, dev_status); break;
-    case 2: predict_tau_group_kernel<2><<<grid, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau, dev_status); break;
-    case 4: predict_tau_group_kernel<4><<<grid, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau, dev_status); break;
-    case 8: predict_tau_group_kernel<8><<<grid, kTauThreads, 0, s>>>(dims->Hq, dims->d, q, W, bias, tau, dev_status); break;
+    case 1: kern = predict_tau_group_kernel<1>; break;
+    case 2: kern = predict_tau_group_kernel<2>; break;
+    case 4: kern = predict_tau_group_kernel<4>; break;
+    case 8: kern = predict_tau_group_kernel<8>; break;
     default: return ETA_ERR_UNSUPPORTED;
   }
-  return launch_status();
+  return launch_k(kern, grid, dim3(kTauThreads), 0, s, dims->Hq, dims->d, q, W, bias, tau,
+                  dev_status);
 }

@@ -27,6 +27,7 @@ screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
               const int32_t* __restrict__ cnt, int bound, float z, float scale,
               uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
               float* __restrict__ bounds_out) {
+  ETA_PDL_ENTRY();
   __shared__ __align__(16) float qs[D * G];
   __shared__ float qn[G], ts[G];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -97,6 +98,7 @@ screen4_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q
                const int32_t* __restrict__ cnt, int bound, float z, float scale,
                uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
                float* __restrict__ bounds_out) {
+  ETA_PDL_ENTRY();
   __shared__ __align__(16) float qs[D * G];
   __shared__ float qn[G], ts[G];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,6 +200,7 @@ __global__ void __launch_bounds__(kCompactThreads)
 compact_kernel(int Hq, int Hkv, int G, int NB, int NW, const uint32_t* __restrict__ union_words,
                const uint32_t* __restrict__ head_mask, int32_t* __restrict__ union_idx,
                int32_t* __restrict__ union_cnt, int32_t* __restrict__ head_cnt) {
+  ETA_PDL_ENTRY();
   __shared__ uint32_t wbuf[kCompactThreads];
   __shared__ int woff[kCompactThreads];
   __shared__ int wsum[kCompactThreads / 32];
@@ -248,45 +251,25 @@ compact_kernel(int Hq, int Hkv, int G, int NB, int NW, const uint32_t* __restric
 }
 
 template <int D>
-static void launch_screen(int G, dim3 grid, cudaStream_t s, int Hq, int Hkv, int NB, int NW,
-                          const eta_bf16_t* q, const float* tau, const float* cent,
-                          const float* rmax, const float* var, const int32_t* cnt, int bound,
-                          float z, float scale, uint32_t* head_mask, uint32_t* uw,
-                          float* bounds_out) {
-  const dim3 block(kScreenWarps * 32);
-#define ETA_SCREEN_CASE(GG)                                                                  \
-  case GG:                                                                                   \
-    screen_kernel<D, GG><<<grid, block, 0, s>>>(Hq, Hkv, NB, NW, q, tau, cent, rmax, var, cnt, \
-                                                bound, z, scale, head_mask, uw, bounds_out); \
-    break;
+static eta_status_t launch_screen(bool vec, int G, dim3 grid, cudaStream_t s, int Hq, int Hkv,
+                                  int NB, int NW, const eta_bf16_t* q, const float* tau,
+                                  const float* cent, const float* rmax, const float* var,
+                                  const int32_t* cnt, int bound, float z, float scale,
+                                  uint32_t* head_mask, uint32_t* uw, float* bounds_out) {
+  using KernT = void (*)(int, int, int, int, const eta_bf16_t*, const float*, const float*,
+                         const float*, const float*, const int32_t*, int, float, float,
+                         uint32_t*, uint32_t*, float*);
+  KernT kern = nullptr;
   switch (G) {
-    ETA_SCREEN_CASE(1)
-    ETA_SCREEN_CASE(2)
-    ETA_SCREEN_CASE(4)
-    ETA_SCREEN_CASE(8)
+    case 1: kern = vec ? screen4_kernel<D, 1> : screen_kernel<D, 1>; break;
+    case 2: kern = vec ? screen4_kernel<D, 2> : screen_kernel<D, 2>; break;
+    case 4: kern = vec ? screen4_kernel<D, 4> : screen_kernel<D, 4>; break;
+    case 8: kern = vec ? screen4_kernel<D, 8> : screen_kernel<D, 8>; break;
+    default: return ETA_ERR_UNSUPPORTED;
   }
-#undef ETA_SCREEN_CASE
-}
-
-template <int D>
-static void launch_screen4(int G, dim3 grid, cudaStream_t s, int Hq, int Hkv, int NB, int NW,
-                           const eta_bf16_t* q, const float* tau, const float* cent,
-                           const float* rmax, const float* var, const int32_t* cnt, int bound,
-                           float z, float scale, uint32_t* head_mask, uint32_t* uw,
-                           float* bounds_out) {
-  const dim3 block(kScreen4Warps * 32);
-#define ETA_SCREEN4_CASE(GG)                                                                  \
-  case GG:                                                                                    \
-    screen4_kernel<D, GG><<<grid, block, 0, s>>>(Hq, Hkv, NB, NW, q, tau, cent, rmax, var, cnt, \
-                                                 bound, z, scale, head_mask, uw, bounds_out); \
-    break;
-  switch (G) {
-    ETA_SCREEN4_CASE(1)
-    ETA_SCREEN4_CASE(2)
-    ETA_SCREEN4_CASE(4)
-    ETA_SCREEN4_CASE(8)
-  }
-#undef ETA_SCREEN4_CASE
+  const dim3 block((vec ? kScreen4Warps : kScreenWarps) * 32);
+  return launch_k(kern, grid, block, 0, s, Hq, Hkv, NB, NW, q, tau, cent, rmax, var, cnt, bound,
+                  z, scale, head_mask, uw, bounds_out);
 }
 
 }  // namespace eta
@@ -319,28 +302,21 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool vec = (NB % 4 == 0) && aligned16(cent) && aligned16(rmax) && aligned16(cnt) &&
                    (!var || aligned16(var)) && (!bounds_out || aligned16(bounds_out));
+  dim3 grid;
   if (vec) {
     const int ngroups = (NB + 127) / 128;
     const int per_cta = kScreen4Warps * kGroupsPerWarp;
-    dim3 grid((ngroups + per_cta - 1) / per_cta, R);
-    if (dims->d == 128)
-      launch_screen4<128>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
-                          (int)bound, z, scale, head_mask, uw, bounds_out);
-    else
-      launch_screen4<64>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
-                         (int)bound, z, scale, head_mask, uw, bounds_out);
+    grid = dim3((ngroups + per_cta - 1) / per_cta, R);
   } else {
-    dim3 grid((NW + kScreenWarps - 1) / kScreenWarps, R);
-    if (dims->d == 128)
-      launch_screen<128>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
-                         (int)bound, z, scale, head_mask, uw, bounds_out);
-    else
-      launch_screen<64>(G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, cnt,
-                        (int)bound, z, scale, head_mask, uw, bounds_out);
+    grid = dim3((NW + kScreenWarps - 1) / kScreenWarps, R);
   }
-  st = launch_status();
+  st = dims->d == 128
+           ? launch_screen<128>(vec, G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax,
+                                var, cnt, (int)bound, z, scale, head_mask, uw, bounds_out)
+           : launch_screen<64>(vec, G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax,
+                               var, cnt, (int)bound, z, scale, head_mask, uw, bounds_out);
   if (st != ETA_OK) return st;
-  compact_kernel<<<R, kCompactThreads, 0, s>>>(dims->Hq, dims->Hkv, G, NB, NW, uw, head_mask,
-                                               union_idx, union_cnt, head_cnt);
-  return launch_status();
+  return launch_k(compact_kernel, dim3(R), dim3(kCompactThreads), 0, s, dims->Hq, dims->Hkv, G,
+                  NB, NW, (const uint32_t*)uw, (const uint32_t*)head_mask, union_idx, union_cnt,
+                  head_cnt);
 }

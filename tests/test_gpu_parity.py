@@ -223,3 +223,15 @@ def test_calibration_matches_oracle_rule():
         valid[i] = np.repeat(meta["cnt"][rows[i]] > 0, w.G, axis=0)
     tau_ref = O.calibrate_const_tau(bounds, valid, 0.38)
     np.testing.assert_allclose(tau_gpu, tau_ref, rtol=0, atol=2e-5)
+
+
+def test_bounded_wait_times_out_with_status_and_context_survives():
+    from long_context_decoding_eta_b200 import _lib as L
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    flag = torch.zeros(1, dtype=torch.int32, device=DEV)     # nothing ever sets it
+    L.eta_selftest_wait_timeout(1 << 12, flag, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & L.DEVSTAT_TIMEOUT
+    assert L.eta_status_from_device(int(status.item())) == 5
+    # the context is still usable: a normal decode runs and matches the oracle
+    rep, gpu, sc = full_parity(synth.TINY.with_(seed=86))

@@ -421,10 +421,17 @@ struct CombineParams {
   float* lse;
 };
 
+// One CTA per (row, KV head), thread = dim.  Three rounds of memory latency: the
+// row's slot range, then every (head, slot) (m, l) pair at once into shared memory,
+// then every (head, slot) partial o of this dim at once.
+constexpr int kCombineMaxPairs = 256;   // (head, slot) pairs staged in shared memory
+
 template <int D, int G>
 __global__ void __launch_bounds__(D) combine_kernel(const CombineParams p) {
   ETA_PDL_ENTRY();
-  __shared__ uint32_t adm[65536 / 32];
+  extern __shared__ uint32_t adm[];     // FLOOR mode: admitted-block bitmap of the row
+  __shared__ float sm_m[kCombineMaxPairs], sm_w[kCombineMaxPairs];
+  __shared__ float sM[G], sL[G];
   __shared__ int s_nfloor;
   const int r = blockIdx.x, b = r / p.Hkv, g = r % p.Hkv;
   const int dd = threadIdx.x;
@@ -454,31 +461,78 @@ __global__ void __launch_bounds__(D) combine_kernel(const CombineParams p) {
     __syncthreads();
     nfloor = s_nfloor;
   }
-  for (int h = 0; h < G; ++h) {
-    float M = -INFINITY, L = 0.f, O = 0.f;
-    if (c > 0) {
-      const int p0 = off / chunk, p1 = (off + c - 1) / chunk;
-      for (int pp = p0; pp <= p1; ++pp) M = fmaxf(M, p.part_ml[(((size_t)pp + r) * G + h) * 2]);
-      if (M != -INFINITY) {
-        for (int pp = p0; pp <= p1; ++pp) {
-          const size_t sl = ((size_t)pp + r) * G + h;
-          const float sc = expf(p.part_ml[sl * 2] - M);
-          L = fmaf(p.part_ml[sl * 2 + 1], sc, L);
-          O = fmaf(p.part_o[sl * D + dd], sc, O);
-        }
+  const int p0 = c > 0 ? off / chunk : 0;
+  const int ns = c > 0 ? (off + c - 1) / chunk - p0 + 1 : 0;
+  float O[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) O[h] = 0.f;
+  if (ns > 0) {
+    const int np = G * ns;                 // pair k = slot * G + h
+    if (np <= kCombineMaxPairs) {
+      for (int k = dd; k < np; k += D) {
+        const size_t sl = ((size_t)(p0 + k / G) + r) * G + (k % G);
+        sm_m[k] = p.part_ml[sl * 2];
+        sm_w[k] = p.part_ml[sl * 2 + 1];
       }
+      __syncthreads();
+      if (dd < G) {
+        float M = -INFINITY;
+        for (int k = dd; k < np; k += G) M = fmaxf(M, sm_m[k]);
+        float L = 0.f;
+        for (int k = dd; k < np; k += G) {
+          const float w = (M == -INFINITY) ? 0.f : expf(sm_m[k] - M);
+          L = fmaf(sm_w[k], w, L);
+          sm_m[k] = w;                       // now the slot weight
+        }
+        sM[dd] = M;
+        sL[dd] = L;
+      }
+      __syncthreads();
+      for (int k = 0; k < np; ++k) {
+        const size_t sl = ((size_t)(p0 + k / G) + r) * G + (k % G);
+        const float v = p.part_o[sl * D + dd];
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+          if (k % G == h) O[h] = fmaf(v, sm_m[k], O[h]);
+      }
+    } else {
+      // very long rows spread over many CTAs: plain two-pass merge per head
+      if (dd < G) { sM[dd] = -INFINITY; sL[dd] = 0.f; }
+      __syncthreads();
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float M = -INFINITY;
+        for (int k = 0; k < ns; ++k)
+          M = fmaxf(M, p.part_ml[(((size_t)(p0 + k) + r) * G + h) * 2]);
+        float L = 0.f;
+        for (int k = 0; k < ns; ++k) {
+          const size_t sl = ((size_t)(p0 + k) + r) * G + h;
+          const float w = (M == -INFINITY) ? 0.f : expf(p.part_ml[sl * 2] - M);
+          L = fmaf(p.part_ml[sl * 2 + 1], w, L);
+          O[h] = fmaf(p.part_o[sl * D + dd], w, O[h]);
+        }
+        if (dd == 0) { sM[h] = M; sL[h] = L; }
+      }
+      __syncthreads();
     }
+  } else {
+    if (dd < G) { sM[dd] = -INFINITY; sL[dd] = 0.f; }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float M = sM[h], L = sL[h], Oh = O[h];
     if (nfloor > 0) {
       const float Mf = fmaxf(M, 0.f);
       const float a = (M == -INFINITY) ? 0.f : expf(M - Mf);
       const float e0 = expf(-Mf);
-      O = O * a + fv * e0;
+      Oh = Oh * a + fv * e0;
       L = L * a + (float)nfloor * e0;
       M = Mf;
     }
     const size_t oh = (size_t)b * p.Hq + (size_t)g * G + h;
     if (L > 0.f) {
-      p.o[oh * D + dd] = O / L;
+      p.o[oh * D + dd] = Oh / L;
       if (dd == 0) p.lse[oh] = M + logf(L);
     } else {
       p.o[oh * D + dd] = 0.f;
@@ -542,9 +596,10 @@ eta_status_t launch_decode(const eta_dims_t* dims, const DecodeParams& prm, int 
 inline eta_status_t launch_combine(const eta_dims_t* dims, const CombineParams& cp,
                                    cudaStream_t s) {
   const int G = dims->Hq / dims->Hkv, R = dims->B * dims->Hkv;
+  const size_t smem = cp.floor_mode ? (size_t)((num_blocks(dims) + 31) / 32) * 4 : 0;
 #define ETA_CMB_CASE(DD, GG)                                              \
   if (dims->d == DD && G == GG)                                           \
-    return launch_k(combine_kernel<DD, GG>, dim3(R), dim3(DD), 0, s, cp);
+    return launch_k(combine_kernel<DD, GG>, dim3(R), dim3(DD), smem, s, cp);
   ETA_CMB_CASE(128, 1) ETA_CMB_CASE(128, 2) ETA_CMB_CASE(128, 4) ETA_CMB_CASE(128, 8)
   ETA_CMB_CASE(64, 1) ETA_CMB_CASE(64, 2) ETA_CMB_CASE(64, 4) ETA_CMB_CASE(64, 8)
 #undef ETA_CMB_CASE

@@ -71,6 +71,28 @@ def density_offset(bounds: np.ndarray, tau0: np.ndarray, valid: np.ndarray, dens
     return float(np.partition(v, k)[k])
 
 
+def decode_traffic(admitted_kv: int, engine_tc: bool):
+    """DRAM bytes per decode launch from the committed ncu capture
+    (profiles/decode_tc_traffic.json), scaled to this workload by its admitted K/V
+    bytes; None when the kernel source changed since the capture or the capture
+    does not cover the engine that ran."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "decode_tc_traffic.json")
+    if not engine_tc or not os.path.exists(p):
+        return None
+    rec = json.load(open(p))
+    m = hashlib.sha256()
+    for f in rec["source_files"]:
+        fp = os.path.join(ROOT, f)
+        if not os.path.exists(fp):
+            return None
+        m.update(open(fp, "rb").read())
+    if m.hexdigest() != rec["source_sha256"]:
+        return None
+    per = (rec["dram_bytes_read"] + rec["dram_bytes_write"]) / rec["admitted_kv_bytes"]
+    return per * admitted_kv
+
+
 def reduce_max(x: float, device) -> float:
     """Max over ranks of a per-rank figure (the job time of the independent,
     weak-scaled replicas).  Identity when not running distributed."""
@@ -314,7 +336,11 @@ def run_eta(args, rank, world, device):
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
                      "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
-                     "decode_ms": dec_ms, "traffic": None},
+                     "decode_ms": dec_ms,
+                     "traffic": decode_traffic(by["admitted_kv"], w.d == 128 and
+                                               args.engine in ("auto", "tcgen05")),
+                     "traffic_source": "profiles/decode_tc_traffic.json (ncu dram__bytes_read"
+                                       "+write of one full-size launch, scaled by admitted KV)"},
         "dense_baseline": {"ms": dense_ms, "steps_per_s_decode_only": 1e3 / dense_ms,
                            "gbs": by["dense_kv"] / (dense_ms * 1e-3) / 1e9,
                            "speedup_of_eta_decode": dense_ms / dec_ms},
@@ -368,6 +394,7 @@ def threads_used():
 
 
 def cpu_baseline(w, g, dec, W, bias, tau_const, rows=2):
+    rows = max(1, min(rows, w.B))
     dt, cores = oracle_sample_step(w, g, W, bias, tau_const, range(rows))
     per_step = dt * w.B / rows
     return {"value": 1.0 / per_step, "unit": "steps/s", "cores": cores, "kind": "oracle",
@@ -382,7 +409,7 @@ def run_reference(args, rank, world, device):
     from oracle import eta_oracle as O
     w = workload_by_name(args.workload, args.B)
     g = synth.generate(w, device, seed=w.seed)
-    rows = list(range(args.cpu_rows))
+    rows = list(range(max(1, min(args.cpu_rows, w.B))))
     K64 = g["K"][rows].double().cpu().numpy()
     q64 = g["q"][rows].double().cpu().numpy()
     L = g["lengths"][rows].cpu().numpy()

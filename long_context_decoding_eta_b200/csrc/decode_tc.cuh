@@ -236,15 +236,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         ++it;
         return true;
       };
-      for (int pos = a; pos < e && ok; ++pos) {
-        while (pos >= rend) {
-          ++r;
-          roff = rend;
-          rend = p.row_off[r + 1];
+      // The block index of position pos+1 is loaded before the stages of position pos
+      // are emitted, so its L2 latency overlaps the wait for a free stage.
+      auto fetch = [&](int pos, int& rr, int& ro, int& re) -> int {
+        while (pos >= re) {
+          ++rr;
+          ro = re;
+          re = p.row_off[rr + 1];
         }
+        return DENSE ? pos - ro : p.union_idx[(size_t)rr * p.NB + (pos - ro)];
+      };
+      int nr = r, nroff = roff, nrend = rend;
+      int j_next = a < e ? fetch(a, nr, nroff, nrend) : 0;
+      for (int pos = a; pos < e && ok; ++pos) {
+        const int j = j_next;
+        r = nr; roff = nroff; rend = nrend;
+        if (pos + 1 < e) j_next = fetch(pos + 1, nr, nroff, nrend);
         const int b = r / p.Hkv;
         const int len = min(max(p.lengths[b], 0), p.T_max);
-        const int j = DENSE ? pos - roff : p.union_idx[(size_t)r * p.NB + (pos - roff)];
         if (j < 0 || j >= p.NB || j * p.blk >= len) {
           set_status(p.status, ETA_DEVSTAT_BAD_BLOCK);
           continue;

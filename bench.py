@@ -164,11 +164,11 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def setup(w: synth.Workload, device, rank: int):
+def setup(w: synth.Workload, device, rank: int, cent_format: str = "f32"):
     from long_context_decoding_eta_b200.api import EtaDecoder
     g = synth.generate(w, device, seed=w.seed + 7919 * rank)
     dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, bound=w.bound, z=w.z,
-                     T=w.gate_T, keep_bounds=True)
+                     T=w.gate_T, keep_bounds=True, cent_format=cent_format)
     dec.build_meta()
     # workload calibration: bias so that tau hits the density target
     if w.tau_mode == "const":
@@ -202,8 +202,9 @@ def step_bytes(dec, w):
     adm_kv = int(keys) * d * 2 * 2                          # K + V, bf16
     qbytes = B * w.Hq * d * 2
     obytes = B * w.Hq * (d + 1) * 4
-    meta = B * Hkv * NB * (4 * d + 12)                      # cent + rmax + var + cnt read by screen
-    tail = B * Hkv * (blk * d * 2 + (4 * d + 12))           # tail block keys read + meta written
+    cb = 2 if dec.cent.dtype == torch.bfloat16 else 4
+    meta = B * Hkv * NB * (cb * d + 12)                     # cent + rmax + var + cnt read by screen
+    tail = B * Hkv * (blk * d * 2 + (cb * d + 12))          # tail block keys read + meta written
     tau_bytes = w.Hq * d * w.Hq * 4 + B * w.Hq * 4
     dens_union = float(ucnt.sum()) / max(1.0, float((cnt > 0).sum()))
     dens_head = float(dec.head_cnt.to(torch.int64).sum()) / max(
@@ -217,7 +218,7 @@ def run_eta(args, rank, world, device):
     from long_context_decoding_eta_b200 import _lib
     _lib.eta_set_decode_engine(args.engine)
     w = workload_by_name(args.workload, args.B)
-    g, dec, W, bias, tau_const = setup(w, device, rank)
+    g, dec, W, bias, tau_const = setup(w, device, rank, args.cent)
     q = g["q"]
     stream = torch.cuda.current_stream()
     # one step to measure densities / bytes, then check status
@@ -321,7 +322,7 @@ def run_eta(args, rank, world, device):
         "config": {
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
             "context": w.ctx, "blk": w.blk, "bound": w.bound, "gate_T": w.gate_T,
-            "tau_mode": w.tau_mode, "engine": args.engine,
+            "tau_mode": w.tau_mode, "engine": args.engine, "centroids": args.cent,
             "density_target": f"{w.density:.2f} {w.density_kind}",
             "union_density": round(by["union_density"], 4),
             "head_density": round(by["head_density"], 4),
@@ -476,6 +477,8 @@ def main():
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     ap.add_argument("--engine", default="auto", choices=["auto", "tcgen05", "fma"],
                     help="decode engine of libeta.so")
+    ap.add_argument("--cent", default="bf16", choices=["f32", "bf16"],
+                    help="storage of the block centroids the screen reads")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

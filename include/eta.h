@@ -69,6 +69,10 @@ typedef struct {
 } eta_dims_t;
 
 typedef enum { ETA_BOUND_EXACT = 0, ETA_BOUND_PROB = 1 } eta_bound_t;
+/* Storage of the block centroids.  ETA_CENT_BF16 halves the bytes the screen reads;
+   the centroid is then rounded to bf16 (nearest even) before rmax and var are
+   measured against it, so the geometric bound stays exact for what is stored. */
+typedef enum { ETA_CENT_F32 = 0, ETA_CENT_BF16 = 1 } eta_cent_format_t;
 typedef enum { ETA_PRUNE_SKIP = 0, ETA_PRUNE_FLOOR = 1 } eta_prune_t;
 
 /* blk_begin value selecting the tail block (the one holding token lengths[b]-1)
@@ -80,8 +84,8 @@ typedef enum { ETA_PRUNE_SKIP = 0, ETA_PRUNE_FLOOR = 1 } eta_prune_t;
  * centroid/variance/max-norm metadata"; abstract: "cached geometric-probabilistic
  * bounds").  For block j of (row b, KV head g) with n_j = clamp(lengths[b] - j*blk,
  * 0, blk) valid keys k_t:
- *   cent_j = (1/n_j) sum_t k_t                       (fp32)
- *   rmax_j >= max_t ||k_t - cent_j||, measured against the stored fp32 cent_j and
+ *   cent_j = (1/n_j) sum_t k_t   (fp32, or rounded to bf16 with ETA_CENT_BF16)
+ *   rmax_j >= max_t ||k_t - cent_j||, measured against the stored cent_j and
  *            rounded up so that the Cauchy-Schwarz bound stays sound in fp32
  *   var_j  = (1/n_j) sum_t ||k_t - cent_j||^2
  *   cnt_j  = n_j;  vsum_j = sum_t v_t (only when vsum != NULL)
@@ -92,15 +96,16 @@ typedef enum { ETA_PRUNE_SKIP = 0, ETA_PRUNE_FLOOR = 1 } eta_prune_t;
  * blk_begin, blk_end: recompute blocks [blk_begin, blk_end) of every row
  *          (blk_end = -1: up to NB); blk_begin = ETA_TAIL_BLOCK: only the tail
  *          block of each row (rows with lengths[b] = 0 are left untouched).
- * cent     fp32 [B, Hkv, d, NB]  (dimension-major per row, for coalesced screening)
+ * cent_format, cent: fp32 or bf16 [B, Hkv, d, NB] (dimension-major per row, for
+ *          coalesced screening)
  * rmax,var fp32 [B, Hkv, NB];  cnt int32 [B, Hkv, NB]
  * vsum     fp32 [B, Hkv, NB, d] or NULL (needed only by ETA_PRUNE_FLOOR)
  */
 eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_bf16_t* K,
                                   const eta_bf16_t* V, const int32_t* lengths,
-                                  int32_t blk_begin, int32_t blk_end, float* cent,
-                                  float* rmax, float* var, int32_t* cnt, float* vsum,
-                                  void* stream);
+                                  int32_t blk_begin, int32_t blk_end,
+                                  eta_cent_format_t cent_format, void* cent, float* rmax,
+                                  float* var, int32_t* cnt, float* vsum, void* stream);
 
 /*
  * eta_predict_tau -- per-query, per-head threshold (review Methodology Assessment,
@@ -123,6 +128,7 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  * "in O(1) time using cached geometric-probabilistic bounds"; co-admission across
  * the query heads of a KV group).
  *   UB[b,h,j] = scale * (q.cent_j + ||q|| * R_j),  q = q[b,h], g = h / G
+ *   (cent in the format eta_build_block_meta stored it)
  *     ETA_BOUND_EXACT: R_j = rmax_j                      (Cauchy-Schwarz, sound)
  *     ETA_BOUND_PROB:  R_j = min(rmax_j, z * sqrt(var_j / d))
  *   admit[b,h,j] = cnt_j > 0 && UB[b,h,j] >= tau[b,h]
@@ -138,7 +144,8 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  */
 size_t eta_screen_workspace_size(const eta_dims_t* dims);
 eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
-                        const float* cent, const float* rmax, const float* var,
+                        eta_cent_format_t cent_format, const void* cent, const float* rmax,
+                        const float* var,
                         const int32_t* cnt, eta_bound_t bound, float z, float scale,
                         uint32_t* head_mask, int32_t* union_idx, int32_t* union_cnt,
                         float* bounds_out, int32_t* head_cnt, void* ws, size_t ws_bytes,

@@ -25,7 +25,8 @@ from . import _lib as L
 class EtaDecoder:
     def __init__(self, K: torch.Tensor, V: torch.Tensor, lengths: torch.Tensor, Hq: int,
                  blk: int, *, bound: str = "exact", z: float = 3.0, T: float = 0.0,
-                 scale: float = 0.0, prune: str = "skip", keep_bounds: bool = False):
+                 scale: float = 0.0, prune: str = "skip", keep_bounds: bool = False,
+                 cent_format: str = "f32"):
         if not K.is_cuda:
             raise ValueError("K/V must be CUDA tensors")
         if K.dtype != torch.bfloat16 or V.dtype != torch.bfloat16:
@@ -41,7 +42,10 @@ class EtaDecoder:
         self.scale = float(scale) if scale else 1.0 / math.sqrt(d)
         dev = K.device
         f32, i32 = torch.float32, torch.int32
-        self.cent = torch.zeros(B, Hkv, d, self.NB, dtype=f32, device=dev)
+        if cent_format not in ("f32", "bf16"):
+            raise ValueError(cent_format)
+        self.cent = torch.zeros(B, Hkv, d, self.NB, device=dev,
+                                dtype=torch.bfloat16 if cent_format == "bf16" else f32)
         self.rmax = torch.zeros(B, Hkv, self.NB, dtype=f32, device=dev)
         self.var = torch.zeros(B, Hkv, self.NB, dtype=f32, device=dev)
         self.cnt = torch.zeros(B, Hkv, self.NB, dtype=i32, device=dev)

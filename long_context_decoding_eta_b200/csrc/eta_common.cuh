@@ -2,6 +2,7 @@
 // waits with an iteration limit, and 1-D TMA bulk copies global -> shared.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 

@@ -6,6 +6,8 @@
 // each key row is one coalesced 128/256-byte warp load.  Blocks live in L2 between
 // the two passes over their keys (16-32 KB each).  Tail refresh (the per-token
 // append): one CTA per block, keys split over its 8 warps.
+#include <type_traits>
+
 #include "eta_common.cuh"
 #include "eta_host.h"
 
@@ -28,11 +30,28 @@ ETA_DEV void load_row(const eta_bf16_t* p, float (&x)[DPL]) {
   }
 }
 
-template <int D>
+// Centroid storage: CF = 0 fp32, CF = 1 bf16.  With bf16 the key sum is accumulated
+// in fp64 (exact for up to 128 bf16 keys of ordinary range), divided in fp64 and
+// rounded once to bf16 (nearest even), so the stored centroid is the correctly
+// rounded mean; rmax and var are then measured against that stored centroid and the
+// bound stays exact for what the screen reads.
+ETA_DEV float bf16_round_from_double(double m) {
+  return __bfloat162float(__double2bfloat16(m));
+}
+
+template <int CF>
+ETA_DEV void store_centroid(void* cent, size_t idx, float c) {
+  if constexpr (CF == 1)
+    reinterpret_cast<uint16_t*>(cent)[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(c));
+  else
+    reinterpret_cast<float*>(cent)[idx] = c;
+}
+
+template <int D, int CF>
 __global__ void __launch_bounds__(kMetaWarps * 32)
 meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restrict__ K,
                   const eta_bf16_t* __restrict__ V, const int32_t* __restrict__ lengths,
-                  int blk_begin, int nblk, int tail, float* __restrict__ cent,
+                  int blk_begin, int nblk, void* __restrict__ cent,
                   float* __restrict__ rmax, float* __restrict__ var, int32_t* __restrict__ cnt,
                   float* __restrict__ vsum, int32_t* status) {
   ETA_PDL_ENTRY();
@@ -45,15 +64,9 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
     if (lane == 0 && warp == 0 && blockIdx.x == 0) set_status(status, ETA_DEVSTAT_BAD_LENGTH);
     len = min(max(len, 0), T_max);
   }
-  int j;
-  if (tail) {
-    if (blockIdx.x != 0 || warp != 0 || len == 0) return;
-    j = (len - 1) / blk;
-  } else {
-    const int jj = blockIdx.x * kMetaWarps + warp;
-    if (jj >= nblk) return;
-    j = blk_begin + jj;
-  }
+  const int jj = blockIdx.x * kMetaWarps + warp;
+  if (jj >= nblk) return;
+  const int j = blk_begin + jj;
   const int n = min(max(len - j * blk, 0), blk);
   const size_t rowj = (size_t)r * NB + j;
   const eta_bf16_t* kb = K + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
@@ -66,25 +79,32 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
   float c[DPL];
 #pragma unroll
   for (int i = 0; i < DPL; ++i) c[i] = 0.f;
-  // pass 1: centroid
+  // pass 1: centroid (fp32 sums, or exact fp64 sums for bf16 storage)
+  using Acc = typename std::conditional<CF == 1, double, float>::type;
+  Acc csum[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) csum[i] = 0;
   for (int w = 0; w < kMetaWarps; ++w) {
     const int lo = min(w * per, n), hi = min(lo + per, n);
-    float pc[DPL];
+    Acc pc[DPL];
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) pc[i] = 0.f;
+    for (int i = 0; i < DPL; ++i) pc[i] = 0;
 #pragma unroll 4
     for (int t = lo; t < hi; ++t) {
       float x[DPL];
       load_row<DPL>(kb + (size_t)t * D, x);
 #pragma unroll
-      for (int i = 0; i < DPL; ++i) pc[i] += x[i];
+      for (int i = 0; i < DPL; ++i) pc[i] += (Acc)x[i];
     }
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) c[i] += pc[i];
+    for (int i = 0; i < DPL; ++i) csum[i] += pc[i];
   }
   if (n > 0) {
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) c[i] = c[i] / (float)n;
+    for (int i = 0; i < DPL; ++i) {
+      if constexpr (CF == 1) c[i] = bf16_round_from_double(csum[i] / (double)n);
+      else c[i] = csum[i] / (float)n;
+    }
   }
   // pass 2: squared distances to the stored fp32 centroid
   float r2max = 0.f, s2 = 0.f;
@@ -107,9 +127,9 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
     }
     s2 += ps;
   }
-  float* cr = cent + (size_t)r * D * NB + j;
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) cr[(size_t)(lane * DPL + i) * NB] = c[i];
+  for (int i = 0; i < DPL; ++i)
+    store_centroid<CF>(cent, ((size_t)r * D + lane * DPL + i) * NB + j, c[i]);
   if (lane == 0) {
     rmax[rowj] = n > 0 ? __fmul_ru(__fsqrt_ru(r2max), kRadiusInflate) : 0.f;
     var[rowj] = n > 0 ? s2 / (float)n : 0.f;
@@ -147,11 +167,11 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
 // split over the 8 warps of a CTA so the latency chain is blk/8 keys instead of blk.
 // The chunk sums are combined in warp order, the same order meta_build_kernel
 // uses, so both kernels give bit-identical metadata for the same block.
-template <int D>
+template <int D, int CF>
 __global__ void __launch_bounds__(kMetaWarps * 32)
 meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restrict__ K,
                  const eta_bf16_t* __restrict__ V, const int32_t* __restrict__ lengths,
-                 float* __restrict__ cent, float* __restrict__ rmax, float* __restrict__ var,
+                 void* __restrict__ cent, float* __restrict__ rmax, float* __restrict__ var,
                  int32_t* __restrict__ cnt, float* __restrict__ vsum) {
   ETA_PDL_ENTRY();
   constexpr int DPL = D / 32;
@@ -168,24 +188,28 @@ meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restri
   const size_t rowj = (size_t)r * NB + j;
   const eta_bf16_t* kb = K + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
 
+  using Acc = typename std::conditional<CF == 1, double, float>::type;
+  __shared__ Acc cpart[kMetaWarps][D];
   float c[DPL];
+  Acc pc[DPL];
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) c[i] = 0.f;
+  for (int i = 0; i < DPL; ++i) pc[i] = 0;
   for (int t = t_lo; t < t_hi; ++t) {
     float x[DPL];
     load_row<DPL>(kb + (size_t)t * D, x);
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) c[i] += x[i];
+    for (int i = 0; i < DPL; ++i) pc[i] += (Acc)x[i];
   }
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) part[warp][lane * DPL + i] = c[i];
+  for (int i = 0; i < DPL; ++i) cpart[warp][lane * DPL + i] = pc[i];
   __syncthreads();
 #pragma unroll
   for (int i = 0; i < DPL; ++i) {
-    float s = 0.f;
+    Acc sum = 0;
 #pragma unroll
-    for (int w = 0; w < kMetaWarps; ++w) s += part[w][lane * DPL + i];
-    c[i] = s / (float)n;
+    for (int w = 0; w < kMetaWarps; ++w) sum += cpart[w][lane * DPL + i];
+    if constexpr (CF == 1) c[i] = bf16_round_from_double(sum / (double)n);
+    else c[i] = sum / (float)n;
   }
   float r2max = 0.f, s2 = 0.f;
   for (int t = t_lo; t < t_hi; ++t) {
@@ -206,9 +230,9 @@ meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restri
     red_sum[warp] = s2;
   }
   if (warp == 0) {
-    float* cr = cent + (size_t)r * D * NB + j;
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) cr[(size_t)(lane * DPL + i) * NB] = c[i];
+    for (int i = 0; i < DPL; ++i)
+      store_centroid<CF>(cent, ((size_t)r * D + lane * DPL + i) * NB + j, c[i]);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -250,18 +274,34 @@ meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restri
   }
 }
 
+template <int D, int CF>
+static eta_status_t launch_meta(bool tail, const eta_dims_t* dims, int NB, int R, int blk_begin,
+                                int nblk, const eta_bf16_t* K, const eta_bf16_t* V,
+                                const int32_t* lengths, void* cent, float* rmax, float* var,
+                                int32_t* cnt, float* vsum, cudaStream_t s) {
+  if (tail)
+    return launch_k(meta_tail_kernel<D, CF>, dim3(R), dim3(kMetaWarps * 32), 0, s, dims->Hkv,
+                    dims->T_max, dims->blk, NB, K, V, lengths, cent, rmax, var, cnt, vsum);
+  dim3 grid((nblk + kMetaWarps - 1) / kMetaWarps, R);
+  return launch_k(meta_build_kernel<D, CF>, grid, dim3(kMetaWarps * 32), 0, s, dims->Hkv,
+                  dims->T_max, dims->blk, NB, K, V, lengths, blk_begin, nblk, cent, rmax, var,
+                  cnt, vsum, (int32_t*)nullptr);
+}
+
 }  // namespace eta
 
 using namespace eta;
 
 extern "C" eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_bf16_t* K,
                                              const eta_bf16_t* V, const int32_t* lengths,
-                                             int32_t blk_begin, int32_t blk_end, float* cent,
+                                             int32_t blk_begin, int32_t blk_end,
+                                             eta_cent_format_t cent_format, void* cent,
                                              float* rmax, float* var, int32_t* cnt, float* vsum,
                                              void* stream) {
   eta_status_t st = check_dims(dims);
   if (st != ETA_OK) return st;
   if (!K || !lengths || !cent || !rmax || !var || !cnt) return ETA_ERR_INVALID_ARG;
+  if (cent_format != ETA_CENT_F32 && cent_format != ETA_CENT_BF16) return ETA_ERR_INVALID_ARG;
   if (vsum && !V) return ETA_ERR_INVALID_ARG;
   if (!aligned16(K) || (V && !aligned16(V))) return ETA_ERR_INVALID_ARG;
   const int NB = num_blocks(dims);
@@ -275,14 +315,14 @@ extern "C" eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_b
     if (nblk == 0) return ETA_OK;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (tail) {
-    auto kern = dims->d == 128 ? meta_tail_kernel<128> : meta_tail_kernel<64>;
-    return launch_k(kern, dim3(R), dim3(kMetaWarps * 32), 0, s, dims->Hkv, dims->T_max,
-                    dims->blk, NB, K, V, lengths, cent, rmax, var, cnt, vsum);
-  }
-  dim3 grid((nblk + kMetaWarps - 1) / kMetaWarps, R);
-  auto kern = dims->d == 128 ? meta_build_kernel<128> : meta_build_kernel<64>;
-  return launch_k(kern, grid, dim3(kMetaWarps * 32), 0, s, dims->Hkv, dims->T_max, dims->blk,
-                  NB, K, V, lengths, blk_begin, nblk, 0, cent, rmax, var, cnt, vsum,
-                  (int32_t*)nullptr);
+  const bool bf = cent_format == ETA_CENT_BF16;
+  if (dims->d == 128)
+    return bf ? launch_meta<128, 1>(tail, dims, NB, R, blk_begin, nblk, K, V, lengths, cent, rmax,
+                                   var, cnt, vsum, s)
+              : launch_meta<128, 0>(tail, dims, NB, R, blk_begin, nblk, K, V, lengths, cent, rmax,
+                                   var, cnt, vsum, s);
+  return bf ? launch_meta<64, 1>(tail, dims, NB, R, blk_begin, nblk, K, V, lengths, cent, rmax,
+                                var, cnt, vsum, s)
+            : launch_meta<64, 0>(tail, dims, NB, R, blk_begin, nblk, K, V, lengths, cent, rmax,
+                                var, cnt, vsum, s);
 }

@@ -11,6 +11,8 @@
 //   head's 32-bit admit word directly; the union word is their OR.
 // compact_kernel: one CTA per (row, KV head) turns union words into the ascending
 //   list of admitted block indices (popcount prefix over words, lane = bit).
+#include <type_traits>
+
 #include "eta_common.cuh"
 #include "eta_host.h"
 
@@ -19,10 +21,16 @@ namespace eta {
 constexpr int kScreenWarps = 8;
 constexpr int kCompactThreads = 256;
 
-template <int D, int G>
+template <int CF>
+ETA_DEV float load_cent(const void* cent, size_t i) {
+  if constexpr (CF == 1) return bf16_to_f(__ldg(reinterpret_cast<const uint16_t*>(cent) + i));
+  else return __ldg(reinterpret_cast<const float*>(cent) + i);
+}
+
+template <int D, int G, int CF>
 __global__ void __launch_bounds__(kScreenWarps * 32)
 screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
-              const float* __restrict__ tau, const float* __restrict__ cent,
+              const float* __restrict__ tau, const void* __restrict__ cent,
               const float* __restrict__ rmax, const float* __restrict__ var,
               const int32_t* __restrict__ cnt, int bound, float z, float scale,
               uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
@@ -54,13 +62,13 @@ screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
   if (w >= NW) return;
   const int j = w * 32 + lane;
   const bool vj = j < NB;
-  const float* cp = cent + (size_t)r * D * NB + (vj ? j : 0);
+  const size_t c0 = (size_t)r * D * NB + (vj ? j : 0);
   float acc[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) acc[h] = 0.f;
 #pragma unroll 16
   for (int k = 0; k < D; ++k) {
-    const float c = vj ? __ldg(cp + (size_t)k * NB) : 0.f;
+    const float c = vj ? load_cent<CF>(cent, c0 + (size_t)k * NB) : 0.f;
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = fmaf(qs[k * G + h], c, acc[h]);
   }
@@ -81,24 +89,27 @@ screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
   if (lane == 0) union_words[(size_t)r * NW + w] = uni;
 }
 
-// Vector form for NB % 4 == 0: lane l of a warp owns the 4 consecutive blocks
-// 4l..4l+3 of a 128-block group, so each of the d loads of a lane is one 16-byte
-// load and a warp moves 512 bytes per dimension.  A warp's four 32-bit admit words
-// per head are assembled from the lanes' 4-bit nibbles with an OR butterfly over
-// groups of 8 lanes.  Each warp walks kGroupsPerWarp groups so that the per-CTA
-// prologue (the group's queries in shared memory, their norms) is amortized.
-constexpr int kGroupsPerWarp = 1;
-constexpr int kScreen4Warps = 4;
+// Vector form: lane l of a warp owns VW = 4 consecutive blocks, so each of the d
+// loads of a lane is one 16-byte (fp32 centroids) or 8-byte (bf16) load and a warp
+// covers a group of 128 blocks.
+// The lanes' VW-bit admit chunks are assembled into 32-bit words with an OR
+// butterfly over the 32 / VW lanes of each word.  Needs NB % VW == 0 and 16-byte
+// aligned metadata.
+constexpr int kScreenVecWarps = 4;
+constexpr int kLoadBatch = 16;   // independent 16-byte loads in flight per lane
 
-template <int D, int G>
-__global__ void __launch_bounds__(kScreen4Warps * 32)
-screen4_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
-               const float* __restrict__ tau, const float* __restrict__ cent,
-               const float* __restrict__ rmax, const float* __restrict__ var,
-               const int32_t* __restrict__ cnt, int bound, float z, float scale,
-               uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
-               float* __restrict__ bounds_out) {
+template <int D, int G, int CF>
+__global__ void __launch_bounds__(kScreenVecWarps * 32)
+screen_vec_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
+                  const float* __restrict__ tau, const void* __restrict__ cent,
+                  const float* __restrict__ rmax, const float* __restrict__ var,
+                  const int32_t* __restrict__ cnt, int bound, float z, float scale,
+                  uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
+                  float* __restrict__ bounds_out) {
   ETA_PDL_ENTRY();
+  constexpr int VW = 4;                         // blocks per lane
+  constexpr int GB = 32 * VW;                   // blocks per warp group
+  constexpr int LPW = 32 / VW;                  // lanes per 32-bit word
   __shared__ __align__(16) float qs[D * G];
   __shared__ float qn[G], ts[G];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -110,7 +121,7 @@ screen4_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q
     qs[k * G + h] = bf16_to_f(q[(qhead0 + h) * D + k]);
   }
   __syncthreads();
-  for (int h = warp; h < G; h += kScreen4Warps) {
+  for (int h = warp; h < G; h += kScreenVecWarps) {
     float s = 0.f;
     for (int k = lane; k < D; k += 32) s = fmaf(qs[k * G + h], qs[k * G + h], s);
     s = warp_sum(s);
@@ -121,79 +132,90 @@ screen4_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q
   }
   __syncthreads();
 
-  const int ngroups = (NB + 127) / 128;
-  for (int it = 0; it < kGroupsPerWarp; ++it) {
-    const int grp = (blockIdx.x * kScreen4Warps + warp) * kGroupsPerWarp + it;
-    if (grp >= ngroups) return;
-    const int j0 = grp * 128 + lane * 4;
-    const bool vj = j0 < NB;                       // NB % 4 == 0: all 4 valid or none
-    const float4* cp = reinterpret_cast<const float4*>(cent + (size_t)r * D * NB + (vj ? j0 : 0));
-    const size_t rowq = (size_t)NB / 4;            // float4 stride between dimensions
-    float acc[4][G];
+  const int grp = blockIdx.x * kScreenVecWarps + warp;
+  if (grp * GB >= NB) return;
+  const int j0 = grp * GB + lane * VW;
+  const bool vj = j0 < NB;                      // NB % VW == 0: all VW valid or none
+  // one load per dimension: 4 centroids = 16 bytes (fp32) or 8 bytes (bf16)
+  using LdT = typename std::conditional<CF == 1, uint2, uint4>::type;
+  const size_t rowv = (size_t)NB / 4;           // LdT units per dimension
+  const LdT* cp = reinterpret_cast<const LdT*>(
+      reinterpret_cast<const unsigned char*>(cent) + ((size_t)r * D * NB + (vj ? j0 : 0)) *
+                                                        (CF == 1 ? 2 : 4));
+  float acc[VW][G];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
+  for (int k = 0; k < VW; ++k)
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[k][h] = 0.f;
-    // batches of kLoadBatch independent 16-byte loads in flight per lane
-    constexpr int kLoadBatch = 16;
+    for (int h = 0; h < G; ++h) acc[k][h] = 0.f;
 #pragma unroll 1
-    for (int d0 = 0; d0 < D; d0 += kLoadBatch) {
-      float4 cb[kLoadBatch];
+  for (int d0 = 0; d0 < D; d0 += kLoadBatch) {
+    LdT cb[kLoadBatch];
 #pragma unroll
-      for (int u = 0; u < kLoadBatch; ++u)
-        cb[u] = vj ? __ldg(cp + (size_t)(d0 + u) * rowq) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kLoadBatch; ++u)
+      cb[u] = vj ? __ldg(cp + (size_t)(d0 + u) * rowv) : LdT{};
 #pragma unroll
-      for (int u = 0; u < kLoadBatch; ++u) {
+    for (int u = 0; u < kLoadBatch; ++u) {
+      float cv[VW];
+      if constexpr (CF == 1) {
+        cv[0] = bf16_lo(cb[u].x); cv[1] = bf16_hi(cb[u].x); cv[2] = bf16_lo(cb[u].y);
+        cv[3] = bf16_hi(cb[u].y);
+      } else {
+        cv[0] = __uint_as_float(cb[u].x); cv[1] = __uint_as_float(cb[u].y);
+        cv[2] = __uint_as_float(cb[u].z); cv[3] = __uint_as_float(cb[u].w);
+      }
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float qv = qs[(d0 + u) * G + h];
-          acc[0][h] = fmaf(qv, cb[u].x, acc[0][h]);
-          acc[1][h] = fmaf(qv, cb[u].y, acc[1][h]);
-          acc[2][h] = fmaf(qv, cb[u].z, acc[2][h]);
-          acc[3][h] = fmaf(qv, cb[u].w, acc[3][h]);
-        }
+      for (int h = 0; h < G; ++h) {
+        const float qv = qs[(d0 + u) * G + h];
+#pragma unroll
+        for (int k = 0; k < VW; ++k) acc[k][h] = fmaf(qv, cv[k], acc[k][h]);
       }
     }
-    const size_t rj = (size_t)r * NB + j0;
-    float rad[4] = {0.f, 0.f, 0.f, 0.f};
-    int n[4] = {0, 0, 0, 0};
-    if (vj) {
-      const float4 rr = __ldg(reinterpret_cast<const float4*>(rmax + rj));
-      const int4 cc = __ldg(reinterpret_cast<const int4*>(cnt + rj));
-      rad[0] = rr.x; rad[1] = rr.y; rad[2] = rr.z; rad[3] = rr.w;
-      n[0] = cc.x; n[1] = cc.y; n[2] = cc.z; n[3] = cc.w;
-      if (bound == ETA_BOUND_PROB) {
-        const float4 vv = __ldg(reinterpret_cast<const float4*>(var + rj));
-        rad[0] = fminf(rad[0], z * sqrtf(vv.x / (float)D));
-        rad[1] = fminf(rad[1], z * sqrtf(vv.y / (float)D));
-        rad[2] = fminf(rad[2], z * sqrtf(vv.z / (float)D));
-        rad[3] = fminf(rad[3], z * sqrtf(vv.w / (float)D));
-      }
-    }
-    uint32_t uni = 0;
-    const int wsel = lane >> 3;                    // word of the group this lane's nibble lands in
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      uint32_t nib = 0;
-      float ubv[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        ubv[k] = scale * fmaf(qn[h], rad[k], acc[k][h]);
-        if (vj && n[k] > 0 && ubv[k] >= ts[h]) nib |= 1u << k;
-      }
-      if (bounds_out && vj)
-        *reinterpret_cast<float4*>(bounds_out + (qhead0 + h) * NB + j0) =
-            make_float4(ubv[0], ubv[1], ubv[2], ubv[3]);
-      uint32_t word = nib << (4 * (lane & 7));
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      word |= __shfl_xor_sync(0xffffffffu, word, 4);
-      // lanes 8w..8w+7 now hold word w of the group
-      if ((lane & 7) == 0 && grp * 4 + wsel < NW) head_mask[(qhead0 + h) * NW + grp * 4 + wsel] = word;
-      uni |= word;
-    }
-    if ((lane & 7) == 0 && grp * 4 + wsel < NW) union_words[(size_t)r * NW + grp * 4 + wsel] = uni;
   }
+  const size_t rj = (size_t)r * NB + j0;
+  float rad[VW];
+  int n[VW];
+#pragma unroll
+  for (int k = 0; k < VW; ++k) { rad[k] = 0.f; n[k] = 0; }
+  if (vj) {
+#pragma unroll
+    for (int v = 0; v < VW / 4; ++v) {
+      const float4 rr = __ldg(reinterpret_cast<const float4*>(rmax + rj) + v);
+      const int4 cc = __ldg(reinterpret_cast<const int4*>(cnt + rj) + v);
+      rad[4 * v] = rr.x; rad[4 * v + 1] = rr.y; rad[4 * v + 2] = rr.z; rad[4 * v + 3] = rr.w;
+      n[4 * v] = cc.x; n[4 * v + 1] = cc.y; n[4 * v + 2] = cc.z; n[4 * v + 3] = cc.w;
+      if (bound == ETA_BOUND_PROB) {
+        const float4 vv = __ldg(reinterpret_cast<const float4*>(var + rj) + v);
+        rad[4 * v] = fminf(rad[4 * v], z * sqrtf(vv.x / (float)D));
+        rad[4 * v + 1] = fminf(rad[4 * v + 1], z * sqrtf(vv.y / (float)D));
+        rad[4 * v + 2] = fminf(rad[4 * v + 2], z * sqrtf(vv.z / (float)D));
+        rad[4 * v + 3] = fminf(rad[4 * v + 3], z * sqrtf(vv.w / (float)D));
+      }
+    }
+  }
+  uint32_t uni = 0;
+  const int wsel = grp * VW + lane / LPW;        // word index of this lane's chunk
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    uint32_t bits = 0;
+    float ubv[VW];
+#pragma unroll
+    for (int k = 0; k < VW; ++k) {
+      ubv[k] = scale * fmaf(qn[h], rad[k], acc[k][h]);
+      if (vj && n[k] > 0 && ubv[k] >= ts[h]) bits |= 1u << k;
+    }
+    if (bounds_out && vj) {
+#pragma unroll
+      for (int v = 0; v < VW / 4; ++v)
+        reinterpret_cast<float4*>(bounds_out + (qhead0 + h) * NB + j0)[v] =
+            make_float4(ubv[4 * v], ubv[4 * v + 1], ubv[4 * v + 2], ubv[4 * v + 3]);
+    }
+    uint32_t word = bits << (VW * (lane % LPW));
+#pragma unroll
+    for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+    if (lane % LPW == 0 && wsel < NW) head_mask[(qhead0 + h) * NW + wsel] = word;
+    uni |= word;
+  }
+  if (lane % LPW == 0 && wsel < NW) union_words[(size_t)r * NW + wsel] = uni;
 }
 
 __global__ void __launch_bounds__(kCompactThreads)
@@ -250,24 +272,24 @@ compact_kernel(int Hq, int Hkv, int G, int NB, int NW, const uint32_t* __restric
   }
 }
 
-template <int D>
+template <int D, int CF>
 static eta_status_t launch_screen(bool vec, int G, dim3 grid, cudaStream_t s, int Hq, int Hkv,
                                   int NB, int NW, const eta_bf16_t* q, const float* tau,
-                                  const float* cent, const float* rmax, const float* var,
+                                  const void* cent, const float* rmax, const float* var,
                                   const int32_t* cnt, int bound, float z, float scale,
                                   uint32_t* head_mask, uint32_t* uw, float* bounds_out) {
-  using KernT = void (*)(int, int, int, int, const eta_bf16_t*, const float*, const float*,
+  using KernT = void (*)(int, int, int, int, const eta_bf16_t*, const float*, const void*,
                          const float*, const float*, const int32_t*, int, float, float,
                          uint32_t*, uint32_t*, float*);
   KernT kern = nullptr;
   switch (G) {
-    case 1: kern = vec ? screen4_kernel<D, 1> : screen_kernel<D, 1>; break;
-    case 2: kern = vec ? screen4_kernel<D, 2> : screen_kernel<D, 2>; break;
-    case 4: kern = vec ? screen4_kernel<D, 4> : screen_kernel<D, 4>; break;
-    case 8: kern = vec ? screen4_kernel<D, 8> : screen_kernel<D, 8>; break;
+    case 1: kern = vec ? screen_vec_kernel<D, 1, CF> : screen_kernel<D, 1, CF>; break;
+    case 2: kern = vec ? screen_vec_kernel<D, 2, CF> : screen_kernel<D, 2, CF>; break;
+    case 4: kern = vec ? screen_vec_kernel<D, 4, CF> : screen_kernel<D, 4, CF>; break;
+    case 8: kern = vec ? screen_vec_kernel<D, 8, CF> : screen_kernel<D, 8, CF>; break;
     default: return ETA_ERR_UNSUPPORTED;
   }
-  const dim3 block((vec ? kScreen4Warps : kScreenWarps) * 32);
+  const dim3 block((vec ? kScreenVecWarps : kScreenWarps) * 32);
   return launch_k(kern, grid, block, 0, s, Hq, Hkv, NB, NW, q, tau, cent, rmax, var, cnt, bound,
                   z, scale, head_mask, uw, bounds_out);
 }
@@ -282,7 +304,8 @@ extern "C" size_t eta_screen_workspace_size(const eta_dims_t* dims) {
 }
 
 extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
-                                   const float* cent, const float* rmax, const float* var,
+                                   eta_cent_format_t cent_format, const void* cent,
+                                   const float* rmax, const float* var,
                                    const int32_t* cnt, eta_bound_t bound, float z, float scale,
                                    uint32_t* head_mask, int32_t* union_idx, int32_t* union_cnt,
                                    float* bounds_out, int32_t* head_cnt, void* ws,
@@ -293,6 +316,7 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   if (!q || !tau || !cent || !rmax || !cnt || !head_mask || !union_idx || !union_cnt)
     return ETA_ERR_INVALID_ARG;
   if (bound != ETA_BOUND_EXACT && bound != ETA_BOUND_PROB) return ETA_ERR_INVALID_ARG;
+  if (cent_format != ETA_CENT_F32 && cent_format != ETA_CENT_BF16) return ETA_ERR_INVALID_ARG;
   if (bound == ETA_BOUND_PROB && (!var || !(z >= 0.f))) return ETA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < eta_screen_workspace_size(dims)) return ETA_ERR_WORKSPACE;
   if (scale == 0.f) scale = 1.f / sqrtf((float)dims->d);
@@ -300,21 +324,24 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   const int R = dims->B * dims->Hkv, G = dims->Hq / dims->Hkv;
   uint32_t* uw = static_cast<uint32_t*>(ws);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool vec = (NB % 4 == 0) && aligned16(cent) && aligned16(rmax) && aligned16(cnt) &&
+  const bool bf = cent_format == ETA_CENT_BF16;
+  const int VW = 4;
+  const bool vec = (NB % VW == 0) && aligned16(cent) && aligned16(rmax) && aligned16(cnt) &&
                    (!var || aligned16(var)) && (!bounds_out || aligned16(bounds_out));
   dim3 grid;
   if (vec) {
-    const int ngroups = (NB + 127) / 128;
-    const int per_cta = kScreen4Warps * kGroupsPerWarp;
-    grid = dim3((ngroups + per_cta - 1) / per_cta, R);
+    const int ngroups = (NB + 32 * VW - 1) / (32 * VW);
+    grid = dim3((ngroups + kScreenVecWarps - 1) / kScreenVecWarps, R);
   } else {
     grid = dim3((NW + kScreenWarps - 1) / kScreenWarps, R);
   }
-  st = dims->d == 128
-           ? launch_screen<128>(vec, G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax,
-                                var, cnt, (int)bound, z, scale, head_mask, uw, bounds_out)
-           : launch_screen<64>(vec, G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax,
-                               var, cnt, (int)bound, z, scale, head_mask, uw, bounds_out);
+#define ETA_SCREEN_ARGS vec, G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, \
+                        cnt, (int)bound, z, scale, head_mask, uw, bounds_out
+  if (dims->d == 128)
+    st = bf ? launch_screen<128, 1>(ETA_SCREEN_ARGS) : launch_screen<128, 0>(ETA_SCREEN_ARGS);
+  else
+    st = bf ? launch_screen<64, 1>(ETA_SCREEN_ARGS) : launch_screen<64, 0>(ETA_SCREEN_ARGS);
+#undef ETA_SCREEN_ARGS
   if (st != ETA_OK) return st;
   return launch_k(compact_kernel, dim3(R), dim3(kCompactThreads), 0, s, dims->Hq, dims->Hkv, G,
                   NB, NW, (const uint32_t*)uw, (const uint32_t*)head_mask, union_idx, union_cnt,

@@ -52,13 +52,24 @@ def default_scale(d: int) -> float:
 # ----------------------------------------------------------------------------
 # (1) per-block metadata  [review-sum; abstract: "cached ... bounds"]
 # ----------------------------------------------------------------------------
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (8 significant bits), ties to
+    even.  Written from the definition of the format: x = m * 2**e, 0.5 <= |m| < 1,
+    keep m to 8 bits.  (Normal range only, which is all the metadata needs.)"""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.round(m * 256.0) / 256.0, e)
+
+
 def block_meta(K_seq: np.ndarray, n_valid: int, blk: int,
-               V_seq: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+               V_seq: Optional[np.ndarray] = None,
+               cent_format: str = "f32") -> Dict[str, np.ndarray]:
     """Metadata of every block of one (batch row, KV head) key sequence.
 
     K_seq: [T_max, d] float64; keys t < n_valid are valid.
     Block j holds keys [j*blk, min((j+1)*blk, n_valid)).  For its n_j valid keys:
-      cent_j = mean of the keys
+      cent_j = mean of the keys (cent_format "bf16": the mean rounded to bf16,
+               the centroid the compact metadata stores)
       rmax_j = max_t ||k_t - cent_j||            (max deviation norm)
       var_j  = (1/n_j) sum_t ||k_t - cent_j||^2  (total variance, one scalar)
       cnt_j  = n_j
@@ -80,6 +91,8 @@ def block_meta(K_seq: np.ndarray, n_valid: int, blk: int,
             continue
         keys = K_seq[lo:hi]
         c = keys.mean(axis=0)
+        if cent_format == "bf16":
+            c = round_to_bf16(c)
         dist = np.sqrt(((keys - c) ** 2).sum(axis=1))
         cent[j] = c
         rmax[j] = dist.max()
@@ -94,11 +107,11 @@ def block_meta(K_seq: np.ndarray, n_valid: int, blk: int,
 
 
 def cache_meta(K: np.ndarray, lengths: Sequence[int], blk: int,
-               V: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+               V: Optional[np.ndarray] = None, cent_format: str = "f32") -> Dict[str, np.ndarray]:
     """block_meta over a whole cache K [B, Hkv, T_max, d] -> arrays [B, Hkv, NB, ...]."""
     B, Hkv = K.shape[:2]
     rows = [[block_meta(K[b, h], int(lengths[b]), blk,
-                        None if V is None else V[b, h]) for h in range(Hkv)]
+                        None if V is None else V[b, h], cent_format) for h in range(Hkv)]
             for b in range(B)]
     keys = rows[0][0].keys()
     return {k: np.stack([np.stack([rows[b][h][k] for h in range(Hkv)]) for b in range(B)])

@@ -147,8 +147,8 @@ def compare_step(gpu: Dict[str, np.ndarray], ref_tau: np.ndarray, ref_sc, ref_o,
 
 
 def oracle_step(K64, V64, q64, L, W64, bias, blk, scale, T, bound="exact", z=3.0,
-                prune="skip", tau_const=None):
-    meta = O.cache_meta(K64, L, blk, V64 if prune == "floor" else None)
+                prune="skip", tau_const=None, cent_format="f32"):
+    meta = O.cache_meta(K64, L, blk, V64 if prune == "floor" else None, cent_format)
     if tau_const is None:
         tau = O.predict_tau(q64, W64, bias)
     else:
@@ -158,11 +158,12 @@ def oracle_step(K64, V64, q64, L, W64, bias, blk, scale, T, bound="exact", z=3.0
     return meta, tau, sc, o, lse
 
 
-def density_bias(K64, q64, L, W64, blk, scale, G, density, kind, bound="exact", z=3.0):
+def density_bias(K64, q64, L, W64, blk, scale, G, density, kind, bound="exact", z=3.0,
+                 cent_format="f32"):
     """Per-head bias that makes the predictor hit a density target on the given
     rows (oracle arithmetic only): bias_h = offset such that tau = qW + bias admits
     the target fraction of (head, block) or (group, block) pairs."""
-    meta = O.cache_meta(K64, L, blk)
+    meta = O.cache_meta(K64, L, blk, cent_format=cent_format)
     tau0 = O.predict_tau(q64, W64, np.zeros(q64.shape[1]))
     ub = O.screen(q64, tau0, meta, scale, bound, z)["bounds"]
     valid = np.repeat(meta["cnt"] > 0, G, axis=1)

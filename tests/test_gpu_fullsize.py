@@ -23,13 +23,13 @@ def rows_f64(t, rows):
     return t[rows].double().cpu().numpy()
 
 
-def sampled_oracle_bias(w, g, rows, scale):
+def sampled_oracle_bias(w, g, rows, scale, cent_format="f32"):
     """Threshold offset from the oracle on the sampled rows (density target of the
     workload), so that no input of the comparison comes from the CUDA path."""
     K64 = rows_f64(g["K"], rows)
     q64 = rows_f64(g["q"], rows)
     L64 = g["lengths"][rows].cpu().numpy()
-    meta = O.cache_meta(K64, L64, w.blk)
+    meta = O.cache_meta(K64, L64, w.blk, cent_format=cent_format)
     W64 = g["W"].double().cpu().numpy()
     tau0 = O.predict_tau(q64, W64, np.zeros(w.Hq))
     ub = O.screen(q64, tau0, meta, scale, w.bound, w.z)["bounds"]
@@ -53,15 +53,15 @@ def whole_batch_properties(dec, gpu, w):
     return un.mean()
 
 
-def run_fullsize(w, rows, tau_const=None, engine="auto"):
+def run_fullsize(w, rows, tau_const=None, engine="auto", cent_format="f32"):
     L.eta_set_decode_engine(engine)
     scale = 1.0 / math.sqrt(w.d)
     g = synth.generate(w, "cuda")
     dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, bound=w.bound, z=w.z,
-                     T=w.gate_T, keep_bounds=True)
+                     T=w.gate_T, keep_bounds=True, cent_format=cent_format)
     dec.build_meta()
     if tau_const is None:
-        bias = sampled_oracle_bias(w, g, rows, scale)
+        bias = sampled_oracle_bias(w, g, rows, scale, cent_format)
         gpu = run_cuda(dec, g["q"], g["W"], torch.full((w.Hq,), bias, device="cuda"))
         b64 = np.full(w.Hq, bias)
     else:
@@ -72,7 +72,7 @@ def run_fullsize(w, rows, tau_const=None, engine="auto"):
     # oracle on the sampled rows
     K64, V64, q64 = rows_f64(g["K"], rows), rows_f64(g["V"], rows), rows_f64(g["q"], rows)
     L64 = g["lengths"][rows].cpu().numpy()
-    meta = O.cache_meta(K64, L64, w.blk)
+    meta = O.cache_meta(K64, L64, w.blk, cent_format=cent_format)
     if tau_const is None:
         tau = O.predict_tau(q64, g["W"].double().cpu().numpy(), b64)
     else:
@@ -89,10 +89,10 @@ def run_fullsize(w, rows, tau_const=None, engine="auto"):
     return rep, union_density
 
 
-@pytest.mark.parametrize("engine", ["auto", "fma"])
-def test_long_128k_b64_union16(engine):
+@pytest.mark.parametrize("engine,cent", [("auto", "f32"), ("fma", "f32"), ("auto", "bf16")])
+def test_long_128k_b64_union16(engine, cent):
     w = synth.LONG128K
-    rep, dens = run_fullsize(w, rows=[0, 37, 63], engine=engine)
+    rep, dens = run_fullsize(w, rows=[0, 37, 63], engine=engine, cent_format=cent)
     # the density target is set on the 3 sampled rows only; across the batch it
     # varies with the rows' thresholds: require real pruning and real admission
     assert 0.01 < dens < 0.6, dens

@@ -38,7 +38,7 @@ def to_dev(g):
 
 
 def full_parity(w, *, lengths=None, prune="skip", T=None, bound=None, z=None, density=None,
-                kind=None, seed=None, tau_const=None):
+                kind=None, seed=None, tau_const=None, cent_format="f32"):
     T = w.gate_T if T is None else T
     bound = w.bound if bound is None else bound
     z = w.z if z is None else z
@@ -49,16 +49,16 @@ def full_parity(w, *, lengths=None, prune="skip", T=None, bound=None, z=None, de
     L = g["lengths"].numpy().astype(np.int64)
     scale = 1.0 / math.sqrt(w.d)
     bias = np.full(w.Hq, density_bias(K64, q64, L, W64, w.blk, scale, w.G, density, kind,
-                                      bound, z))
+                                      bound, z, cent_format))
     gd = to_dev(g)
     dec = EtaDecoder(gd["K"], gd["V"], gd["lengths"], w.Hq, w.blk, bound=bound, z=z, T=T,
-                     prune=prune, keep_bounds=True)
+                     prune=prune, keep_bounds=True, cent_format=cent_format)
     dec.build_meta()
     bias_t = torch.tensor(bias, dtype=torch.float32, device=DEV)
     tc = None if tau_const is None else torch.tensor(tau_const, dtype=torch.float32, device=DEV)
     gpu = run_cuda(dec, gd["q"], gd["W"], bias_t, tc)
     meta, tau, sc, o, lse = oracle_step(K64, V64, q64, L, W64, bias, w.blk, scale, T, bound, z,
-                                        prune, tau_const)
+                                        prune, tau_const, cent_format)
     check_meta(gpu_meta(dec), meta)
     rep = compare_step(gpu, tau, sc, o, lse, q64, K64, V64, L, w.blk, scale, T, w.G)
     return rep, gpu, sc
@@ -154,11 +154,13 @@ def test_tau_above_every_score_gives_uniform_mean():
             assert abs(gpu["lse"][b, h] - math.log(4096)) < 1e-5
 
 
-def test_tail_append_update_matches_rebuild():
+@pytest.mark.parametrize("cent_format", ["f32", "bf16"])
+def test_tail_append_update_matches_rebuild(cent_format):
     w = synth.MID.with_(B=3, ctx=4096, needles=0, seed=83)
     lengths = torch.tensor([4000, 4095, 100], dtype=torch.int32)
     g = to_dev(make(w, lengths=lengths))
-    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, prune="floor")
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, prune="floor",
+                     cent_format=cent_format)
     dec.build_meta()
     # append one token per row and update only the tail blocks
     for b in range(w.B):
@@ -172,7 +174,8 @@ def test_tail_append_update_matches_rebuild():
     full = gpu_meta(dec)
     for k in full:
         assert np.array_equal(inc[k], full[k]), k
-    o_meta = O.cache_meta(f64(dec.K), dec.lengths.cpu().numpy(), w.blk, f64(dec.V))
+    o_meta = O.cache_meta(f64(dec.K), dec.lengths.cpu().numpy(), w.blk, f64(dec.V),
+                          cent_format)
     check_meta(full, o_meta)
 
 
@@ -235,3 +238,16 @@ def test_bounded_wait_times_out_with_status_and_context_survives():
     assert L.eta_status_from_device(int(status.item())) == 5
     # the context is still usable: a normal decode runs and matches the oracle
     rep, gpu, sc = full_parity(synth.TINY.with_(seed=86))
+
+
+@pytest.mark.parametrize("d,G,blk,ctx", [(128, 4, 64, 8192), (128, 4, 64, 3000), (64, 8, 128, 4096),
+                                          (128, 2, 128, 5000)])
+def test_bf16_centroids(d, G, blk, ctx):
+    """Compact metadata: centroids rounded to bf16, radii measured against them
+    (vector screen when NB % 8 == 0, scalar otherwise)."""
+    w = synth.Workload("bf16cent", B=3, Hq=2 * G, Hkv=2, d=d, ctx=ctx, blk=blk, n_clusters=16,
+                       seg=200, needles=2, gate_T=0.0, density=0.3, density_kind="head",
+                       q_scale=4.0, seed=300 + d + G + blk)
+    rep, gpu, sc = full_parity(w, cent_format="bf16")
+    for prune in ("skip", "floor"):
+        full_parity(w, cent_format="bf16", prune=prune, bound="prob", z=2.0)

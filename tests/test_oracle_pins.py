@@ -445,3 +445,41 @@ def test_hand_derived_example():
                       O.PRUNE_FLOOR, meta)
     np.testing.assert_allclose(o[0, 0], want["o_floor"], atol=1e-15)
     assert abs(lse[0, 0] - want["lse_floor"]) < 1e-14
+
+
+# --------------------------------------------------------------------------
+# bf16 centroids (compact metadata)
+# --------------------------------------------------------------------------
+def test_round_to_bf16_matches_torch_on_float32_inputs():
+    rng = np.random.default_rng(21)
+    x = np.concatenate([rng.normal(size=20000) * 10.0 ** rng.integers(-6, 6, 20000),
+                        np.array([1.0, -1.0, 1.00390625, 1.005859375, 3.0, 0.1])])
+    x32 = x.astype(np.float32)
+    want = torch.from_numpy(x32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(O.round_to_bf16(x32.astype(np.float64)), want)
+    # ties go to even: 1 + 2^-8 is halfway between 1 and 1 + 2^-7
+    assert O.round_to_bf16(np.array([1.0 + 2.0 ** -8]))[0] == 1.0
+    assert O.round_to_bf16(np.array([1.0 + 3 * 2.0 ** -8]))[0] == 1.0 + 2 * 2.0 ** -7
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 8.0])
+def test_bf16_centroid_bound_still_dominates_every_key(q_scale):
+    w, K, V, q, L, W = tiny(seed=22, q_scale=q_scale, lengths=torch.tensor([200, 150]),
+                            needles=3)
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk, cent_format="bf16")
+    G = w.G
+    assert np.array_equal(O.round_to_bf16(meta["cent"]), meta["cent"])
+    for b in range(w.B):
+        for h in range(w.Hq):
+            ub = O.block_bounds(q[b, h], meta["cent"][b, h // G], meta["rmax"][b, h // G],
+                                meta["var"][b, h // G], scale)
+            for j in range(w.NB):
+                n = meta["cnt"][b, h // G, j]
+                if n == 0:
+                    continue
+                s = scale * K[b, h // G, j * w.blk: j * w.blk + n] @ q[b, h]
+                assert s.max() <= ub[j] * (1 + 1e-12) + 1e-12
+    # r is measured against the rounded centroid, not the exact mean
+    m32 = O.cache_meta(K, L, w.blk)
+    assert not np.allclose(meta["rmax"], m32["rmax"], rtol=0, atol=1e-12)

@@ -227,13 +227,22 @@ def run_eta(args, rank, world, device):
     dec.check_status()
     by = step_bytes(dec, w)
 
+    if args.graph:
+        g_pre, g_dec = dec.capture(q, W, bias, tau_const, split=True)
+
     def one_step(ev=None):
-        dec.append_update()
-        dec.predict_tau(q, W, bias, tau_const)
-        dec.screen(q)
+        if args.graph:
+            g_pre.replay()
+        else:
+            dec.append_update()
+            dec.predict_tau(q, W, bias, tau_const)
+            dec.screen(q)
         if ev is not None:
             ev[0].record(stream)
-        dec.decode(q)
+        if args.graph:
+            g_dec.replay()
+        else:
+            dec.decode(q)
         if ev is not None:
             ev[1].record(stream)
 
@@ -323,6 +332,7 @@ def run_eta(args, rank, world, device):
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
             "context": w.ctx, "blk": w.blk, "bound": w.bound, "gate_T": w.gate_T,
             "tau_mode": w.tau_mode, "engine": args.engine, "centroids": args.cent,
+            "cuda_graph": bool(args.graph),
             "density_target": f"{w.density:.2f} {w.density_kind}",
             "union_density": round(by["union_density"], 4),
             "head_density": round(by["head_density"], 4),
@@ -477,6 +487,8 @@ def main():
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     ap.add_argument("--engine", default="auto", choices=["auto", "tcgen05", "fma"],
                     help="decode engine of libeta.so")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay the step as CUDA graphs (launch-bound small workloads)")
     ap.add_argument("--cent", default="bf16", choices=["f32", "bf16"],
                     help="storage of the block centroids the screen reads")
     args = ap.parse_args()

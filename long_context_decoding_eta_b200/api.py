@@ -107,6 +107,41 @@ class EtaDecoder:
         self.screen(q, stream=stream)
         return self.decode(q, stream=stream)
 
+    # -- CUDA graphs ----------------------------------------------------------
+    def capture(self, q: torch.Tensor, W=None, bias=None, tau_const=None, split: bool = False):
+        """Captures the step into CUDA graph(s) bound to the tensors given (write new
+        queries into `q` in place, then call `replay()`).  split=True captures the
+        decode call as a second graph so that it can be timed on its own.  Launch
+        overhead then no longer bounds small workloads."""
+        stream = torch.cuda.Stream()
+        stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(stream):
+            for _ in range(2):                       # warm the launch paths
+                self.step(q, W, bias, tau_const)
+            torch.cuda.synchronize()
+            g_pre = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_pre, stream=stream):
+                self.append_update()
+                self.predict_tau(q, W, bias, tau_const)
+                self.screen(q)
+                if not split:
+                    self.decode(q)
+            g_dec = None
+            if split:
+                g_dec = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g_dec, stream=stream):
+                    self.decode(q)
+        torch.cuda.current_stream().wait_stream(stream)
+        self._graphs = (g_pre, g_dec)
+        return self._graphs
+
+    def replay(self):
+        g_pre, g_dec = self._graphs
+        g_pre.replay()
+        if g_dec is not None:
+            g_dec.replay()
+        return self.o, self.lse
+
     # -- status ---------------------------------------------------------------
     def check_status(self):
         """Synchronizes, reads the device status word, raises on any error bit."""

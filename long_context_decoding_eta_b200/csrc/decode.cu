@@ -575,9 +575,7 @@ eta_status_t launch_decode_t(const eta_dims_t* dims, const DecodeParams& prm, in
   constexpr int NS = StagesFor<D>::value;
   using C = DecodeCfg<D, G, kNCW, NS>;
   auto kern = decode_kernel<D, G, DENSE, kNCW, NS>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
-      cudaSuccess)
-    return ETA_ERR_CUDA;
+  if (!set_smem_once<decode_kernel<D, G, DENSE, kNCW, NS>>(C::SMEM)) return ETA_ERR_CUDA;
   return launch_k(kern, dim3(P), dim3(C::NT), C::SMEM, s, prm);
 }
 
@@ -652,9 +650,7 @@ template <int G, bool DENSE>
 eta_status_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq,
                          const tc::TcParams& prm, int P, cudaStream_t s) {
   auto kern = tc::decode_tc_kernel<G, DENSE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES) !=
-      cudaSuccess)
-    return ETA_ERR_CUDA;
+  if (!set_smem_once<tc::decode_tc_kernel<G, DENSE>>(tc::SMEM_BYTES)) return ETA_ERR_CUDA;
   return launch_k(kern, dim3(P), dim3(tc::NT), tc::SMEM_BYTES, s, mk, mv, mq, prm);
 }
 

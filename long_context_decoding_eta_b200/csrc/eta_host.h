@@ -53,6 +53,21 @@ inline eta_status_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size
              : ETA_ERR_CUDA;
 }
 
+// Raises a kernel's dynamic shared-memory limit once per device (so that calls made
+// during stream capture issue no attribute change).  One flag set per kernel.
+template <auto Kern>
+inline bool set_smem_once(int bytes) {
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (done[dev]) return true;
+  if (cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  done[dev] = true;
+  return true;
+}
+
 inline eta_status_t launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;

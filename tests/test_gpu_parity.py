@@ -251,3 +251,22 @@ def test_bf16_centroids(d, G, blk, ctx):
     rep, gpu, sc = full_parity(w, cent_format="bf16")
     for prune in ("skip", "floor"):
         full_parity(w, cent_format="bf16", prune=prune, bound="prob", z=2.0)
+
+
+def test_cuda_graph_replay_matches_eager_step():
+    w = synth.MID.with_(B=4, ctx=8192, seed=87)
+    g = to_dev(make(w))
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, T=w.gate_T, cent_format="bf16")
+    dec.build_meta()
+    bias = torch.full((w.Hq,), 1.9, device=DEV)
+    q = g["q"].clone()
+    o_e, l_e = [t.clone() for t in dec.step(q, g["W"], bias)]
+    dec.capture(q, g["W"], bias, split=True)
+    for k in range(2):                       # new queries written in place, replayed twice
+        q.copy_(g["q"] * (1.0 + 0.5 * k))
+        o_g, l_g = [t.clone() for t in dec.replay()]
+        o_r, l_r = [t.clone() for t in dec.step(q, g["W"], bias)]
+        torch.cuda.synchronize()
+        dec.check_status()
+        assert torch.equal(o_g, o_r) and torch.equal(l_g, l_r)
+    assert not torch.equal(o_g, o_e)

@@ -68,7 +68,7 @@ typedef struct {
   int32_t T_max;  /* token capacity (stride) of the cache per (row, KV head) */
 } eta_dims_t;
 
-typedef enum { ETA_BOUND_EXACT = 0, ETA_BOUND_PROB = 1 } eta_bound_t;
+typedef enum { ETA_BOUND_EXACT = 0, ETA_BOUND_PROB = 1, ETA_BOUND_PROB_DIM = 2 } eta_bound_t;
 /* Storage of the block centroids.  ETA_CENT_BF16 halves the bytes the screen reads;
    the centroid is then rounded to bf16 (nearest even) before rmax and var are
    measured against it, so the geometric bound stays exact for what is stored. */
@@ -89,6 +89,7 @@ typedef enum { ETA_PRUNE_SKIP = 0, ETA_PRUNE_FLOOR = 1 } eta_prune_t;
  *            rounded up so that the Cauchy-Schwarz bound stays sound in fp32
  *   var_j  = (1/n_j) sum_t ||k_t - cent_j||^2
  *   cnt_j  = n_j;  vsum_j = sum_t v_t (only when vsum != NULL)
+ *   vardim_j[i] = (1/n_j) sum_t (k_t[i] - cent_j[i])^2 (only when vardim != NULL)
  * Empty blocks get zeros.
  *
  * K, V     bf16 [B, Hkv, T_max, d].  V may be NULL when vsum is NULL.
@@ -100,12 +101,15 @@ typedef enum { ETA_PRUNE_SKIP = 0, ETA_PRUNE_FLOOR = 1 } eta_prune_t;
  *          coalesced screening)
  * rmax,var fp32 [B, Hkv, NB];  cnt int32 [B, Hkv, NB]
  * vsum     fp32 [B, Hkv, NB, d] or NULL (needed only by ETA_PRUNE_FLOOR)
+ * vardim   fp32 [B, Hkv, d, NB] or NULL (dimension-major; needed only by
+ *          ETA_BOUND_PROB_DIM)
  */
 eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_bf16_t* K,
                                   const eta_bf16_t* V, const int32_t* lengths,
                                   int32_t blk_begin, int32_t blk_end,
                                   eta_cent_format_t cent_format, void* cent, float* rmax,
-                                  float* var, int32_t* cnt, float* vsum, void* stream);
+                                  float* var, int32_t* cnt, float* vsum, float* vardim,
+                                  void* stream);
 
 /*
  * eta_predict_tau -- per-query, per-head threshold (review Methodology Assessment,
@@ -131,6 +135,9 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  *   (cent in the format eta_build_block_meta stored it)
  *     ETA_BOUND_EXACT: R_j = rmax_j                      (Cauchy-Schwarz, sound)
  *     ETA_BOUND_PROB:  R_j = min(rmax_j, z * sqrt(var_j / d))
+ *     ETA_BOUND_PROB_DIM: ||q|| * R_j is replaced by
+ *                      min(||q|| rmax_j, z * sqrt(sum_i q_i^2 vardim_j[i]))
+ *                      (per-dimension variance; needs vardim, never looser than exact)
  *   admit[b,h,j] = cnt_j > 0 && UB[b,h,j] >= tau[b,h]
  *   union[b,g,j] = OR over the G query heads of group g
  * Outputs:
@@ -145,7 +152,7 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
 size_t eta_screen_workspace_size(const eta_dims_t* dims);
 eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                         eta_cent_format_t cent_format, const void* cent, const float* rmax,
-                        const float* var,
+                        const float* var, const float* vardim,
                         const int32_t* cnt, eta_bound_t bound, float z, float scale,
                         uint32_t* head_mask, int32_t* union_idx, int32_t* union_cnt,
                         float* bounds_out, int32_t* head_cnt, void* ws, size_t ws_bytes,

@@ -20,7 +20,7 @@ ETA_OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape",
                 3: "workspace missing or too small", 4: "CUDA error",
                 5: "device wait timed out", 6: "non-finite query"}
-BOUND = {"exact": 0, "prob": 1}
+BOUND = {"exact": 0, "prob": 1, "prob_dim": 2}
 CENT = {"f32": 0, "bf16": 1}
 PRUNE = {"skip": 0, "floor": 1}
 TAIL_BLOCK = -1
@@ -69,11 +69,11 @@ def lib() -> C.CDLL:
         raise RuntimeError(f"{LIB_PATH} is missing: build it with "
                            "`python -m long_context_decoding_eta_b200.build`")
     L = C.CDLL(LIB_PATH)
-    L.eta_build_block_meta.argtypes = [DIMS, P, P, P, I32, I32, I32, P, P, P, P, P, P]
+    L.eta_build_block_meta.argtypes = [DIMS, P, P, P, I32, I32, I32, P, P, P, P, P, P, P]
     L.eta_predict_tau.argtypes = [DIMS, P, P, P, P, P, P, P]
     L.eta_screen_workspace_size.argtypes = [DIMS]
     L.eta_screen_workspace_size.restype = C.c_size_t
-    L.eta_screen.argtypes = [DIMS, P, P, I32, P, P, P, P, I32, F32, F32, P, P, P, P, P, P,
+    L.eta_screen.argtypes = [DIMS, P, P, I32, P, P, P, P, P, I32, F32, F32, P, P, P, P, P, P,
                              C.c_size_t, P, P]
     L.eta_decode_workspace_size.argtypes = [DIMS]
     L.eta_decode_workspace_size.restype = C.c_size_t
@@ -122,11 +122,12 @@ def _cent_format(cent) -> int:
 
 
 def eta_build_block_meta(dims: Dims, K, V, lengths, blk_begin, blk_end, cent, rmax, var, cnt,
-                         vsum=None, stream=None):
+                         vsum=None, stream=None, vardim=None):
     """cent: fp32 or bf16 tensor [B, Hkv, d, NB]; its dtype selects the format."""
     _check("eta_build_block_meta", lib().eta_build_block_meta(
         C.byref(dims), _p(K), _p(V), _p(lengths), int(blk_begin), int(blk_end),
-        _cent_format(cent), _p(cent), _p(rmax), _p(var), _p(cnt), _p(vsum), _stream(stream)))
+        _cent_format(cent), _p(cent), _p(rmax), _p(var), _p(cnt), _p(vsum), _p(vardim),
+        _stream(stream)))
 
 
 def eta_predict_tau(dims: Dims, q, W, bias, tau_const, tau, dev_status=None, stream=None):
@@ -140,9 +141,11 @@ def eta_screen_workspace_size(dims: Dims) -> int:
 
 
 def eta_screen(dims: Dims, q, tau, cent, rmax, var, cnt, bound, z, scale, head_mask,
-               union_idx, union_cnt, bounds_out, head_cnt, ws, dev_status=None, stream=None):
+               union_idx, union_cnt, bounds_out, head_cnt, ws, dev_status=None, stream=None,
+               vardim=None):
     _check("eta_screen", lib().eta_screen(
-        C.byref(dims), _p(q), _p(tau), _cent_format(cent), _p(cent), _p(rmax), _p(var), _p(cnt),
+        C.byref(dims), _p(q), _p(tau), _cent_format(cent), _p(cent), _p(rmax), _p(var),
+        _p(vardim), _p(cnt),
         BOUND[bound] if isinstance(bound, str) else int(bound), float(z), float(scale),
         _p(head_mask), _p(union_idx), _p(union_cnt), _p(bounds_out), _p(head_cnt), _p(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _p(dev_status), _stream(stream)))

@@ -51,6 +51,8 @@ class EtaDecoder:
         self.cnt = torch.zeros(B, Hkv, self.NB, dtype=i32, device=dev)
         self.vsum = (torch.zeros(B, Hkv, self.NB, d, dtype=f32, device=dev)
                      if prune == "floor" else None)
+        self.vardim = (torch.zeros(B, Hkv, d, self.NB, dtype=f32, device=dev)
+                       if bound == "prob_dim" else None)
         self.tau = torch.zeros(B, Hq, dtype=f32, device=dev)
         self.head_mask = torch.zeros(B, Hq, self.NW, dtype=torch.int32, device=dev)
         self.union_idx = torch.zeros(B, Hkv, self.NB, dtype=i32, device=dev)
@@ -69,7 +71,8 @@ class EtaDecoder:
     # -- metadata -------------------------------------------------------------
     def build_meta(self, blk_begin: int = 0, blk_end: int = -1, stream=None):
         L.eta_build_block_meta(self.dims, self.K, self.V, self.lengths, blk_begin, blk_end,
-                               self.cent, self.rmax, self.var, self.cnt, self.vsum, stream)
+                               self.cent, self.rmax, self.var, self.cnt, self.vsum, stream,
+                               self.vardim)
 
     def append_update(self, stream=None):
         """Recompute the tail block of every row (call after appending a token)."""
@@ -85,7 +88,7 @@ class EtaDecoder:
         L.eta_screen(self.dims, q, tau, self.cent, self.rmax, self.var, self.cnt, self.bound,
                      self.z, self.scale, self.head_mask, self.union_idx, self.union_cnt,
                      self.bounds if bounds is None else bounds, self.head_cnt, self.ws_screen,
-                     self.dev_status, stream)
+                     self.dev_status, stream, self.vardim)
 
     def decode(self, q, tau=None, stream=None):
         tau = self.tau if tau is None else tau

@@ -53,7 +53,7 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
                   const eta_bf16_t* __restrict__ V, const int32_t* __restrict__ lengths,
                   int blk_begin, int nblk, void* __restrict__ cent,
                   float* __restrict__ rmax, float* __restrict__ var, int32_t* __restrict__ cnt,
-                  float* __restrict__ vsum, int32_t* status) {
+                  float* __restrict__ vsum, float* __restrict__ vardim, int32_t* status) {
   ETA_PDL_ENTRY();
   constexpr int DPL = D / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -108,9 +108,15 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
   }
   // pass 2: squared distances to the stored fp32 centroid
   float r2max = 0.f, s2 = 0.f;
+  float vd[DPL];                // per-dimension squared deviations (ETA_BOUND_PROB_DIM)
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) vd[i] = 0.f;
   for (int w = 0; w < kMetaWarps; ++w) {
     const int lo = min(w * per, n), hi = min(lo + per, n);
     float ps = 0.f;
+    float pv[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) pv[i] = 0.f;
 #pragma unroll 4
     for (int t = lo; t < hi; ++t) {
       float x[DPL];
@@ -120,12 +126,20 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
       for (int i = 0; i < DPL; ++i) {
         const float dv = x[i] - c[i];
         p = fmaf(dv, dv, p);
+        pv[i] = fmaf(dv, dv, pv[i]);
       }
       p = warp_sum(p);          // butterfly: bit-identical in every lane
       r2max = fmaxf(r2max, p);
       ps += p;
     }
     s2 += ps;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) vd[i] += pv[i];
+  }
+  if (vardim) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i)
+      vardim[((size_t)r * D + lane * DPL + i) * NB + j] = n > 0 ? vd[i] / (float)n : 0.f;
   }
 #pragma unroll
   for (int i = 0; i < DPL; ++i)
@@ -172,7 +186,7 @@ __global__ void __launch_bounds__(kMetaWarps * 32)
 meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restrict__ K,
                  const eta_bf16_t* __restrict__ V, const int32_t* __restrict__ lengths,
                  void* __restrict__ cent, float* __restrict__ rmax, float* __restrict__ var,
-                 int32_t* __restrict__ cnt, float* __restrict__ vsum) {
+                 int32_t* __restrict__ cnt, float* __restrict__ vsum, float* __restrict__ vardim) {
   ETA_PDL_ENTRY();
   constexpr int DPL = D / 32;
   __shared__ float part[kMetaWarps][D];
@@ -212,6 +226,9 @@ meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restri
     else c[i] = sum / (float)n;
   }
   float r2max = 0.f, s2 = 0.f;
+  float pv[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) pv[i] = 0.f;
   for (int t = t_lo; t < t_hi; ++t) {
     float x[DPL];
     load_row<DPL>(kb + (size_t)t * D, x);
@@ -220,10 +237,26 @@ meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restri
     for (int i = 0; i < DPL; ++i) {
       const float dv = x[i] - c[i];
       pd = fmaf(dv, dv, pd);
+      pv[i] = fmaf(dv, dv, pv[i]);
     }
     pd = warp_sum(pd);
     r2max = fmaxf(r2max, pd);
     s2 += pd;
+  }
+  if (vardim) {
+    __shared__ float vpart[kMetaWarps][D];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) vpart[warp][lane * DPL + i] = pv[i];
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMetaWarps; ++w) sum += vpart[w][lane * DPL + i];
+        vardim[((size_t)r * D + lane * DPL + i) * NB + j] = sum / (float)n;
+      }
+    }
   }
   if (lane == 0) {
     red_max[warp] = r2max;
@@ -278,14 +311,15 @@ template <int D, int CF>
 static eta_status_t launch_meta(bool tail, const eta_dims_t* dims, int NB, int R, int blk_begin,
                                 int nblk, const eta_bf16_t* K, const eta_bf16_t* V,
                                 const int32_t* lengths, void* cent, float* rmax, float* var,
-                                int32_t* cnt, float* vsum, cudaStream_t s) {
+                                int32_t* cnt, float* vsum, float* vardim, cudaStream_t s) {
   if (tail)
     return launch_k(meta_tail_kernel<D, CF>, dim3(R), dim3(kMetaWarps * 32), 0, s, dims->Hkv,
-                    dims->T_max, dims->blk, NB, K, V, lengths, cent, rmax, var, cnt, vsum);
+                    dims->T_max, dims->blk, NB, K, V, lengths, cent, rmax, var, cnt, vsum,
+                    vardim);
   dim3 grid((nblk + kMetaWarps - 1) / kMetaWarps, R);
   return launch_k(meta_build_kernel<D, CF>, grid, dim3(kMetaWarps * 32), 0, s, dims->Hkv,
                   dims->T_max, dims->blk, NB, K, V, lengths, blk_begin, nblk, cent, rmax, var,
-                  cnt, vsum, (int32_t*)nullptr);
+                  cnt, vsum, vardim, (int32_t*)nullptr);
 }
 
 }  // namespace eta
@@ -297,7 +331,7 @@ extern "C" eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_b
                                              int32_t blk_begin, int32_t blk_end,
                                              eta_cent_format_t cent_format, void* cent,
                                              float* rmax, float* var, int32_t* cnt, float* vsum,
-                                             void* stream) {
+                                             float* vardim, void* stream) {
   eta_status_t st = check_dims(dims);
   if (st != ETA_OK) return st;
   if (!K || !lengths || !cent || !rmax || !var || !cnt) return ETA_ERR_INVALID_ARG;
@@ -318,11 +352,11 @@ extern "C" eta_status_t eta_build_block_meta(const eta_dims_t* dims, const eta_b
   const bool bf = cent_format == ETA_CENT_BF16;
   if (dims->d == 128)
     return bf ? launch_meta<128, 1>(tail, dims, NB, R, blk_begin, nblk, K, V, lengths, cent, rmax,
-                                   var, cnt, vsum, s)
+                                   var, cnt, vsum, vardim, s)
               : launch_meta<128, 0>(tail, dims, NB, R, blk_begin, nblk, K, V, lengths, cent, rmax,
-                                   var, cnt, vsum, s);
+                                   var, cnt, vsum, vardim, s);
   return bf ? launch_meta<64, 1>(tail, dims, NB, R, blk_begin, nblk, K, V, lengths, cent, rmax,
-                                var, cnt, vsum, s)
+                                var, cnt, vsum, vardim, s)
             : launch_meta<64, 0>(tail, dims, NB, R, blk_begin, nblk, K, V, lengths, cent, rmax,
-                                var, cnt, vsum, s);
+                                var, cnt, vsum, vardim, s);
 }

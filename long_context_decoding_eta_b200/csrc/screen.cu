@@ -27,11 +27,12 @@ ETA_DEV float load_cent(const void* cent, size_t i) {
   else return __ldg(reinterpret_cast<const float*>(cent) + i);
 }
 
-template <int D, int G, int CF>
+template <int D, int G, int CF, bool VD>
 __global__ void __launch_bounds__(kScreenWarps * 32)
 screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
               const float* __restrict__ tau, const void* __restrict__ cent,
               const float* __restrict__ rmax, const float* __restrict__ var,
+              const float* __restrict__ vardim,
               const int32_t* __restrict__ cnt, int bound, float z, float scale,
               uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
               float* __restrict__ bounds_out) {
@@ -63,14 +64,19 @@ screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
   const int j = w * 32 + lane;
   const bool vj = j < NB;
   const size_t c0 = (size_t)r * D * NB + (vj ? j : 0);
-  float acc[G];
+  float acc[G], acc2[G];
 #pragma unroll
-  for (int h = 0; h < G; ++h) acc[h] = 0.f;
+  for (int h = 0; h < G; ++h) { acc[h] = 0.f; acc2[h] = 0.f; }
 #pragma unroll 16
   for (int k = 0; k < D; ++k) {
     const float c = vj ? load_cent<CF>(cent, c0 + (size_t)k * NB) : 0.f;
+    float vdk = 0.f;
+    if constexpr (VD) vdk = vj ? __ldg(vardim + c0 + (size_t)k * NB) : 0.f;
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = fmaf(qs[k * G + h], c, acc[h]);
+    for (int h = 0; h < G; ++h) {
+      acc[h] = fmaf(qs[k * G + h], c, acc[h]);
+      if constexpr (VD) acc2[h] = fmaf(qs[k * G + h] * qs[k * G + h], vdk, acc2[h]);
+    }
   }
   const size_t rj = (size_t)r * NB + j;
   float rad = vj ? __ldg(rmax + rj) : 0.f;
@@ -79,7 +85,9 @@ screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
   uint32_t uni = 0;
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    const float ub = scale * fmaf(qn[h], rad, acc[h]);
+    float ub;
+    if constexpr (VD) ub = scale * (acc[h] + fminf(qn[h] * rad, z * sqrtf(acc2[h])));
+    else ub = scale * fmaf(qn[h], rad, acc[h]);
     if (bounds_out && vj) bounds_out[(qhead0 + h) * NB + j] = ub;
     const bool adm = vj && n > 0 && ub >= ts[h];
     const uint32_t m = __ballot_sync(0xffffffffu, adm);
@@ -98,11 +106,12 @@ screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
 constexpr int kScreenVecWarps = 4;
 constexpr int kLoadBatch = 16;   // independent 16-byte loads in flight per lane
 
-template <int D, int G, int CF>
+template <int D, int G, int CF, bool VD>
 __global__ void __launch_bounds__(kScreenVecWarps * 32)
 screen_vec_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
                   const float* __restrict__ tau, const void* __restrict__ cent,
                   const float* __restrict__ rmax, const float* __restrict__ var,
+                  const float* __restrict__ vardim,
                   const int32_t* __restrict__ cnt, int bound, float z, float scale,
                   uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
                   float* __restrict__ bounds_out) {
@@ -142,11 +151,17 @@ screen_vec_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict_
   const LdT* cp = reinterpret_cast<const LdT*>(
       reinterpret_cast<const unsigned char*>(cent) + ((size_t)r * D * NB + (vj ? j0 : 0)) *
                                                         (CF == 1 ? 2 : 4));
-  float acc[VW][G];
+  float acc[VW][G], acc2[VW][VD ? G : 1];
 #pragma unroll
-  for (int k = 0; k < VW; ++k)
+  for (int k = 0; k < VW; ++k) {
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[k][h] = 0.f;
+#pragma unroll
+    for (int h = 0; h < (VD ? G : 1); ++h) acc2[k][h] = 0.f;
+  }
+  const float4* vdp = VD ? reinterpret_cast<const float4*>(
+                               vardim + (size_t)r * D * NB + (vj ? j0 : 0))
+                         : nullptr;
 #pragma unroll 1
   for (int d0 = 0; d0 < D; d0 += kLoadBatch) {
     LdT cb[kLoadBatch];
@@ -168,6 +183,17 @@ screen_vec_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict_
         const float qv = qs[(d0 + u) * G + h];
 #pragma unroll
         for (int k = 0; k < VW; ++k) acc[k][h] = fmaf(qv, cv[k], acc[k][h]);
+      }
+      if constexpr (VD) {
+        const float4 vv = vj ? __ldg(vdp + (size_t)(d0 + u) * (NB / 4))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float vk[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float q2 = qs[(d0 + u) * G + h] * qs[(d0 + u) * G + h];
+#pragma unroll
+          for (int k = 0; k < VW; ++k) acc2[k][h] = fmaf(q2, vk[k], acc2[k][h]);
+        }
       }
     }
   }
@@ -200,7 +226,10 @@ screen_vec_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict_
     float ubv[VW];
 #pragma unroll
     for (int k = 0; k < VW; ++k) {
-      ubv[k] = scale * fmaf(qn[h], rad[k], acc[k][h]);
+      if constexpr (VD)
+        ubv[k] = scale * (acc[k][h] + fminf(qn[h] * rad[k], z * sqrtf(acc2[k][h])));
+      else
+        ubv[k] = scale * fmaf(qn[h], rad[k], acc[k][h]);
       if (vj && n[k] > 0 && ubv[k] >= ts[h]) bits |= 1u << k;
     }
     if (bounds_out && vj) {
@@ -272,26 +301,27 @@ compact_kernel(int Hq, int Hkv, int G, int NB, int NW, const uint32_t* __restric
   }
 }
 
-template <int D, int CF>
+template <int D, int CF, bool VD>
 static eta_status_t launch_screen(bool vec, int G, dim3 grid, cudaStream_t s, int Hq, int Hkv,
                                   int NB, int NW, const eta_bf16_t* q, const float* tau,
                                   const void* cent, const float* rmax, const float* var,
-                                  const int32_t* cnt, int bound, float z, float scale,
-                                  uint32_t* head_mask, uint32_t* uw, float* bounds_out) {
+                                  const float* vardim, const int32_t* cnt, int bound, float z,
+                                  float scale, uint32_t* head_mask, uint32_t* uw,
+                                  float* bounds_out) {
   using KernT = void (*)(int, int, int, int, const eta_bf16_t*, const float*, const void*,
-                         const float*, const float*, const int32_t*, int, float, float,
-                         uint32_t*, uint32_t*, float*);
+                         const float*, const float*, const float*, const int32_t*, int, float,
+                         float, uint32_t*, uint32_t*, float*);
   KernT kern = nullptr;
   switch (G) {
-    case 1: kern = vec ? screen_vec_kernel<D, 1, CF> : screen_kernel<D, 1, CF>; break;
-    case 2: kern = vec ? screen_vec_kernel<D, 2, CF> : screen_kernel<D, 2, CF>; break;
-    case 4: kern = vec ? screen_vec_kernel<D, 4, CF> : screen_kernel<D, 4, CF>; break;
-    case 8: kern = vec ? screen_vec_kernel<D, 8, CF> : screen_kernel<D, 8, CF>; break;
+    case 1: kern = vec ? screen_vec_kernel<D, 1, CF, VD> : screen_kernel<D, 1, CF, VD>; break;
+    case 2: kern = vec ? screen_vec_kernel<D, 2, CF, VD> : screen_kernel<D, 2, CF, VD>; break;
+    case 4: kern = vec ? screen_vec_kernel<D, 4, CF, VD> : screen_kernel<D, 4, CF, VD>; break;
+    case 8: kern = vec ? screen_vec_kernel<D, 8, CF, VD> : screen_kernel<D, 8, CF, VD>; break;
     default: return ETA_ERR_UNSUPPORTED;
   }
   const dim3 block((vec ? kScreenVecWarps : kScreenWarps) * 32);
-  return launch_k(kern, grid, block, 0, s, Hq, Hkv, NB, NW, q, tau, cent, rmax, var, cnt, bound,
-                  z, scale, head_mask, uw, bounds_out);
+  return launch_k(kern, grid, block, 0, s, Hq, Hkv, NB, NW, q, tau, cent, rmax, var, vardim, cnt,
+                  bound, z, scale, head_mask, uw, bounds_out);
 }
 
 }  // namespace eta
@@ -305,7 +335,7 @@ extern "C" size_t eta_screen_workspace_size(const eta_dims_t* dims) {
 
 extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                                    eta_cent_format_t cent_format, const void* cent,
-                                   const float* rmax, const float* var,
+                                   const float* rmax, const float* var, const float* vardim,
                                    const int32_t* cnt, eta_bound_t bound, float z, float scale,
                                    uint32_t* head_mask, int32_t* union_idx, int32_t* union_cnt,
                                    float* bounds_out, int32_t* head_cnt, void* ws,
@@ -315,7 +345,9 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   if (st != ETA_OK) return st;
   if (!q || !tau || !cent || !rmax || !cnt || !head_mask || !union_idx || !union_cnt)
     return ETA_ERR_INVALID_ARG;
-  if (bound != ETA_BOUND_EXACT && bound != ETA_BOUND_PROB) return ETA_ERR_INVALID_ARG;
+  if (bound != ETA_BOUND_EXACT && bound != ETA_BOUND_PROB && bound != ETA_BOUND_PROB_DIM)
+    return ETA_ERR_INVALID_ARG;
+  if (bound == ETA_BOUND_PROB_DIM && (!vardim || !(z >= 0.f))) return ETA_ERR_INVALID_ARG;
   if (cent_format != ETA_CENT_F32 && cent_format != ETA_CENT_BF16) return ETA_ERR_INVALID_ARG;
   if (bound == ETA_BOUND_PROB && (!var || !(z >= 0.f))) return ETA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < eta_screen_workspace_size(dims)) return ETA_ERR_WORKSPACE;
@@ -326,8 +358,10 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf = cent_format == ETA_CENT_BF16;
   const int VW = 4;
+  const bool vd = bound == ETA_BOUND_PROB_DIM;
   const bool vec = (NB % VW == 0) && aligned16(cent) && aligned16(rmax) && aligned16(cnt) &&
-                   (!var || aligned16(var)) && (!bounds_out || aligned16(bounds_out));
+                   (!var || aligned16(var)) && (!vardim || aligned16(vardim)) &&
+                   (!bounds_out || aligned16(bounds_out));
   dim3 grid;
   if (vec) {
     const int ngroups = (NB + 32 * VW - 1) / (32 * VW);
@@ -336,11 +370,18 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
     grid = dim3((NW + kScreenWarps - 1) / kScreenWarps, R);
   }
 #define ETA_SCREEN_ARGS vec, G, grid, s, dims->Hq, dims->Hkv, NB, NW, q, tau, cent, rmax, var, \
-                        cnt, (int)bound, z, scale, head_mask, uw, bounds_out
-  if (dims->d == 128)
-    st = bf ? launch_screen<128, 1>(ETA_SCREEN_ARGS) : launch_screen<128, 0>(ETA_SCREEN_ARGS);
-  else
-    st = bf ? launch_screen<64, 1>(ETA_SCREEN_ARGS) : launch_screen<64, 0>(ETA_SCREEN_ARGS);
+                        vardim, cnt, (int)bound, z, scale, head_mask, uw, bounds_out
+  if (dims->d == 128) {
+    if (vd) st = bf ? launch_screen<128, 1, true>(ETA_SCREEN_ARGS)
+                    : launch_screen<128, 0, true>(ETA_SCREEN_ARGS);
+    else st = bf ? launch_screen<128, 1, false>(ETA_SCREEN_ARGS)
+                 : launch_screen<128, 0, false>(ETA_SCREEN_ARGS);
+  } else {
+    if (vd) st = bf ? launch_screen<64, 1, true>(ETA_SCREEN_ARGS)
+                    : launch_screen<64, 0, true>(ETA_SCREEN_ARGS);
+    else st = bf ? launch_screen<64, 1, false>(ETA_SCREEN_ARGS)
+                 : launch_screen<64, 0, false>(ETA_SCREEN_ARGS);
+  }
 #undef ETA_SCREEN_ARGS
   if (st != ETA_OK) return st;
   return launch_k(compact_kernel, dim3(R), dim3(kCompactThreads), 0, s, dims->Hq, dims->Hkv, G,

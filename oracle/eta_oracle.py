@@ -39,6 +39,7 @@ import numpy as np
 
 BOUND_EXACT = "exact"
 BOUND_PROB = "prob"
+BOUND_PROB_DIM = "prob_dim"
 PRUNE_SKIP = "skip"
 PRUNE_FLOOR = "floor"
 
@@ -74,6 +75,7 @@ def block_meta(K_seq: np.ndarray, n_valid: int, blk: int,
       var_j  = (1/n_j) sum_t ||k_t - cent_j||^2  (total variance, one scalar)
       cnt_j  = n_j
       vsum_j = sum_t v_t                         (only if V_seq is given)
+      vardim_j[i] = (1/n_j) sum_t (k_t[i] - cent_j[i])^2   (per-dimension variance)
     Empty blocks (n_j = 0) get zeros.
     """
     T_max, d = K_seq.shape
@@ -82,6 +84,7 @@ def block_meta(K_seq: np.ndarray, n_valid: int, blk: int,
     rmax = np.zeros(NB)
     var = np.zeros(NB)
     cnt = np.zeros(NB, dtype=np.int64)
+    vardim = np.zeros((NB, d))
     vsum = np.zeros((NB, d)) if V_seq is not None else None
     for j in range(NB):
         lo = j * blk
@@ -97,10 +100,11 @@ def block_meta(K_seq: np.ndarray, n_valid: int, blk: int,
         cent[j] = c
         rmax[j] = dist.max()
         var[j] = (dist ** 2).mean()
+        vardim[j] = ((keys - c) ** 2).mean(axis=0)
         cnt[j] = n
         if vsum is not None:
             vsum[j] = V_seq[lo:hi].sum(axis=0)
-    out = dict(cent=cent, rmax=rmax, var=var, cnt=cnt)
+    out = dict(cent=cent, rmax=rmax, var=var, cnt=cnt, vardim=vardim)
     if vsum is not None:
         out["vsum"] = vsum
     return out
@@ -141,22 +145,26 @@ def const_tau(B: int, tau_const: np.ndarray) -> np.ndarray:
 #                      review-FAQ "best possible score falls below the threshold"]
 # ----------------------------------------------------------------------------
 def block_bounds(q_h: np.ndarray, cent: np.ndarray, rmax: np.ndarray, var: np.ndarray,
-                 scale: float, bound: str = BOUND_EXACT, z: float = 3.0) -> np.ndarray:
+                 scale: float, bound: str = BOUND_EXACT, z: float = 3.0,
+                 vardim: Optional[np.ndarray] = None) -> np.ndarray:
     """Upper bound on scale*(q.k) over each block, in logit units, shape [NB].
 
     exact (Cauchy-Schwarz):  scale * (q.c + ||q|| * rmax)
     prob  (variance):        scale * (q.c + ||q|| * min(rmax, z * sqrt(var / d)))
+    prob_dim (per-dimension variance, vardim [NB, d]):
+                             scale * (q.c + min(||q|| * rmax, z * sqrt(sum_i q_i^2 vardim_i)))
     """
     d = q_h.shape[0]
     qc = cent @ q_h
     qn = math.sqrt(float(q_h @ q_h))
     if bound == BOUND_EXACT:
-        radius = rmax
-    elif bound == BOUND_PROB:
-        radius = np.minimum(rmax, z * np.sqrt(var / d))
-    else:
-        raise ValueError(bound)
-    return scale * (qc + qn * radius)
+        return scale * (qc + qn * rmax)
+    if bound == BOUND_PROB:
+        return scale * (qc + qn * np.minimum(rmax, z * np.sqrt(var / d)))
+    if bound == BOUND_PROB_DIM:
+        spread = np.sqrt(vardim @ (q_h * q_h))
+        return scale * (qc + np.minimum(qn * rmax, z * spread))
+    raise ValueError(bound)
 
 
 def screen(q: np.ndarray, tau: np.ndarray, meta: Dict[str, np.ndarray], scale: float,
@@ -176,7 +184,8 @@ def screen(q: np.ndarray, tau: np.ndarray, meta: Dict[str, np.ndarray], scale: f
         for h in range(Hq):
             g = h // G
             UB[b, h] = block_bounds(q[b, h], meta["cent"][b, g], meta["rmax"][b, g],
-                                    meta["var"][b, g], scale, bound, z)
+                                    meta["var"][b, g], scale, bound, z,
+                                    meta["vardim"][b, g] if "vardim" in meta else None)
     nonempty = meta["cnt"] > 0                                   # [B, Hkv, NB]
     nonempty_h = np.repeat(nonempty, G, axis=1)                  # [B, Hq, NB]
     admit = (UB >= tau[:, :, None]) & nonempty_h

@@ -54,6 +54,8 @@ def gpu_meta(dec, rows=None) -> Dict[str, np.ndarray]:
              var=f64(sel(dec.var)), cnt=sel(dec.cnt).cpu().numpy().astype(np.int64))
     if dec.vsum is not None:
         m["vsum"] = f64(sel(dec.vsum))
+    if getattr(dec, "vardim", None) is not None:
+        m["vardim"] = f64(sel(dec.vardim).transpose(2, 3))
     return m
 
 
@@ -68,6 +70,8 @@ def check_meta(gm: Dict[str, np.ndarray], om: Dict[str, np.ndarray], rows=None):
     np.testing.assert_allclose(sel(gm["var"]), om["var"], rtol=2e-5, atol=1e-6)
     if "vsum" in gm and "vsum" in om:
         np.testing.assert_allclose(sel(gm["vsum"]), om["vsum"], rtol=0, atol=2e-4)
+    if "vardim" in gm and "vardim" in om:
+        np.testing.assert_allclose(sel(gm["vardim"]), om["vardim"], rtol=2e-5, atol=1e-6)
 
 
 @dataclass

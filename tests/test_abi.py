@@ -71,19 +71,19 @@ def test_argument_validation_without_gpu():
                        0, None, None, None, None, None, 0, None, None)
     assert r == 1
     bad = L.Dims.of(2, 16, 4, 96, 64, 4096)            # d = 96 unsupported
-    r = lib.eta_screen(ctypes.byref(bad), None, None, 0, *([None] * 4), 0, 0.0, 0.0,
+    r = lib.eta_screen(ctypes.byref(bad), None, None, 0, *([None] * 5), 0, 0.0, 0.0,
                        *([None] * 6), 0, None, None)
     assert r == 2
     odd = L.Dims.of(2, 16, 4, 128, 64, 4000)           # T_max not a multiple of blk
     assert lib.eta_build_block_meta(ctypes.byref(odd), None, None, None, 0, -1, 0,
-                                    *([None] * 6)) == 2
+                                    *([None] * 7)) == 2
     # unknown centroid format -> invalid argument (before any CUDA call)
     ok = L.Dims.of(2, 16, 4, 128, 64, 4096)
     import torch as _t
     buf = _t.zeros(8)
     p = ctypes.c_void_p(buf.data_ptr())
     assert lib.eta_build_block_meta(ctypes.byref(ok), p, None, p, 0, -1, 7, p, p, p, p, None,
-                                    None) == 1
+                                    None, None) == 1
     g3 = L.Dims.of(2, 12, 4, 128, 64, 4096)            # G = 3 unsupported
     assert lib.eta_predict_tau(ctypes.byref(g3), *([None] * 7)) == 2
     assert L.eta_screen_workspace_size(dims) == 256       # 2*4 rows x 2 words, 256-aligned

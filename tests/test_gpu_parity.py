@@ -270,3 +270,11 @@ def test_cuda_graph_replay_matches_eager_step():
         dec.check_status()
         assert torch.equal(o_g, o_r) and torch.equal(l_g, l_r)
     assert not torch.equal(o_g, o_e)
+
+
+@pytest.mark.parametrize("cent_format", ["f32", "bf16"])
+@pytest.mark.parametrize("ctx", [8192, 3000])
+def test_per_dimension_variance_bound(cent_format, ctx):
+    w = synth.MID.with_(B=3, ctx=ctx, needles=4, q_scale=4.0, density=0.3, seed=310 + ctx)
+    for z in (1.0, 3.0):
+        full_parity(w, bound="prob_dim", z=z, cent_format=cent_format, T=0.0)

@@ -483,3 +483,39 @@ def test_bf16_centroid_bound_still_dominates_every_key(q_scale):
     # r is measured against the rounded centroid, not the exact mean
     m32 = O.cache_meta(K, L, w.blk)
     assert not np.allclose(meta["rmax"], m32["rmax"], rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# per-dimension variance bound
+# --------------------------------------------------------------------------
+def test_per_dimension_variance_bound_properties():
+    w, K, V, q, L, W = tiny(seed=23, q_scale=4.0)
+    scale = O.default_scale(w.d)
+    meta = O.cache_meta(K, L, w.blk)
+    # vardim sums to the scalar variance (total variance = sum of per-dim variances)
+    np.testing.assert_allclose(meta["vardim"].sum(axis=-1), meta["var"], rtol=1e-12, atol=1e-14)
+    ex = O.screen(q, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_EXACT)["bounds"]
+    for z in (0.5, 2.0, 3.0):
+        pd = O.screen(q, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_PROB_DIM, z)["bounds"]
+        assert np.all(pd <= ex + 1e-12)
+    pd = O.screen(q, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_PROB_DIM, 1e9)["bounds"]
+    np.testing.assert_allclose(pd, ex, atol=1e-12)
+    # isotropic query: sum_i q_i^2 vardim_i = |q|^2 var / d -> equals the scalar prob bound
+    qi = np.ones_like(q) * 0.3
+    pr = O.screen(qi, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_PROB, 2.0)["bounds"]
+    pdi = O.screen(qi, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_PROB_DIM, 2.0)["bounds"]
+    np.testing.assert_allclose(pdi, pr, rtol=1e-12, atol=1e-12)
+
+
+def test_per_dimension_variance_bound_brute_force_values():
+    rng = np.random.default_rng(24)
+    keys = rng.normal(size=(7, 5)) * np.array([0.1, 2.0, 0.5, 1.0, 0.01])
+    m = O.block_meta(keys, 7, 8)
+    c = keys.mean(0)
+    assert np.allclose(m["vardim"][0], [np.mean((keys[:, i] - c[i]) ** 2) for i in range(5)])
+    qv = rng.normal(size=5)
+    ub = O.block_bounds(qv, m["cent"], m["rmax"], m["var"], 1.0, O.BOUND_PROB_DIM, 1.5,
+                        m["vardim"])
+    want = c @ qv + min(np.linalg.norm(qv) * m["rmax"][0],
+                        1.5 * math.sqrt(sum(qv[i] ** 2 * m["vardim"][0][i] for i in range(5))))
+    assert abs(ub[0] - want) < 1e-12

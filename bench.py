@@ -473,6 +473,56 @@ def run_reference(args, rank, world, device):
     }
 
 
+def run_prefill(args, rank, world, device):
+    """Dense gated causal prefill (eta_prefill): tensor-core roofline."""
+    from long_context_decoding_eta_b200 import _lib as L
+    B, Hq, Hkv, d, T = args.pf_B, 16, 4, 128, args.pf_T
+    g = torch.Generator(device=device)
+    g.manual_seed(2000 + rank)
+    q = torch.randn(B, Hq, T, d, generator=g, device=device).to(torch.bfloat16)
+    K = torch.randn(B, Hkv, T, d, generator=g, device=device).to(torch.bfloat16)
+    V = torch.randn(B, Hkv, T, d, generator=g, device=device).to(torch.bfloat16)
+    # thresholds from the Eq. 1 predictor applied to every token's concatenated heads
+    W = torch.randn(Hq * d, Hq, generator=g, device=device) * (0.1 / math.sqrt(d))
+    qt = q.permute(0, 2, 1, 3).reshape(B * T, Hq, d).contiguous()
+    tdims = L.Dims.of(B * T, Hq, Hkv, d, 64, 128)
+    tau_bt = torch.empty(B * T, Hq, device=device)
+    L.eta_predict_tau(tdims, qt, W, torch.full((Hq,), 0.5, device=device), None, tau_bt)
+    tau = tau_bt.reshape(B, T, Hq).permute(0, 2, 1).contiguous()
+    lengths = torch.full((B,), T, dtype=torch.int32, device=device)
+    dims = L.Dims.of(B, Hq, Hkv, d, 64, T)
+    O = torch.empty(B, Hq, T, d, device=device)
+    lse = torch.empty(B, Hq, T, device=device)
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    run = lambda: L.eta_prefill(dims, q, tau, K, V, lengths, args.pf_gate_T, 0.0, O, lse, st)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(device.index or 0) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 4.0 * d * B * Hq * (T * (T + 1) / 2)       # QK^T + PV over causal pairs
+    tf = flops / (ms * 1e-3) / 1e12
+    pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"] \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1590.0
+    return {"metric": "gated causal prefill TFLOP/s", "value": tf, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": f"prefill-b{B}-h{Hq}x{Hkv}-d{d}-T{T}-causal",
+                       "gate_T": args.pf_gate_T},
+            "roofline": {"kernel": "prefill_tc_kernel", "bound": "tensor", "achieved": tf,
+                         "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
+                         "peak_kind": "measured cuBLAS bf16 burst"},
+            "gpu_launches": args.steps, "clocks": clk.summary()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -480,6 +530,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=synth.LONG128K.name)
     ap.add_argument("--impl", default="eta", choices=["eta", "reference"])
+    ap.add_argument("--mode", default="decode", choices=["decode", "prefill"],
+                    help="decode: the ETA decode step (default); prefill: eta_prefill")
+    ap.add_argument("--pf-B", type=int, default=4)
+    ap.add_argument("--pf-T", type=int, default=8192)
+    ap.add_argument("--pf-gate-T", type=float, default=0.0)
     ap.add_argument("--cpu-rows", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clock-soak-s", type=float, default=1.0,
@@ -509,6 +564,8 @@ def main():
     try:
         if args.impl == "reference":
             res = run_reference(args, rank, 1, device)
+        elif args.mode == "prefill":
+            res = run_prefill(args, rank, world, device)
         else:
             res = run_eta(args, rank, world, device)
         if rank == 0:

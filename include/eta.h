@@ -242,6 +242,26 @@ eta_status_t eta_set_decode_engine(eta_engine_t engine);
 eta_engine_t eta_get_decode_engine(void);
 
 /*
+ * eta_prefill -- dense gated causal attention of a prefill chunk (the gate of the
+ * review's Methodology Assessment, Eq. 2-3, on every (query, key) pair; the
+ * inference-side counterpart of the paper's dense gated training forward).  For
+ * query position t < lengths[b] of head h (KV head h / G):
+ *   s_t' = scale * q_t . k_t',  t' <= t (causal)
+ *   gated s'' = s' * sigmoid((s' - tau_t) / T)   (T > 0)  or  s' >= tau_t ? s' : 0 (T == 0)
+ *   O[b,h,t] = sum_t' e^{s''} v_t' / sum_t' e^{s''},  lse[b,h,t] = log sum_t' e^{s''}
+ * Q    bf16 [B, Hq, T_max, d] (head-major, like the cache), 16-byte aligned
+ * K, V bf16 [B, Hkv, T_max, d];  tau fp32 [B, Hq, T_max] (per query token and head)
+ * O    fp32 [B, Hq, T_max, d];  lse fp32 [B, Hq, T_max]; rows t >= lengths[b] untouched.
+ * Tensor cores (tcgen05): S = Q K^T and O += P V on 128 x 128 tiles, fp32 TMEM
+ * accumulators, P in bf16.  d = 128 and T_max % 128 == 0 only (else
+ * ETA_ERR_UNSUPPORTED).  No workspace.  dev_status: ETA_DEVSTAT_TIMEOUT.
+ */
+eta_status_t eta_prefill(const eta_dims_t* dims, const eta_bf16_t* Q, const float* tau,
+                         const eta_bf16_t* K, const eta_bf16_t* V, const int32_t* lengths,
+                         float T, float scale, float* O, float* lse, int32_t* dev_status,
+                         void* stream);
+
+/*
  * eta_calibrate_const_tau -- offline calibration of frozen per-head thresholds
  * (abstract: "an offline calibration algorithm ... that freezes per-head constant
  * thresholds").  HOST pointers.  The pages do not print the algorithm; the rule

@@ -30,7 +30,7 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_screen", "eta_decode_workspace_size", "eta_decode", "eta_dense_decode",
            "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string",
            "eta_set_decode_engine", "eta_get_decode_engine", "eta_decode_static",
-           "eta_decode_static_max_workspace", "eta_selftest_wait_timeout")
+           "eta_decode_static_max_workspace", "eta_selftest_wait_timeout", "eta_prefill")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 
 
@@ -89,6 +89,8 @@ def lib() -> C.CDLL:
     L.eta_decode_static.restype = I32
     L.eta_decode_static_max_workspace.argtypes = []
     L.eta_decode_static_max_workspace.restype = C.c_size_t
+    L.eta_prefill.argtypes = [DIMS, P, P, P, P, P, F32, F32, P, P, P, P]
+    L.eta_prefill.restype = I32
     L.eta_selftest_wait_timeout.argtypes = [C.c_uint32, P, P, P]
     L.eta_selftest_wait_timeout.restype = I32
     L.eta_set_decode_engine.argtypes = [I32]
@@ -222,3 +224,11 @@ def eta_selftest_wait_timeout(wait_limit: int, never_set, dev_status, stream=Non
     """Runs the bounded-wait diagnostic kernel (see include/eta.h)."""
     _check("eta_selftest_wait_timeout", lib().eta_selftest_wait_timeout(
         int(wait_limit), _p(never_set), _p(dev_status), _stream(stream)))
+
+
+def eta_prefill(dims: Dims, Q, tau, K, V, lengths, T, scale, O, lse, dev_status=None,
+                stream=None) -> None:
+    """Dense gated causal prefill attention (see include/eta.h)."""
+    _check("eta_prefill", lib().eta_prefill(
+        C.byref(dims), _p(Q), _p(tau), _p(K), _p(V), _p(lengths), float(T), float(scale), _p(O),
+        _p(lse), _p(dev_status), _stream(stream)))

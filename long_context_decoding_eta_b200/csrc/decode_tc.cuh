@@ -347,9 +347,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     bool pending = false;   // stage i-1 still has to be folded into o_acc
     bool ok = true;
 
+    // every lane polls; the warp agrees on the outcome so collectives stay converged
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
     auto correct = [&](int k) -> bool {    // fold PV of stage k into o_acc
       const int pb = k & 1;
-      if (!mbar_wait(&ms->o_full[pb], (uint32_t)(k >> 1) & 1u, abort_flag)) return false;
+      if (!wwait(&ms->o_full[pb], (uint32_t)(k >> 1) & 1u)) return false;
       tc_fence_after();
       float c[16];
       tmem_ld16(tO0 + pb * 16 + lane_sel, c);
@@ -390,7 +394,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     int i = 0;
     for (;; ++i) {
       const int s = i % NSTAGE;
-      if (!mbar_wait(&ms->full[s], (uint32_t)(i / NSTAGE) & 1u, abort_flag)) { ok = false; break; }
+      if (!wwait(&ms->full[s], (uint32_t)(i / NSTAGE) & 1u)) { ok = false; break; }
       const TcStage inf = ms->info[s];
       if (inf.flags) break;
       if (inf.row != cur) {
@@ -408,7 +412,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
       }
       // S of stage i
       const int sb = i & 1;
-      if (!mbar_wait(&ms->s_full[sb], (uint32_t)(i >> 1) & 1u, abort_flag)) { ok = false; break; }
+      if (!wwait(&ms->s_full[sb], (uint32_t)(i >> 1) & 1u)) { ok = false; break; }
       tc_fence_after();
       float sv[16];
       tmem_ld16(tS0 + sb * 16 + lane_sel, sv);

@@ -16,8 +16,9 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline int num_blocks(const eta_dims_t* d) { return d->T_max / d->blk; }
 inline int num_words(const eta_dims_t* d) { return (num_blocks(d) + 31) / 32; }
 
-// Common shape validation.  Returns ETA_OK or the error to report.
-inline eta_status_t check_dims(const eta_dims_t* d) {
+// Common shape validation.  Returns ETA_OK or the error to report.  `rows_in_grid_y`:
+// the caller launches B * Hkv CTAs along grid.y (65535 at most).
+inline eta_status_t check_dims(const eta_dims_t* d, bool rows_in_grid_y = true) {
   if (!d) return ETA_ERR_INVALID_ARG;
   if (d->B <= 0 || d->Hq <= 0 || d->Hkv <= 0 || d->d <= 0 || d->blk <= 0 || d->T_max <= 0)
     return ETA_ERR_INVALID_ARG;
@@ -27,7 +28,7 @@ inline eta_status_t check_dims(const eta_dims_t* d) {
   if (!(d->d == 64 || d->d == 128)) return ETA_ERR_UNSUPPORTED;
   if (!(d->blk == 64 || d->blk == 128)) return ETA_ERR_UNSUPPORTED;
   if (d->T_max % d->blk != 0) return ETA_ERR_UNSUPPORTED;
-  if ((int64_t)d->B * d->Hkv > 65535) return ETA_ERR_UNSUPPORTED;   // grid.y limit
+  if (rows_in_grid_y && (int64_t)d->B * d->Hkv > 65535) return ETA_ERR_UNSUPPORTED;
   if (num_blocks(d) > 65536) return ETA_ERR_UNSUPPORTED;
   if (d->Hq > 256) return ETA_ERR_UNSUPPORTED;
   return ETA_OK;

@@ -71,7 +71,7 @@ extern "C" eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t
                                         const float* W, const float* bias,
                                         const float* tau_const, float* tau, int32_t* dev_status,
                                         void* stream) {
-  eta_status_t st = check_dims(dims);
+  eta_status_t st = check_dims(dims, /*rows_in_grid_y=*/false);   // grid (B, Hkv)
   if (st != ETA_OK) return st;
   if (!tau) return ETA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

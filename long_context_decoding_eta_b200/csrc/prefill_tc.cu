@@ -1,0 +1,455 @@
+// Dense gated causal attention for a prefill chunk on the tensor cores (tcgen05).
+//
+// The gate of the evolve.pub review of arXiv 2609.20888 (Methodology Assessment,
+// Eq. 2-3: m = sigmoid(beta (S - tau)), gated logits S * m) applied to every
+// (query, key) pair of a causal prefill, with beta = 1/T (T = 0: hard gate); the
+// inference-side counterpart of the paper's dense gated training forward.
+//
+// One CTA per (batch row, query head, 128-query tile), 192 threads:
+//   warp 4  TMA producer: the 128 x 128 query tile once, then 128-key K and V
+//           tiles (two 64-dim boxes each, 128-byte swizzle) into a 2-stage ring
+//   warp 5  MMA issuer: S = Q K^T (M = 128 queries, N = 128 keys, K = d) into one of
+//           two TMEM buffers, then O += P V (M = 128 queries, N = d, K = 128 keys,
+//           V read MN-major from its swizzled tile) into the TMEM accumulator
+//   warps 0-3 softmax, thread = query row = TMEM lane: causal mask, gate, running
+//           row max; O is rescaled in TMEM only when the row max grew by more than
+//           kRescale (FA-style conditional rescaling), P is written as bf16 into a
+//           swizzled shared tile (the A operand of P V).
+// TMEM: S 2 x 128 columns, O 128 columns (512 allocated).  Every wait is bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "decode_tc.cuh"
+#include "eta_common.cuh"
+#include "eta_host.h"
+
+namespace eta {
+namespace pf {
+
+using tc::mma_commit;
+using tc::mma_f16;
+using tc::smem_desc;
+using tc::tc_fence_after;
+using tc::tc_fence_before;
+using tc::fence_async_smem;
+using tc::tma_load_2d;
+
+constexpr int D = 128;
+constexpr int TILE = 128;                       // queries per CTA, keys per KV tile
+constexpr int HALF = TILE * 128;                // [128 rows x 64 dims] bf16 = 16 KB
+constexpr int NKV = 2;                          // KV ring stages
+constexpr int OFF_Q = 0;                        // 2 halves
+constexpr int OFF_KV = 2 * HALF;                // stage s: K0 K1 V0 V1
+constexpr int KV_STAGE = 4 * HALF;              // 64 KB
+constexpr int OFF_P = OFF_KV + NKV * KV_STAGE;  // 2 buffers x 2 halves
+constexpr int OFF_MISC = OFF_P + 2 * 2 * HALF;
+constexpr int NWARP_SM = 4;
+constexpr int NT = (NWARP_SM + 2) * 32;
+constexpr int kTmemCols = 512;
+constexpr float kRescale = 8.0f;                // rescale O when the max grows by > 8 (e^8)
+
+struct Misc {
+  uint64_t q_full, kv_full[NKV], kv_empty[NKV];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done, fin;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr int SMEM_BYTES = OFF_MISC + (int)sizeof(Misc) + 1024;
+
+// kind::f16, D fp32, A/B bf16, M = 128, N = 128
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) |
+                                ((128u >> 4) << 24);
+constexpr uint32_t kIdescQK = kIdescBase;                 // A, B K-major
+constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);    // A K-major, B (V) MN-major
+
+ETA_DEV void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+ETA_DEV void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::
+          "r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+ETA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+ETA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+struct PrefillParams {
+  int Hq, Hkv, T_max, ntiles;
+  float scale, invT;      // invT < 0: hard gate
+  const float* tau;       // [B, Hq, T_max]
+  const int32_t* lengths;
+  float* O;               // [B, Hq, T_max, d]
+  float* lse;             // [B, Hq, T_max]
+  int32_t* status;
+};
+
+template <int G>
+__global__ void __launch_bounds__(NT, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  ETA_PDL_ENTRY();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Misc* ms = reinterpret_cast<Misc*>(smem + OFF_MISC);
+  volatile int* abort_flag = &ms->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // heaviest tiles (most keys) first
+  const int qt = p.ntiles - 1 - (int)(blockIdx.x % p.ntiles);
+  const int bh = blockIdx.x / p.ntiles;
+  const int b = bh / p.Hq, h = bh % p.Hq, g = h / G;
+  const int len = min(max(p.lengths[b], 0), p.T_max);
+  const int q0 = qt * TILE;
+  if (q0 >= len) return;                              // uniform, before any barrier
+  const int nkv = (min(q0 + TILE, len) + TILE - 1) / TILE;   // key tiles 0 .. nkv-1
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ms->q_full, 1);
+    for (int s = 0; s < NKV; ++s) {
+      mbar_init(&ms->kv_full[s], 1);
+      mbar_init(&ms->kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ms->s_full[i], 1);
+      mbar_init(&ms->s_free[i], NWARP_SM);
+      mbar_init(&ms->p_full[i], NWARP_SM);
+    }
+    mbar_init(&ms->o_done, 1);
+    mbar_init(&ms->fin, 1);
+    ms->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == NWARP_SM + 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&ms->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+  const uint32_t tS = tmem, tO = tmem + 256;
+
+  if (warp == NWARP_SM) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      const int qrow = (b * p.Hq + h) * p.T_max + q0;
+      mbar_arrive_expect_tx(&ms->q_full, 2 * HALF);
+      tma_load_2d(smem + OFF_Q, &tmQ, 0, qrow, &ms->q_full);
+      tma_load_2d(smem + OFF_Q + HALF, &tmQ, 64, qrow, &ms->q_full);
+      int j = 0;
+      for (; j < nkv && ok; ++j) {
+        const int s = j % NKV;
+        if (!mbar_wait(&ms->kv_empty[s], ((uint32_t)(j / NKV) & 1u) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        unsigned char* st = smem + OFF_KV + s * KV_STAGE;
+        const int krow = (b * p.Hkv + g) * p.T_max + j * TILE;
+        mbar_arrive_expect_tx(&ms->kv_full[s], 4 * HALF);
+        tma_load_2d(st, &tmK, 0, krow, &ms->kv_full[s]);
+        tma_load_2d(st + HALF, &tmK, 64, krow, &ms->kv_full[s]);
+        tma_load_2d(st + 2 * HALF, &tmV, 0, krow, &ms->kv_full[s]);
+        tma_load_2d(st + 3 * HALF, &tmV, 64, krow, &ms->kv_full[s]);
+      }
+      if (!ok) {
+        set_status(p.status, ETA_DEVSTAT_TIMEOUT);
+        *abort_flag = 1;
+        mbar_wait(&ms->q_full, 0, nullptr);
+        for (int k = max(0, j - NKV); k < j; ++k)
+          mbar_wait(&ms->kv_full[k % NKV], (uint32_t)(k / NKV) & 1u, nullptr);
+      }
+    }
+  } else if (warp == NWARP_SM + 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&ms->q_full, 0, abort_flag);
+      const uint32_t qa = smem_u32(smem + OFF_Q);
+      auto issue_pv = [&](int k) -> bool {
+        const int s = k % NKV, pb = k & 1;
+        if (!mbar_wait(&ms->p_full[pb], (uint32_t)(k >> 1) & 1u, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(smem + OFF_P + pb * 2 * HALF);
+        const uint32_t v0 = smem_u32(smem + OFF_KV + s * KV_STAGE + 2 * HALF);
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) {
+          const uint32_t aoff = (uint32_t)(kk >> 2) * HALF + (uint32_t)(kk & 3) * 32;
+          mma_f16(tO, smem_desc(pa + aoff, 16, 1024, tc::kSwizzle128),
+                  smem_desc(v0 + kk * 2048, HALF, 1024, tc::kSwizzle128), kIdescPV,
+                  (k > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&ms->o_done);
+        mma_commit(&ms->kv_empty[s]);
+        return true;
+      };
+      int j = 0;
+      for (; j < nkv && ok; ++j) {
+        const int s = j % NKV, sb = j & 1;
+        if (!mbar_wait(&ms->kv_full[s], (uint32_t)(j / NKV) & 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&ms->s_free[sb], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ka = smem_u32(smem + OFF_KV + s * KV_STAGE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * HALF + (uint32_t)(kk & 3) * 32;
+          mma_f16(tS + sb * 128, smem_desc(qa + off, 16, 1024, tc::kSwizzle128),
+                  smem_desc(ka + off, 16, 1024, tc::kSwizzle128), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&ms->s_full[sb]);
+        if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && nkv > 0) ok = issue_pv(nkv - 1);
+      if (!ok) {
+        set_status(p.status, ETA_DEVSTAT_TIMEOUT);
+        *abort_flag = 1;
+      }
+      mma_commit(&ms->fin);
+      mbar_wait(&ms->fin, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int row = threadIdx.x;                      // query row of the tile = TMEM lane
+    const int tq = q0 + row;
+    const uint32_t lsel = (uint32_t)(warp * 32) << 16;
+    const float tau = (tq < p.T_max) ? p.tau[((size_t)b * p.Hq + h) * p.T_max + tq] : 0.f;
+    // l: row sum of the bf16-rounded weights (normalizes O, which the tensor core
+    // built from those weights); lx: row sum of the exact fp32 weights (for lse)
+    float m_used = -INFINITY, l = 0.f, lx = 0.f;
+    bool ok = true;
+    float sv[TILE];
+    // every lane polls; the warp agrees on the outcome so collectives stay converged
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    for (int j = 0; j < nkv; ++j) {
+      const int sb = j & 1, s = j % NKV;
+      if (!wwait(&ms->s_full[sb], (uint32_t)(j >> 1) & 1u)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < TILE / 32; ++c) tmem_ld32(tS + sb * 128 + c * 32 + lsel, sv + c * 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->s_free[sb]);
+      const int k0 = j * TILE;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < TILE; ++c) {
+        const float x = p.scale * sv[c];
+        float y = x;
+        if (p.invT < 0.f) y = x >= tau ? x : 0.f;
+        else y = x * __frcp_rn(1.f + __expf((tau - x) * p.invT));
+        y = (k0 + c <= tq) ? y : -INFINITY;
+        sv[c] = y;
+        mx = fmaxf(mx, y);
+      }
+      // running max: the first tile sets it; later tiles rescale O (in TMEM) only
+      // when the max grew by more than kRescale
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_used == -INFINITY) {
+        m_used = mx;
+      } else if (mx > m_used + kRescale) {
+        alpha = __expf(m_used - mx);
+        m_used = mx;
+        resc = true;
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        // O holds tiles 0 .. j-1: wait for the last P V before touching it (P V of
+        // tile j-2 is known complete: it was issued before Q K^T of tile j)
+        if (!wwait(&ms->o_done, (uint32_t)((j - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        float ov[32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          tmem_ld32(tO + c * 32 + lsel, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          tmem_st32(tO + c * 32 + lsel, ov);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        l *= alpha;
+        lx *= alpha;
+      }
+      // P = exp(s' - m) as bf16, row `row` of the swizzled A tile (two 64-key halves)
+      unsigned char* pbuf = smem + OFF_P + sb * 2 * HALF;
+      float ls = 0.f, lsx = 0.f;
+#pragma unroll
+      for (int cch = 0; cch < TILE / 8; ++cch) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = __expf(sv[cch * 8 + 2 * e] - m_used);
+          const float p1 = __expf(sv[cch * 8 + 2 * e + 1] - m_used);
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+          // the row sum uses the rounded weights the tensor core multiplies, so
+          // O / l is an exact convex combination of them (a dominant weight's
+          // rounding cancels between numerator and denominator)
+          const float2 pf = __bfloat1622float2(pr);
+          ls += pf.x + pf.y;
+          lsx += p0 + p1;
+          w[e] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        const int half = cch >> 3, c16 = cch & 7;
+        *reinterpret_cast<uint4*>(pbuf + half * HALF + row * 128 + ((c16 ^ (row & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l += ls;
+      lx += lsx;
+      // the last key tile: V rows past the sequence end must be finite for P V
+      if (k0 + TILE > len && k0 + row >= len) {
+        unsigned char* vt = smem + OFF_KV + s * KV_STAGE + 2 * HALF;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          *reinterpret_cast<uint4*>(vt + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vt + HALF + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->p_full[sb]);
+    }
+    // the last two P V: wait phase by phase so the parity never aliases
+    if (ok && nkv >= 2 && !wwait(&ms->o_done, (uint32_t)((nkv - 2) & 1))) ok = false;
+    if (ok && !wwait(&ms->o_done, (uint32_t)((nkv - 1) & 1))) ok = false;
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      const bool store = tq < len;
+      float* orow = p.O + (((size_t)b * p.Hq + h) * p.T_max + (store ? tq : 0)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float ov[32];
+        tmem_ld32(tO + c * 32 + lsel, ov);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(orow + c * 32 + i) =
+                make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+        }
+      }
+      if (store) p.lse[((size_t)b * p.Hq + h) * p.T_max + tq] = m_used + logf(lx);
+    } else {
+      if (threadIdx.x == 0) set_status(p.status, ETA_DEVSTAT_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == NWARP_SM + 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
+  }
+}
+
+}  // namespace pf
+
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+static EncodeFn prefill_encode() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  }
+  return fn;
+}
+
+static bool prefill_map(CUtensorMap* m, const void* base, uint64_t rows) {
+  EncodeFn fn = prefill_encode();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {128, rows};
+  cuuint64_t gstride[1] = {256};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int G>
+static eta_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk,
+                                   const CUtensorMap& mv, const pf::PrefillParams& prm,
+                                   int ctas, cudaStream_t s) {
+  if (!set_smem_once<pf::prefill_tc_kernel<G>>(pf::SMEM_BYTES)) return ETA_ERR_CUDA;
+  return launch_k(pf::prefill_tc_kernel<G>, dim3(ctas), dim3(pf::NT), pf::SMEM_BYTES, s, mq, mk,
+                  mv, prm);
+}
+
+}  // namespace eta
+
+using namespace eta;
+
+extern "C" eta_status_t eta_prefill(const eta_dims_t* dims, const eta_bf16_t* Q, const float* tau,
+                                    const eta_bf16_t* K, const eta_bf16_t* V,
+                                    const int32_t* lengths, float T, float scale, float* O,
+                                    float* lse, int32_t* dev_status, void* stream) {
+  eta_status_t st = check_dims(dims, /*rows_in_grid_y=*/false);   // 1-D grid
+  if (st != ETA_OK) return st;
+  if (!Q || !tau || !K || !V || !lengths || !O || !lse) return ETA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return ETA_ERR_INVALID_ARG;
+  if (!(T >= 0.f) || isinf(T)) return ETA_ERR_INVALID_ARG;
+  if (dims->d != 128 || dims->T_max % pf::TILE != 0) return ETA_ERR_UNSUPPORTED;
+  const uint64_t kv_rows = (uint64_t)dims->B * dims->Hkv * dims->T_max;
+  const uint64_t q_rows = (uint64_t)dims->B * dims->Hq * dims->T_max;
+  if (q_rows >= (1ull << 31)) return ETA_ERR_UNSUPPORTED;
+  const int ntiles = dims->T_max / pf::TILE;
+  const int64_t ctas = (int64_t)dims->B * dims->Hq * ntiles;
+  if (ctas > 0x7fffffff) return ETA_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv;
+  if (!prefill_map(&mq, Q, q_rows) || !prefill_map(&mk, K, kv_rows) ||
+      !prefill_map(&mv, V, kv_rows))
+    return ETA_ERR_CUDA;
+  pf::PrefillParams prm;
+  prm.Hq = dims->Hq; prm.Hkv = dims->Hkv; prm.T_max = dims->T_max; prm.ntiles = ntiles;
+  prm.scale = scale == 0.f ? 1.f / sqrtf((float)dims->d) : scale;
+  prm.invT = T == 0.f ? -1.f : 1.f / T;
+  prm.tau = tau; prm.lengths = lengths; prm.O = O; prm.lse = lse; prm.status = dev_status;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (dims->Hq / dims->Hkv) {
+    case 1: return launch_prefill<1>(mq, mk, mv, prm, (int)ctas, s);
+    case 2: return launch_prefill<2>(mq, mk, mv, prm, (int)ctas, s);
+    case 4: return launch_prefill<4>(mq, mk, mv, prm, (int)ctas, s);
+    case 8: return launch_prefill<8>(mq, mk, mv, prm, (int)ctas, s);
+  }
+  return ETA_ERR_UNSUPPORTED;
+}

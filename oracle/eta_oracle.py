@@ -309,6 +309,26 @@ def softmax_attention(q_h: np.ndarray, K_seq: np.ndarray, V_seq: np.ndarray,
     return _softmax_out(s, V_seq[:n_valid])
 
 
+def prefill(q: np.ndarray, tau: np.ndarray, K: np.ndarray, V: np.ndarray,
+            lengths: Sequence[int], scale: float, T: float):
+    """Dense gated causal attention of a prefill chunk (Eq. 2-3 on every pair).
+
+    q [B, Hq, T_max, d] (query at position t of row b), tau [B, Hq, T_max],
+    K/V [B, Hkv, T_max, d].  Query t < lengths[b] attends keys 0..t of its KV
+    head h // G with gated logits; returns O [B, Hq, T_max, d], lse [B, Hq, T_max]
+    (rows t >= lengths[b] left at zero)."""
+    B, Hq, Tm, d = q.shape
+    G = Hq // K.shape[1]
+    o = np.zeros((B, Hq, Tm, d))
+    lse = np.zeros((B, Hq, Tm))
+    for b in range(B):
+        for h in range(Hq):
+            for t in range(int(lengths[b])):
+                o[b, h, t], lse[b, h, t] = dense_gated(q[b, h, t], float(tau[b, h, t]),
+                                                       K[b, h // G], V[b, h // G], t + 1, scale, T)
+    return o, lse
+
+
 def dense_decode(q, K, V, lengths, scale):
     """Textbook decode attention for every (b, h), GQA group h // G."""
     B, Hq, d = q.shape

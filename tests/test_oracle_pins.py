@@ -519,3 +519,63 @@ def test_per_dimension_variance_bound_brute_force_values():
     want = c @ qv + min(np.linalg.norm(qv) * m["rmax"][0],
                         1.5 * math.sqrt(sum(qv[i] ** 2 * m["vardim"][0][i] for i in range(5))))
     assert abs(ub[0] - want) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# dense gated causal prefill
+# --------------------------------------------------------------------------
+def _prefill_case(seed=30, B=2, Hq=4, Hkv=2, d=8, T=40):
+    rng = np.random.default_rng(seed)
+    q = rng.normal(size=(B, Hq, T, d))
+    K = rng.normal(size=(B, Hkv, T, d))
+    V = rng.normal(size=(B, Hkv, T, d))
+    return q, K, V, np.array([T, T - 13])
+
+
+@pytest.mark.parametrize("T_gate", [0.0, 0.05])
+def test_prefill_tau_neg_inf_is_causal_softmax_attention(T_gate):
+    q, K, V, L = _prefill_case()
+    scale = O.default_scale(q.shape[-1])
+    tau = np.full(q.shape[:3], -np.inf)
+    o, lse = O.prefill(q, tau, K, V, L, scale, T_gate)
+    G = q.shape[1] // K.shape[1]
+    Kt = torch.from_numpy(K).repeat_interleave(G, 1)
+    Vt = torch.from_numpy(V).repeat_interleave(G, 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q), Kt, Vt,
+                                                           is_causal=True, scale=scale).numpy()
+    s = torch.einsum("bhtd,bhsd->bhts", torch.from_numpy(q), Kt) * scale
+    s = s.masked_fill(torch.triu(torch.ones(q.shape[2], q.shape[2], dtype=torch.bool), 1),
+                      -math.inf)
+    ref_lse = torch.logsumexp(s, -1).numpy()
+    for b in range(q.shape[0]):
+        n = L[b]
+        np.testing.assert_allclose(o[b, :, :n], ref[b, :, :n], atol=1e-12)
+        np.testing.assert_allclose(lse[b, :, :n], ref_lse[b, :, :n], atol=1e-12)
+        assert np.all(o[b, :, n:] == 0)
+
+
+def test_prefill_tau_above_scores_is_cumulative_mean():
+    q, K, V, L = _prefill_case(seed=31)
+    tau = np.full(q.shape[:3], 1e6)
+    o, lse = O.prefill(q, tau, K, V, L, 1.0, 0.0)
+    G = q.shape[1] // K.shape[1]
+    for b in range(q.shape[0]):
+        for h in range(q.shape[1]):
+            cm = np.cumsum(V[b, h // G], axis=0) / np.arange(1, q.shape[2] + 1)[:, None]
+            np.testing.assert_allclose(o[b, h, :L[b]], cm[:L[b]], atol=1e-12)
+            np.testing.assert_allclose(lse[b, h, :L[b]], np.log(np.arange(1, L[b] + 1)), atol=1e-12)
+
+
+def test_prefill_row_equals_gated_decode_over_its_prefix():
+    """Query t of a prefill is the decode of query t over the cache prefix 0..t."""
+    q, K, V, L = _prefill_case(seed=32)
+    rng = np.random.default_rng(33)
+    tau = rng.normal(size=q.shape[:3]) * 0.3
+    scale = O.default_scale(q.shape[-1])
+    o, lse = O.prefill(q, tau, K, V, L, scale, 0.0)
+    G = q.shape[1] // K.shape[1]
+    for (b, h, t) in [(0, 0, 0), (0, 3, 17), (1, 2, 26), (1, 1, 5)]:
+        s = scale * K[b, h // G, :t + 1] @ q[b, h, t]
+        sp = np.where(s >= tau[b, h, t], s, 0.0)
+        p = np.exp(sp - sp.max())
+        np.testing.assert_allclose(o[b, h, t], p @ V[b, h // G, :t + 1] / p.sum(), atol=1e-12)

@@ -51,7 +51,7 @@ constexpr float kRescale = 8.0f;                // rescale O when the max grows 
 
 struct Misc {
   uint64_t q_full, kv_full[NKV], kv_empty[NKV];
-  uint64_t s_full[2], s_free[2], p_full[2], o_done, fin;
+  uint64_t s_full[2], s_free[2], p_full[2], o_done, o_final, fin;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -143,6 +143,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       mbar_init(&ms->p_full[i], NWARP_SM);
     }
     mbar_init(&ms->o_done, 1);
+    mbar_init(&ms->o_final, 1);
     mbar_init(&ms->fin, 1);
     ms->abort_flag = 0;
     fence_mbar_init();
@@ -229,6 +230,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok && nkv > 0) ok = issue_pv(nkv - 1);
+      // one-phase barrier for "every P V done": o_done's parity can alias once two of
+      // its phases complete before a waiter looks
+      if (ok) mma_commit(&ms->o_final);
       if (!ok) {
         set_status(p.status, ETA_DEVSTAT_TIMEOUT);
         *abort_flag = 1;
@@ -262,17 +266,24 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->s_free[sb]);
       const int k0 = j * TILE;
-      float mx = -INFINITY;
+      // 8 independent partial maxima: short dependency chains
+      float pm[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+      const bool hard = p.invT < 0.f;
+      const int lim = tq - k0;                         // keys c <= lim are causal
 #pragma unroll
       for (int c = 0; c < TILE; ++c) {
         const float x = p.scale * sv[c];
-        float y = x;
-        if (p.invT < 0.f) y = x >= tau ? x : 0.f;
-        else y = x * __frcp_rn(1.f + __expf((tau - x) * p.invT));
-        y = (k0 + c <= tq) ? y : -INFINITY;
+        float y;
+        if (hard) y = x >= tau ? x : 0.f;
+        else y = __fdividef(x, 1.f + __expf((tau - x) * p.invT));   // x * sigmoid
+        y = (c <= lim) ? y : -INFINITY;
         sv[c] = y;
-        mx = fmaxf(mx, y);
+        pm[c & 7] = fmaxf(pm[c & 7], y);
       }
+      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       // running max: the first tile sets it; later tiles rescale O (in TMEM) only
       // when the max grew by more than kRescale
       float alpha = 1.f;
@@ -305,7 +316,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       }
       // P = exp(s' - m) as bf16, row `row` of the swizzled A tile (two 64-key halves)
       unsigned char* pbuf = smem + OFF_P + sb * 2 * HALF;
-      float ls = 0.f, lsx = 0.f;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f}, lx4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int cch = 0; cch < TILE / 8; ++cch) {
         uint32_t w[4];
@@ -318,16 +329,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           // O / l is an exact convex combination of them (a dominant weight's
           // rounding cancels between numerator and denominator)
           const float2 pf = __bfloat1622float2(pr);
-          ls += pf.x + pf.y;
-          lsx += p0 + p1;
+          ls4[e] += pf.x + pf.y;
+          lx4[e] += p0 + p1;
           w[e] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         const int half = cch >> 3, c16 = cch & 7;
         *reinterpret_cast<uint4*>(pbuf + half * HALF + row * 128 + ((c16 ^ (row & 7)) << 4)) =
             make_uint4(w[0], w[1], w[2], w[3]);
       }
-      l += ls;
-      lx += lsx;
+      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+      lx += (lx4[0] + lx4[1]) + (lx4[2] + lx4[3]);
       // the last key tile: V rows past the sequence end must be finite for P V
       if (k0 + TILE > len && k0 + row >= len) {
         unsigned char* vt = smem + OFF_KV + s * KV_STAGE + 2 * HALF;
@@ -341,9 +352,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms->p_full[sb]);
     }
-    // the last two P V: wait phase by phase so the parity never aliases
-    if (ok && nkv >= 2 && !wwait(&ms->o_done, (uint32_t)((nkv - 2) & 1))) ok = false;
-    if (ok && !wwait(&ms->o_done, (uint32_t)((nkv - 1) & 1))) ok = false;
+    // every P V done (a single-phase barrier: no parity aliasing)
+    if (ok && !wwait(&ms->o_final, 0u)) ok = false;
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l;

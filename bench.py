@@ -39,6 +39,7 @@ METRIC = "decode attn steps/s and HBM GB/s on admitted KV bytes (% of B200 peak)
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 LAUNCHES_PER_STEP = 7   # meta tail 1 + tau 1 + screen 2 + decode 3 (plan, decode, combine)
+LAUNCHES_PER_FUSED_STEP = 1   # eta_decode_step: one persistent kernel
 
 
 def peaks():
@@ -71,13 +72,12 @@ def density_offset(bounds: np.ndarray, tau0: np.ndarray, valid: np.ndarray, dens
     return float(np.partition(v, k)[k])
 
 
-def decode_traffic(admitted_kv: int, engine_tc: bool):
-    """DRAM bytes per decode launch from the committed ncu capture
-    (profiles/decode_tc_traffic.json), scaled to this workload by its admitted K/V
-    bytes; None when the kernel source changed since the capture or the capture
-    does not cover the engine that ran."""
+def decode_traffic(admitted_kv: int, engine_tc: bool, record: str = "decode_tc_traffic.json"):
+    """DRAM bytes per launch from a committed ncu capture (profiles/<record>), scaled
+    to this workload by its admitted K/V bytes; None when the kernel source changed
+    since the capture or the capture does not cover the engine that ran."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", "decode_tc_traffic.json")
+    p = os.path.join(ROOT, "profiles", record)
     if not engine_tc or not os.path.exists(p):
         return None
     rec = json.load(open(p))
@@ -164,11 +164,11 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def setup(w: synth.Workload, device, rank: int, cent_format: str = "f32"):
+def setup(w: synth.Workload, device, rank: int, cent_format: str = "f32", fused: bool = False):
     from long_context_decoding_eta_b200.api import EtaDecoder
     g = synth.generate(w, device, seed=w.seed + 7919 * rank)
     dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, bound=w.bound, z=w.z,
-                     T=w.gate_T, keep_bounds=True, cent_format=cent_format)
+                     T=w.gate_T, keep_bounds=True, cent_format=cent_format, fused=fused)
     dec.build_meta()
     # workload calibration: bias so that tau hits the density target
     if w.tau_mode == "const":
@@ -218,7 +218,8 @@ def run_eta(args, rank, world, device):
     from long_context_decoding_eta_b200 import _lib
     _lib.eta_set_decode_engine(args.engine)
     w = workload_by_name(args.workload, args.B)
-    g, dec, W, bias, tau_const = setup(w, device, rank, args.cent)
+    fused = bool(args.fused)
+    g, dec, W, bias, tau_const = setup(w, device, rank, args.cent, fused)
     q = g["q"]
     stream = torch.cuda.current_stream()
     # one step to measure densities / bytes, then check status
@@ -228,9 +229,19 @@ def run_eta(args, rank, world, device):
     by = step_bytes(dec, w)
 
     if args.graph:
-        g_pre, g_dec = dec.capture(q, W, bias, tau_const, split=True)
+        g_pre, g_dec = dec.capture(q, W, bias, tau_const, split=not fused)
 
     def one_step(ev=None):
+        if fused:        # the whole step is the one launch the events bracket
+            if ev is not None:
+                ev[0].record(stream)
+            if args.graph:
+                g_pre.replay()
+            else:
+                dec.step_fused(q, W, bias, tau_const)
+            if ev is not None:
+                ev[1].record(stream)
+            return
         if args.graph:
             g_pre.replay()
         else:
@@ -314,7 +325,9 @@ def run_eta(args, rank, world, device):
 
     peak, peak_kind = peaks()
     ms_step = ms / args.steps
-    achieved = by["decode"] / (dec_ms * 1e-3) / 1e9
+    # the dominant kernel: eta_decode's three launches, or the fused step's one launch
+    # (which also reads the screened metadata: its algorithmic bytes are the step's)
+    achieved = (by["step"] if fused else by["decode"]) / (dec_ms * 1e-3) / 1e9
     res = {
         "metric": METRIC,
         "value": job_throughput(world, args.steps, ms),
@@ -332,7 +345,7 @@ def run_eta(args, rank, world, device):
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
             "context": w.ctx, "blk": w.blk, "bound": w.bound, "gate_T": w.gate_T,
             "tau_mode": w.tau_mode, "engine": args.engine, "centroids": args.cent,
-            "cuda_graph": bool(args.graph),
+            "cuda_graph": bool(args.graph), "fused_step": fused,
             "density_target": f"{w.density:.2f} {w.density_kind}",
             "union_density": round(by["union_density"], 4),
             "head_density": round(by["head_density"], 4),
@@ -343,22 +356,28 @@ def run_eta(args, rank, world, device):
         "hbm_frac_of_nominal_8tbs": by["step"] / (ms_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
         "bytes_per_step": {"admitted_kv": by["admitted_kv"], "metadata": by["meta"],
                            "total": by["step"], "dense_kv": by["dense_kv"]},
-        "roofline": {"kernel": "eta_decode (plan + split-KV decode + combine)", "bound": "hbm",
+        "roofline": {"kernel": ("eta_decode_step (one persistent kernel: tail metadata, tau, "
+                                "screen, decode, merge)") if fused else
+                               "eta_decode (plan + split-KV decode + combine)", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
                      "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                      "decode_ms": dec_ms,
-                     "traffic": decode_traffic(by["admitted_kv"], w.d == 128 and
-                                               args.engine in ("auto", "tcgen05")),
-                     "traffic_source": "profiles/decode_tc_traffic.json (ncu dram__bytes_read"
-                                       "+write of one full-size launch, scaled by admitted KV)"},
+                     "traffic": decode_traffic(
+                         by["admitted_kv"], w.d == 128 and (fused or args.engine in
+                                                            ("auto", "tcgen05")),
+                         "step_fused_traffic.json" if fused else "decode_tc_traffic.json"),
+                     "traffic_source": ("profiles/step_fused_traffic.json" if fused else
+                                        "profiles/decode_tc_traffic.json") +
+                                       " (ncu dram__bytes_read+write of one full-size launch, "
+                                       "scaled by admitted KV)"},
         "dense_baseline": {"ms": dense_ms, "steps_per_s_decode_only": 1e3 / dense_ms,
                            "gbs": by["dense_kv"] / (dense_ms * 1e-3) / 1e9,
                            "speedup_of_eta_decode": dense_ms / dec_ms},
         "e2e": {"value": job_throughput(world, 1, e2e_ms), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host.numel() * 2,
                 "d2h_bytes_per_step": o_host.numel() * 4 + lse_host.numel() * 4},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": (LAUNCHES_PER_FUSED_STEP if fused else LAUNCHES_PER_STEP) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -542,6 +561,8 @@ def main():
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     ap.add_argument("--engine", default="auto", choices=["auto", "tcgen05", "fma"],
                     help="decode engine of libeta.so")
+    ap.add_argument("--fused", action="store_true",
+                    help="run the step as one eta_decode_step launch (persistent kernel)")
     ap.add_argument("--graph", action="store_true",
                     help="replay the step as CUDA graphs (launch-bound small workloads)")
     ap.add_argument("--cent", default="bf16", choices=["f32", "bf16"],

@@ -217,6 +217,43 @@ eta_status_t eta_decode_static(const eta_dims_t* dims, const eta_bf16_t* q, cons
 size_t eta_decode_static_max_workspace(void);
 
 /*
+ * eta_decode_step -- the whole decode step in one launch: on append (update_tail != 0)
+ * the tail block's metadata as eta_build_block_meta(ETA_TAIL_BLOCK), then the
+ * thresholds as eta_predict_tau (W/bias, or the frozen tau_const when non-NULL),
+ * the screening as eta_screen and the decode as eta_decode with ETA_PRUNE_SKIP.
+ * (Arithmetic of those four calls: abstract of arXiv 2609.20888 for the cached
+ * bounds, O(1) screening and co-admission; evolve.pub review, Methodology
+ * Assessment, Eq. 1 for tau and Eq. 2-3 for the gate.)  Every output equals, bit for
+ * bit, what the four separate calls write with the same arguments: tau, head_mask,
+ * union_idx, union_cnt, head_cnt (nullable), o, lse, and the refreshed metadata.
+ * One difference: a block at or past lengths[b] is never admitted, whatever its
+ * cnt says (the separate calls rely on cnt alone).
+ * Layouts: as the four calls.  cent_format / cent / rmax / var / vardim / cnt as
+ * eta_screen (vardim nullable unless bound == ETA_BOUND_PROB_DIM; when given it is
+ * refreshed with the tail block too); z for the probabilistic bounds; T: 0 = hard
+ * gate; scale 0 = 1/sqrt(d).
+ * One persistent cooperative kernel, one CTA per SM (no other kernel may hold SMs
+ * the launch needs; else ETA_ERR_CUDA).  Requires d = 128, NB % 4 == 0, 16-byte
+ * aligned q, K, V and metadata (else ETA_ERR_UNSUPPORTED / ETA_ERR_INVALID_ARG).
+ * FLOOR pruning is not offered here (use the separate calls).
+ * Workspace: eta_decode_step_workspace_size(dims) bytes, 16-byte aligned, zero-filled
+ * once before the first call (it holds self-resetting counters) and again after any
+ * call whose dev_status came back with ETA_DEVSTAT_TIMEOUT.  Calls sharing one
+ * workspace must not overlap on the GPU.
+ * dev_status: ETA_DEVSTAT_TIMEOUT (a bounded wait ran out), _NONFINITE_Q, _BAD_BLOCK.
+ */
+size_t eta_decode_step_workspace_size(const eta_dims_t* dims);
+eta_status_t eta_decode_step(const eta_dims_t* dims, const eta_bf16_t* q, const float* W,
+                             const float* bias, const float* tau_const, const eta_bf16_t* K,
+                             const eta_bf16_t* V, const int32_t* lengths, int32_t update_tail,
+                             eta_cent_format_t cent_format, void* cent, float* rmax,
+                             float* var, float* vardim, int32_t* cnt, eta_bound_t bound,
+                             float z, float T, float scale, float* tau, uint32_t* head_mask,
+                             int32_t* union_idx, int32_t* union_cnt, int32_t* head_cnt,
+                             float* o, float* lse, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream);
+
+/*
  * eta_dense_decode -- the dense baseline the speedups are measured against (the
  * pages compare with FlashAttention-2 decode): standard softmax decode attention
  * over every valid key, no threshold, no gate, same split-KV pipeline as eta_decode.

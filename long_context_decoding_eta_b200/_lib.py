@@ -30,7 +30,8 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_screen", "eta_decode_workspace_size", "eta_decode", "eta_dense_decode",
            "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string",
            "eta_set_decode_engine", "eta_get_decode_engine", "eta_decode_static",
-           "eta_decode_static_max_workspace", "eta_selftest_wait_timeout", "eta_prefill")
+           "eta_decode_static_max_workspace", "eta_selftest_wait_timeout", "eta_prefill",
+           "eta_decode_step_workspace_size", "eta_decode_step")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 
 
@@ -91,6 +92,11 @@ def lib() -> C.CDLL:
     L.eta_decode_static_max_workspace.restype = C.c_size_t
     L.eta_prefill.argtypes = [DIMS, P, P, P, P, P, F32, F32, P, P, P, P]
     L.eta_prefill.restype = I32
+    L.eta_decode_step_workspace_size.argtypes = [DIMS]
+    L.eta_decode_step_workspace_size.restype = C.c_size_t
+    L.eta_decode_step.argtypes = [DIMS, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P, I32, F32,
+                                  F32, F32, P, P, P, P, P, P, P, P, C.c_size_t, P, P]
+    L.eta_decode_step.restype = I32
     L.eta_selftest_wait_timeout.argtypes = [C.c_uint32, P, P, P]
     L.eta_selftest_wait_timeout.restype = I32
     L.eta_set_decode_engine.argtypes = [I32]
@@ -176,6 +182,24 @@ def eta_decode_static(dims: Dims, q, tau, K, V, lengths, union_idx, union_cnt, T
         _p(union_cnt), float(T), float(scale),
         PRUNE[prune] if isinstance(prune, str) else int(prune), _p(vsum), _p(cnt), _p(o),
         _p(lse), _p(dev_status), _stream(stream)))
+
+
+def eta_decode_step_workspace_size(dims: Dims) -> int:
+    return int(lib().eta_decode_step_workspace_size(C.byref(dims)))
+
+
+def eta_decode_step(dims: Dims, q, W, bias, tau_const, K, V, lengths, update_tail, cent, rmax,
+                    var, vardim, cnt, bound, z, T, scale, tau, head_mask, union_idx, union_cnt,
+                    head_cnt, o, lse, ws, dev_status=None, stream=None):
+    """The whole decode step in one launch (see include/eta.h).  `ws` must be
+    zero-filled before its first use."""
+    _check("eta_decode_step", lib().eta_decode_step(
+        C.byref(dims), _p(q), _p(W), _p(bias), _p(tau_const), _p(K), _p(V), _p(lengths),
+        1 if update_tail else 0, _cent_format(cent), _p(cent), _p(rmax), _p(var), _p(vardim),
+        _p(cnt), BOUND[bound] if isinstance(bound, str) else int(bound), float(z), float(T),
+        float(scale), _p(tau), _p(head_mask), _p(union_idx), _p(union_cnt), _p(head_cnt),
+        _p(o), _p(lse), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _p(dev_status), _stream(stream)))
 
 
 def eta_decode_static_max_workspace() -> int:

@@ -9,6 +9,9 @@ runs one ETA decode step as four C-ABI calls on the current CUDA stream:
     eta_screen                         O(1) block screening, union compaction
     eta_decode                         gated split-KV attention + LSE combine
 
+With fused=True the same step is one call, eta_decode_step (one persistent
+kernel), writing the same outputs bit for bit.
+
 Every arithmetic step runs in libeta.so's kernels; this module only allocates
 and marshals arguments.
 """
@@ -26,7 +29,7 @@ class EtaDecoder:
     def __init__(self, K: torch.Tensor, V: torch.Tensor, lengths: torch.Tensor, Hq: int,
                  blk: int, *, bound: str = "exact", z: float = 3.0, T: float = 0.0,
                  scale: float = 0.0, prune: str = "skip", keep_bounds: bool = False,
-                 cent_format: str = "f32"):
+                 cent_format: str = "f32", fused: bool = False):
         if not K.is_cuda:
             raise ValueError("K/V must be CUDA tensors")
         if K.dtype != torch.bfloat16 or V.dtype != torch.bfloat16:
@@ -67,6 +70,12 @@ class EtaDecoder:
         self.ws_decode = torch.empty(max(L.eta_decode_workspace_size(self.dims), 256),
                                      dtype=torch.uint8, device=dev)
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
+        self.fused = bool(fused)
+        if self.fused and prune != "skip":
+            raise ValueError("the fused step offers SKIP pruning only")
+        # the fused step's workspace holds self-resetting counters: zero it once
+        self.ws_step = (torch.zeros(max(L.eta_decode_step_workspace_size(self.dims), 256),
+                                    dtype=torch.uint8, device=dev) if self.fused else None)
 
     # -- metadata -------------------------------------------------------------
     def build_meta(self, blk_begin: int = 0, blk_end: int = -1, stream=None):
@@ -102,8 +111,20 @@ class EtaDecoder:
                            self.lse, self.ws_decode, self.dev_status, stream)
         return self.o, self.lse
 
+    def step_fused(self, q, W=None, bias=None, tau_const=None, stream=None,
+                   append: bool = True):
+        """The same step as one eta_decode_step launch."""
+        L.eta_decode_step(self.dims, q, W, bias, tau_const, self.K, self.V, self.lengths,
+                          append, self.cent, self.rmax, self.var, self.vardim, self.cnt,
+                          self.bound, self.z, self.T, self.scale, self.tau, self.head_mask,
+                          self.union_idx, self.union_cnt, self.head_cnt, self.o, self.lse,
+                          self.ws_step, self.dev_status, stream)
+        return self.o, self.lse
+
     def step(self, q, W=None, bias=None, tau_const=None, stream=None, append: bool = True):
         """One decode step: tail-block metadata, tau, screening, gated decode."""
+        if self.fused:
+            return self.step_fused(q, W, bias, tau_const, stream, append)
         if append:
             self.append_update(stream)
         self.predict_tau(q, W, bias, tau_const, stream)
@@ -124,11 +145,15 @@ class EtaDecoder:
             torch.cuda.synchronize()
             g_pre = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g_pre, stream=stream):
-                self.append_update()
-                self.predict_tau(q, W, bias, tau_const)
-                self.screen(q)
-                if not split:
-                    self.decode(q)
+                if self.fused:
+                    self.step_fused(q, W, bias, tau_const)
+                    split = False
+                else:
+                    self.append_update()
+                    self.predict_tau(q, W, bias, tau_const)
+                    self.screen(q)
+                    if not split:
+                        self.decode(q)
             g_dec = None
             if split:
                 g_dec = torch.cuda.CUDAGraph()

@@ -23,14 +23,15 @@
 
 #include <atomic>
 
+#include "combine_dev.cuh"
 #include "decode_tc.cuh"
 #include "eta_common.cuh"
 #include "eta_host.h"
+#include "tma_host.h"
 
 namespace eta {
 
 constexpr int kStageKeys = 64;   // keys per pipeline stage (a 64- or 128-key block = 1 or 2)
-constexpr int kMinChunk = 2;     // minimum admitted blocks per CTA share
 constexpr int kPlanThreads = 1024;
 constexpr int kStageEnd = 1;
 
@@ -407,31 +408,13 @@ plan_kernel(int R, int Hkv, int NB, int blk, int T_max, const int32_t* __restric
   }
 }
 
-struct CombineParams {
-  int Hq, Hkv, NB, blk, T_max, P, floor_mode;
-  const int32_t* row_off;
-  const int32_t* plan;
-  const int32_t* union_idx;
-  const int32_t* lengths;
-  const int32_t* cnt;
-  const float* vsum;
-  const float* part_o;
-  const float* part_ml;
-  float* o;
-  float* lse;
-};
-
-// One CTA per (row, KV head), thread = dim.  Three rounds of memory latency: the
-// row's slot range, then every (head, slot) (m, l) pair at once into shared memory,
-// then every (head, slot) partial o of this dim at once.
-constexpr int kCombineMaxPairs = 256;   // (head, slot) pairs staged in shared memory
-
+// One CTA per (row, KV head), thread = dim: merges the row's partial slots
+// (combine_merge), then in FLOOR mode adds the pruned blocks' keys with logit 0.
 template <int D, int G>
 __global__ void __launch_bounds__(D) combine_kernel(const CombineParams p) {
   ETA_PDL_ENTRY();
   extern __shared__ uint32_t adm[];     // FLOOR mode: admitted-block bitmap of the row
-  __shared__ float sm_m[kCombineMaxPairs], sm_w[kCombineMaxPairs];
-  __shared__ float sM[G], sL[G];
+  __shared__ CombineScratch<G> sc;
   __shared__ int s_nfloor;
   const int r = blockIdx.x, b = r / p.Hkv, g = r % p.Hkv;
   const int dd = threadIdx.x;
@@ -464,64 +447,10 @@ __global__ void __launch_bounds__(D) combine_kernel(const CombineParams p) {
   const int p0 = c > 0 ? off / chunk : 0;
   const int ns = c > 0 ? (off + c - 1) / chunk - p0 + 1 : 0;
   float O[G];
-#pragma unroll
-  for (int h = 0; h < G; ++h) O[h] = 0.f;
-  if (ns > 0) {
-    const int np = G * ns;                 // pair k = slot * G + h
-    if (np <= kCombineMaxPairs) {
-      for (int k = dd; k < np; k += D) {
-        const size_t sl = ((size_t)(p0 + k / G) + r) * G + (k % G);
-        sm_m[k] = p.part_ml[sl * 2];
-        sm_w[k] = p.part_ml[sl * 2 + 1];
-      }
-      __syncthreads();
-      if (dd < G) {
-        float M = -INFINITY;
-        for (int k = dd; k < np; k += G) M = fmaxf(M, sm_m[k]);
-        float L = 0.f;
-        for (int k = dd; k < np; k += G) {
-          const float w = (M == -INFINITY) ? 0.f : expf(sm_m[k] - M);
-          L = fmaf(sm_w[k], w, L);
-          sm_m[k] = w;                       // now the slot weight
-        }
-        sM[dd] = M;
-        sL[dd] = L;
-      }
-      __syncthreads();
-      for (int k = 0; k < np; ++k) {
-        const size_t sl = ((size_t)(p0 + k / G) + r) * G + (k % G);
-        const float v = p.part_o[sl * D + dd];
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-          if (k % G == h) O[h] = fmaf(v, sm_m[k], O[h]);
-      }
-    } else {
-      // very long rows spread over many CTAs: plain two-pass merge per head
-      if (dd < G) { sM[dd] = -INFINITY; sL[dd] = 0.f; }
-      __syncthreads();
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float M = -INFINITY;
-        for (int k = 0; k < ns; ++k)
-          M = fmaxf(M, p.part_ml[(((size_t)(p0 + k) + r) * G + h) * 2]);
-        float L = 0.f;
-        for (int k = 0; k < ns; ++k) {
-          const size_t sl = ((size_t)(p0 + k) + r) * G + h;
-          const float w = (M == -INFINITY) ? 0.f : expf(p.part_ml[sl * 2] - M);
-          L = fmaf(p.part_ml[sl * 2 + 1], w, L);
-          O[h] = fmaf(p.part_o[sl * D + dd], w, O[h]);
-        }
-        if (dd == 0) { sM[h] = M; sL[h] = L; }
-      }
-      __syncthreads();
-    }
-  } else {
-    if (dd < G) { sM[dd] = -INFINITY; sL[dd] = 0.f; }
-    __syncthreads();
-  }
+  combine_merge<D, G, false>(p.part_ml, p.part_o, r, p0, ns, dd, sc, O, [] { __syncthreads(); });
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    float M = sM[h], L = sL[h], Oh = O[h];
+    float M = sc.M[h], L = sc.L[h], Oh = O[h];
     if (nfloor > 0) {
       const float Mf = fmaxf(M, 0.f);
       const float a = (M == -INFINITY) ? 0.f : expf(M - Mf);
@@ -530,14 +459,7 @@ __global__ void __launch_bounds__(D) combine_kernel(const CombineParams p) {
       L = L * a + (float)nfloor * e0;
       M = Mf;
     }
-    const size_t oh = (size_t)b * p.Hq + (size_t)g * G + h;
-    if (L > 0.f) {
-      p.o[oh * D + dd] = Oh / L;
-      if (dd == 0) p.lse[oh] = M + logf(L);
-    } else {
-      p.o[oh * D + dd] = 0.f;
-      if (dd == 0) p.lse[oh] = -INFINITY;
-    }
+    combine_store<D>(p.o, p.lse, (size_t)b * p.Hq + (size_t)g * G + h, dd, M, L, Oh);
   }
 }
 
@@ -615,35 +537,6 @@ inline bool use_tc(const eta_dims_t* d) {
   // AUTO and TCGEN05: the tensor-core engine wherever it applies (measured ~1.6x the
   // FMA engine's bandwidth on the 128K / B = 64 workload)
   return d->d == 128 && fits;
-}
-
-using EncodeTiledFn = PFN_cuTensorMapEncodeTiled_v12000;
-
-inline EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// 2-D view [rows, 128] of a bf16 tensor, box 64 columns x box_rows rows, 128-byte swizzle.
-inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_tiled();
-  if (!fn) return false;
-  cuuint64_t gdim[2] = {128, rows};
-  cuuint64_t gstride[1] = {128 * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
 }
 
 template <int G, bool DENSE>

@@ -31,6 +31,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "combine_dev.cuh"
 #include "eta_common.cuh"
 
 namespace eta {
@@ -73,6 +74,31 @@ struct TcMisc {
   int abort_flag;
 };
 constexpr int SMEM_BYTES = SM_MISC + (int)sizeof(TcMisc) + 1024;   // + alignment slack
+
+// The fused decode step's own shared state, after the decode's barriers: the
+// screening ring's barriers and item records, and the merge scratch.
+constexpr int kFuseStages = 6;
+struct FuseItem {
+  int r, grp, nvalid, flags;
+  float ts[8];
+};
+struct FuseSmem {
+  uint64_t bfull[kFuseStages], bempty[kFuseStages];
+  FuseItem item[kFuseStages];
+  CombineScratch<8> cs;   // sized for the largest group
+  int last;
+  int abort;
+  int gen0;               // grid-barrier generation at launch: names this launch's flags
+  int plan[2];            // this CTA's copy of the share plan: total, share length
+  int cta_row;            // the first (row, KV head) of this CTA's share
+  int wsum[NT / 32];
+};
+constexpr int SM_FUSE = (SM_MISC + (int)sizeof(TcMisc) + 15) / 16 * 16;
+// the fused step keeps the prefix sum of admitted blocks over rows in shared memory
+constexpr int kFusedMaxRows = 2048;
+constexpr int SM_ROWOFF = (SM_FUSE + (int)sizeof(FuseSmem) + 15) / 16 * 16;
+constexpr int FUSED_SMEM_BYTES = SM_ROWOFF + (kFusedMaxRows + 1) * 4 + 1024;
+static_assert(FUSED_SMEM_BYTES <= 227 * 1024, "fused step shared memory");
 
 // Instruction descriptor, kind::f16: D fp32, A/B bf16, M = 128, N = 16.
 constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) |
@@ -146,15 +172,29 @@ struct TcParams {
   int32_t* status;
 };
 
-template <int G, bool DENSE>
-__global__ void __launch_bounds__(NT, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                 const __grid_constant__ CUtensorMap tmQ, const TcParams p) {
-  ETA_PDL_ENTRY();
+// In-kernel merge of the fused step: the CTA that writes the last partial slot of
+// a (row, KV head) pair (counted in pair_cnt, which it resets) merges the pair.
+struct FuseCtx {
+  int32_t* pair_cnt;
+  float* o;
+  float* lse;
+  const int32_t* ready;   // ready[row] == token once the row's union list is written
+  int token;
+};
+
+// The decode of one CTA share.  `smem` is the CTA's dynamic shared memory aligned
+// to 1024 bytes.  Every thread of the CTA calls it.
+// In the fused step the union list and tau were written by other CTAs of the same
+// grid before a grid barrier; plain (L1-cached) loads still see them, because no
+// SM reads those lines before the barrier (the screening reads tau with L2-only
+// loads).  The plan, the prefix sums and the CTA's first row are its own copy in
+// shared memory (p.cta_row points at that one entry).  The partial slots other
+// CTAs write during the decode are read with L2-only loads.
+template <int G, bool DENSE, bool FUSED>
+ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                            const CUtensorMap* tmQ, const TcParams& p, const FuseCtx& fx) {
   static_assert(G >= 1 && G <= 8, "G");
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  static_assert(!(FUSED && DENSE), "the fused step is sparse");
   TcMisc* ms = reinterpret_cast<TcMisc*>(smem + SM_MISC);
   volatile int* abort_flag = &ms->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -205,7 +245,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   if (warp == NWARP_SM) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      int r = p.cta_row[blockIdx.x];
+      int r = FUSED ? p.cta_row[0] : p.cta_row[blockIdx.x];
       int roff = p.row_off[r], rend = p.row_off[r + 1];
       int it = 0;
       bool ok = true;
@@ -223,18 +263,37 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           mbar_arrive_expect_tx(&ms->full[s], (uint32_t)(nsub * 4 * SUB_HALF + 2 * QHALF));
           const int b = row / p.Hkv, g = row % p.Hkv;
           const int qrow = b * p.Hq + g * G;
-          tma_load_2d(st + OFF_Q0, &tmQ, 0, qrow, &ms->full[s]);
-          tma_load_2d(st + OFF_Q1, &tmQ, 64, qrow, &ms->full[s]);
+          tma_load_2d(st + OFF_Q0, tmQ, 0, qrow, &ms->full[s]);
+          tma_load_2d(st + OFF_Q1, tmQ, 64, qrow, &ms->full[s]);
           for (int u = 0; u < nsub; ++u) {
             const int y = row * p.T_max + (u == 0 ? t0a : t0b);
-            tma_load_2d(st + OFF_K0 + u * SUB_HALF, &tmK, 0, y, &ms->full[s]);
-            tma_load_2d(st + OFF_K1 + u * SUB_HALF, &tmK, 64, y, &ms->full[s]);
-            tma_load_2d(st + OFF_V0 + u * SUB_HALF, &tmV, 0, y, &ms->full[s]);
-            tma_load_2d(st + OFF_V1 + u * SUB_HALF, &tmV, 64, y, &ms->full[s]);
+            tma_load_2d(st + OFF_K0 + u * SUB_HALF, tmK, 0, y, &ms->full[s]);
+            tma_load_2d(st + OFF_K1 + u * SUB_HALF, tmK, 64, y, &ms->full[s]);
+            tma_load_2d(st + OFF_V0 + u * SUB_HALF, tmV, 0, y, &ms->full[s]);
+            tma_load_2d(st + OFF_V1 + u * SUB_HALF, tmV, 64, y, &ms->full[s]);
           }
         }
         ++it;
         return true;
+      };
+      // fused step: a row's union list is read once its compaction flag is set
+      int ready_row = -1;
+      bool rows_ok = true;
+      auto row_ready = [&](int rr) -> bool {
+        if constexpr (FUSED) {
+          if (rr == ready_row) return true;
+          for (uint32_t w = 0; w < kWaitLimit; ++w) {
+            if (ld_acquire_gpu(fx.ready + rr) == fx.token) {
+              ready_row = rr;
+              return true;
+            }
+            if (*abort_flag) return false;
+            __nanosleep(32);
+          }
+          return false;
+        } else {
+          return true;
+        }
       };
       // The block index of position pos+1 is loaded before the stages of position pos
       // are emitted, so its L2 latency overlaps the wait for a free stage.
@@ -244,11 +303,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
           ro = re;
           re = p.row_off[rr + 1];
         }
-        return DENSE ? pos - ro : p.union_idx[(size_t)rr * p.NB + (pos - ro)];
+        if (DENSE) return pos - ro;
+        if (!row_ready(rr)) {
+          rows_ok = false;
+          return 0;
+        }
+        return p.union_idx[(size_t)rr * p.NB + (pos - ro)];
       };
       int nr = r, nroff = roff, nrend = rend;
       int j_next = a < e ? fetch(a, nr, nroff, nrend) : 0;
       for (int pos = a; pos < e && ok; ++pos) {
+        if (!rows_ok) {
+          ok = false;
+          break;
+        }
         const int j = j_next;
         r = nr; roff = nroff; rend = nrend;
         if (pos + 1 < e) j_next = fetch(pos + 1, nr, nroff, nrend);
@@ -372,19 +440,69 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         if (lane == 0) ms->lsum[warp][h] = v;
       }
       named_bar_sync(1, NWARP_SM * 32);
-      const size_t slot = (size_t)blockIdx.x + row;
+      int p0 = 0, ns = 0;
+      if constexpr (FUSED) {
+        const int off = p.row_off[row], c = p.row_off[row + 1] - off;
+        const int chunk = p.plan[1];
+        p0 = off / chunk;
+        ns = (off + c - 1) / chunk - p0 + 1;
+      }
+      if (FUSED && ns == 1) {
+        // the whole pair lies in this share: its partial is the merged result (the
+        // one-slot merge written out: weight e^(m - m) = 1, or 0 for an empty softmax)
+        const int b = row / p.Hkv, g = row % p.Hkv;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        p.part_o[(slot * G + h) * D + t] = o_acc[h];
-        if (t == 0) {
+        for (int h = 0; h < G; ++h) {
           float L = 0.f;
 #pragma unroll
           for (int w = 0; w < NWARP_SM; ++w) L += ms->lsum[w][h];
-          p.part_ml[(slot * G + h) * 2] = m_run[h];
-          p.part_ml[(slot * G + h) * 2 + 1] = L;
+          const float wt = m_run[h] == -INFINITY ? 0.f : 1.f;
+          combine_store<D>(fx.o, fx.lse, (size_t)b * p.Hq + (size_t)g * G + h, t, m_run[h],
+                           fmaf(L, wt, 0.f), fmaf(o_acc[h], wt, 0.f));
+        }
+        named_bar_sync(1, NWARP_SM * 32);
+      } else {
+        const size_t slot = (size_t)blockIdx.x + row;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          p.part_o[(slot * G + h) * D + t] = o_acc[h];
+          if (t == 0) {
+            float L = 0.f;
+#pragma unroll
+            for (int w = 0; w < NWARP_SM; ++w) L += ms->lsum[w][h];
+            p.part_ml[(slot * G + h) * 2] = m_run[h];
+            p.part_ml[(slot * G + h) * 2 + 1] = L;
+          }
+        }
+        named_bar_sync(1, NWARP_SM * 32);
+        if constexpr (FUSED) {
+          // this slot of the pair is written: count it; the CTA with the pair's last
+          // slot merges all of them (threadFenceReduction pattern)
+          FuseSmem* fs = reinterpret_cast<FuseSmem*>(smem + SM_FUSE);
+          __threadfence();
+          named_bar_sync(1, NWARP_SM * 32);
+          if (t == 0) {
+            const int old = atomicAdd(fx.pair_cnt + row, 1);
+            const int last = old == ns - 1;
+            if (last) fx.pair_cnt[row] = 0;
+            fs->last = last;
+          }
+          named_bar_sync(1, NWARP_SM * 32);
+          if (fs->last) {
+            __threadfence();
+            CombineScratch<G>& cs = *reinterpret_cast<CombineScratch<G>*>(&fs->cs);
+            float O[G];
+            combine_merge<D, G, true>(p.part_ml, p.part_o, row, p0, ns, t, cs, O,
+                                      [] { named_bar_sync(1, NWARP_SM * 32); });
+            const int b = row / p.Hkv, g = row % p.Hkv;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+              combine_store<D>(fx.o, fx.lse, (size_t)b * p.Hq + (size_t)g * G + h, t, cs.M[h],
+                               cs.L[h], O[h]);
+          }
+          named_bar_sync(1, NWARP_SM * 32);
         }
       }
-      named_bar_sync(1, NWARP_SM * 32);
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         m_run[h] = -INFINITY; l_part[h] = 0.f; o_acc[h] = 0.f;
@@ -497,6 +615,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
   }
+}
+
+template <int G, bool DENSE>
+__global__ void __launch_bounds__(NT, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmQ, const TcParams p) {
+  ETA_PDL_ENTRY();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  decode_tc_body<G, DENSE, false>(smem, &tmK, &tmV, &tmQ, p, FuseCtx{});
 }
 
 }  // namespace tc

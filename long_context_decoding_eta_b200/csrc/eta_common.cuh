@@ -97,6 +97,17 @@ ETA_DEV void bulk_g2s(void* smem_dst, const void* gmem_src, uint32_t bytes, uint
       : "memory");
 }
 
+// gpu-scope acquire load / release store of an int32 flag in global memory.
+ETA_DEV int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+ETA_DEV void st_release_gpu(int32_t* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 ETA_DEV void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

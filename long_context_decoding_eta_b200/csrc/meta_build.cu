@@ -10,42 +10,9 @@
 
 #include "eta_common.cuh"
 #include "eta_host.h"
+#include "meta_dev.cuh"
 
 namespace eta {
-
-// 1 + 2^-20: covers the relative rounding error of the fp32 distance
-// computation below (<= ~6 ulp on the sqrt), so rmax never under-states the
-// true maximum distance to the stored fp32 centroid.
-constexpr float kRadiusInflate = 1.00000095367431640625f;
-constexpr int kMetaWarps = 8;
-
-template <int DPL>
-ETA_DEV void load_row(const eta_bf16_t* p, float (&x)[DPL]) {
-  if constexpr (DPL == 4) {
-    uint2 w = *reinterpret_cast<const uint2*>(p);
-    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
-  } else {
-    uint32_t w = *reinterpret_cast<const uint32_t*>(p);
-    x[0] = bf16_lo(w); x[1] = bf16_hi(w);
-  }
-}
-
-// Centroid storage: CF = 0 fp32, CF = 1 bf16.  With bf16 the key sum is accumulated
-// in fp64 (exact for up to 128 bf16 keys of ordinary range), divided in fp64 and
-// rounded once to bf16 (nearest even), so the stored centroid is the correctly
-// rounded mean; rmax and var are then measured against that stored centroid and the
-// bound stays exact for what the screen reads.
-ETA_DEV float bf16_round_from_double(double m) {
-  return __bfloat162float(__double2bfloat16(m));
-}
-
-template <int CF>
-ETA_DEV void store_centroid(void* cent, size_t idx, float c) {
-  if constexpr (CF == 1)
-    reinterpret_cast<uint16_t*>(cent)[idx] = __bfloat16_as_ushort(__float2bfloat16_rn(c));
-  else
-    reinterpret_cast<float*>(cent)[idx] = c;
-}
 
 template <int D, int CF>
 __global__ void __launch_bounds__(kMetaWarps * 32)
@@ -175,12 +142,9 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
   }
 }
 
-// Tail-block refresh (one block per (row, KV head) after a token is appended):
-// the same arithmetic as meta_build_kernel (sequential fp32 sum over the keys in
-// token order, one division, butterfly distance sums), but the block's keys are
-// split over the 8 warps of a CTA so the latency chain is blk/8 keys instead of blk.
-// The chunk sums are combined in warp order, the same order meta_build_kernel
-// uses, so both kernels give bit-identical metadata for the same block.
+// Tail-block refresh: one CTA of kMetaWarps warps per (row, KV head), so the
+// latency chain is blk / kMetaWarps keys instead of blk (arithmetic in
+// meta_tail_block).
 template <int D, int CF>
 __global__ void __launch_bounds__(kMetaWarps * 32)
 meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restrict__ K,
@@ -188,123 +152,10 @@ meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restri
                  void* __restrict__ cent, float* __restrict__ rmax, float* __restrict__ var,
                  int32_t* __restrict__ cnt, float* __restrict__ vsum, float* __restrict__ vardim) {
   ETA_PDL_ENTRY();
-  constexpr int DPL = D / 32;
-  __shared__ float part[kMetaWarps][D];
-  __shared__ float red_max[kMetaWarps], red_sum[kMetaWarps];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.x, b = r / Hkv;
-  const int len = min(max(lengths[b], 0), T_max);
-  if (len == 0) return;                      // uniform over the CTA
-  const int j = (len - 1) / blk;
-  const int n = min(len - j * blk, blk);
-  const int per = (blk + kMetaWarps - 1) / kMetaWarps;
-  const int t_lo = min(warp * per, n), t_hi = min(t_lo + per, n);
-  const size_t rowj = (size_t)r * NB + j;
-  const eta_bf16_t* kb = K + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
-
-  using Acc = typename std::conditional<CF == 1, double, float>::type;
-  __shared__ Acc cpart[kMetaWarps][D];
-  float c[DPL];
-  Acc pc[DPL];
-#pragma unroll
-  for (int i = 0; i < DPL; ++i) pc[i] = 0;
-  for (int t = t_lo; t < t_hi; ++t) {
-    float x[DPL];
-    load_row<DPL>(kb + (size_t)t * D, x);
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) pc[i] += (Acc)x[i];
-  }
-#pragma unroll
-  for (int i = 0; i < DPL; ++i) cpart[warp][lane * DPL + i] = pc[i];
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < DPL; ++i) {
-    Acc sum = 0;
-#pragma unroll
-    for (int w = 0; w < kMetaWarps; ++w) sum += cpart[w][lane * DPL + i];
-    if constexpr (CF == 1) c[i] = bf16_round_from_double(sum / (double)n);
-    else c[i] = sum / (float)n;
-  }
-  float r2max = 0.f, s2 = 0.f;
-  float pv[DPL];
-#pragma unroll
-  for (int i = 0; i < DPL; ++i) pv[i] = 0.f;
-  for (int t = t_lo; t < t_hi; ++t) {
-    float x[DPL];
-    load_row<DPL>(kb + (size_t)t * D, x);
-    float pd = 0.f;
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) {
-      const float dv = x[i] - c[i];
-      pd = fmaf(dv, dv, pd);
-      pv[i] = fmaf(dv, dv, pv[i]);
-    }
-    pd = warp_sum(pd);
-    r2max = fmaxf(r2max, pd);
-    s2 += pd;
-  }
-  if (vardim) {
-    __shared__ float vpart[kMetaWarps][D];
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) vpart[warp][lane * DPL + i] = pv[i];
-    __syncthreads();
-    if (warp == 0) {
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) {
-        float sum = 0.f;
-#pragma unroll
-        for (int w = 0; w < kMetaWarps; ++w) sum += vpart[w][lane * DPL + i];
-        vardim[((size_t)r * D + lane * DPL + i) * NB + j] = sum / (float)n;
-      }
-    }
-  }
-  if (lane == 0) {
-    red_max[warp] = r2max;
-    red_sum[warp] = s2;
-  }
-  if (warp == 0) {
-#pragma unroll
-    for (int i = 0; i < DPL; ++i)
-      store_centroid<CF>(cent, ((size_t)r * D + lane * DPL + i) * NB + j, c[i]);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float m = 0.f, sum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kMetaWarps; ++w) {
-      m = fmaxf(m, red_max[w]);
-      sum += red_sum[w];
-    }
-    rmax[rowj] = __fmul_ru(__fsqrt_ru(m), kRadiusInflate);
-    var[rowj] = sum / (float)n;
-    cnt[rowj] = n;
-  }
-  if (vsum) {
-    __syncthreads();
-    const eta_bf16_t* vb = V + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
-    float a[DPL];
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) a[i] = 0.f;
-    for (int t = t_lo; t < t_hi; ++t) {
-      float x[DPL];
-      load_row<DPL>(vb + (size_t)t * D, x);
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) a[i] += x[i];
-    }
-#pragma unroll
-    for (int i = 0; i < DPL; ++i) part[warp][lane * DPL + i] = a[i];
-    __syncthreads();
-    if (warp == 0) {
-      float* vr = vsum + rowj * D + lane * DPL;
-#pragma unroll
-      for (int i = 0; i < DPL; ++i) {
-        float s = 0.f;
-#pragma unroll
-        for (int w = 0; w < kMetaWarps; ++w) s += part[w][lane * DPL + i];
-        vr[i] = s;
-      }
-    }
-  }
+  __shared__ TailScratch<D, CF> sc;
+  meta_tail_block<D, CF, kMetaWarps>(blockIdx.x, Hkv, T_max, blk, NB, K, V, lengths, cent, rmax,
+                                     var, cnt, vsum, vardim, sc, threadIdx.x >> 5,
+                                     [] { __syncthreads(); });
 }
 
 template <int D, int CF>

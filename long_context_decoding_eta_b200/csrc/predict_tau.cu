@@ -8,6 +8,7 @@
 // fixed-order block reduction, so results are deterministic.
 #include "eta_common.cuh"
 #include "eta_host.h"
+#include "tau_dev.cuh"
 
 namespace eta {
 
@@ -22,37 +23,10 @@ predict_tau_group_kernel(int Hq, int D, const eta_bf16_t* __restrict__ q,
                          const float* __restrict__ W, const float* __restrict__ bias,
                          float* __restrict__ tau, int32_t* status) {
   ETA_PDL_ENTRY();
-  __shared__ float red[kTauThreads / 32][G];
-  const int b = blockIdx.x, g = blockIdx.y;
-  const int n = Hq * D;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const eta_bf16_t* qb = q + (size_t)b * n;
-  const int h0 = g * G;
-  float acc[G];
-#pragma unroll
-  for (int k = 0; k < G; ++k) acc[k] = 0.f;
-  bool bad = false;
-#pragma unroll 4
-  for (int i = threadIdx.x; i < n; i += kTauThreads) {
-    const float x = bf16_to_f(qb[i]);
-    bad |= !isfinite(x);
-    const float* wr = W + (size_t)i * Hq + h0;
-#pragma unroll
-    for (int k = 0; k < G; ++k) acc[k] = fmaf(x, __ldg(wr + k), acc[k]);
-  }
-#pragma unroll
-  for (int k = 0; k < G; ++k) {
-    const float v = warp_sum(acc[k]);
-    if (lane == 0) red[warp][k] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < G) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < kTauThreads / 32; ++w) s += red[w][threadIdx.x];
-    const int h = h0 + threadIdx.x;
-    tau[(size_t)b * Hq + h] = s + (bias ? bias[h] : 0.f);
-  }
+  __shared__ float red[kTauVirtWarps][G];
+  const int g = blockIdx.y;
+  const bool bad = tau_group<G, kTauThreads / 32>(Hq, D, blockIdx.x, g * G, q, W, bias, red, tau,
+                                                  threadIdx.x >> 5, [] { __syncthreads(); });
   if (bad && g == 0) set_status(status, ETA_DEVSTAT_NONFINITE_Q);
 }
 

@@ -23,6 +23,7 @@
 #include "decode_tc.cuh"
 #include "eta_common.cuh"
 #include "eta_host.h"
+#include "tma_host.h"
 
 namespace eta {
 namespace pf {
@@ -388,34 +389,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
 }  // namespace pf
 
-using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
-
-static EncodeFn prefill_encode() {
-  static EncodeFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(ptr);
-  }
-  return fn;
-}
-
-static bool prefill_map(CUtensorMap* m, const void* base, uint64_t rows) {
-  EncodeFn fn = prefill_encode();
-  if (!fn) return false;
-  cuuint64_t gdim[2] = {128, rows};
-  cuuint64_t gstride[1] = {256};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
 template <int G>
 static eta_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk,
                                    const CUtensorMap& mv, const pf::PrefillParams& prm,
@@ -446,8 +419,8 @@ extern "C" eta_status_t eta_prefill(const eta_dims_t* dims, const eta_bf16_t* Q,
   const int64_t ctas = (int64_t)dims->B * dims->Hq * ntiles;
   if (ctas > 0x7fffffff) return ETA_ERR_UNSUPPORTED;
   CUtensorMap mq, mk, mv;
-  if (!prefill_map(&mq, Q, q_rows) || !prefill_map(&mk, K, kv_rows) ||
-      !prefill_map(&mv, V, kv_rows))
+  if (!make_map(&mq, Q, q_rows, pf::TILE) || !make_map(&mk, K, kv_rows, pf::TILE) ||
+      !make_map(&mv, V, kv_rows, pf::TILE))
     return ETA_ERR_CUDA;
   pf::PrefillParams prm;
   prm.Hq = dims->Hq; prm.Hkv = dims->Hkv; prm.T_max = dims->T_max; prm.ntiles = ntiles;

@@ -15,6 +15,7 @@
 
 #include "eta_common.cuh"
 #include "eta_host.h"
+#include "screen_dev.cuh"
 
 namespace eta {
 
@@ -97,14 +98,7 @@ screen_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict__ q,
   if (lane == 0) union_words[(size_t)r * NW + w] = uni;
 }
 
-// Vector form: lane l of a warp owns VW = 4 consecutive blocks, so each of the d
-// loads of a lane is one 16-byte (fp32 centroids) or 8-byte (bf16) load and a warp
-// covers a group of 128 blocks.
-// The lanes' VW-bit admit chunks are assembled into 32-bit words with an OR
-// butterfly over the 32 / VW lanes of each word.  Needs NB % VW == 0 and 16-byte
-// aligned metadata.
 constexpr int kScreenVecWarps = 4;
-constexpr int kLoadBatch = 16;   // independent 16-byte loads in flight per lane
 
 template <int D, int G, int CF, bool VD>
 __global__ void __launch_bounds__(kScreenVecWarps * 32)
@@ -116,9 +110,6 @@ screen_vec_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict_
                   uint32_t* __restrict__ head_mask, uint32_t* __restrict__ union_words,
                   float* __restrict__ bounds_out) {
   ETA_PDL_ENTRY();
-  constexpr int VW = 4;                         // blocks per lane
-  constexpr int GB = 32 * VW;                   // blocks per warp group
-  constexpr int LPW = 32 / VW;                  // lanes per 32-bit word
   __shared__ __align__(16) float qs[D * G];
   __shared__ float qn[G], ts[G];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,120 +122,19 @@ screen_vec_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict_
   }
   __syncthreads();
   for (int h = warp; h < G; h += kScreenVecWarps) {
-    float s = 0.f;
-    for (int k = lane; k < D; k += 32) s = fmaf(qs[k * G + h], qs[k * G + h], s);
-    s = warp_sum(s);
+    const float s = query_norm<D, G>(qs, h);
     if (lane == 0) {
-      qn[h] = sqrtf(s);
+      qn[h] = s;
       ts[h] = tau[qhead0 + h];
     }
   }
   __syncthreads();
 
   const int grp = blockIdx.x * kScreenVecWarps + warp;
-  if (grp * GB >= NB) return;
-  const int j0 = grp * GB + lane * VW;
-  const bool vj = j0 < NB;                      // NB % VW == 0: all VW valid or none
-  // one load per dimension: 4 centroids = 16 bytes (fp32) or 8 bytes (bf16)
-  using LdT = typename std::conditional<CF == 1, uint2, uint4>::type;
-  const size_t rowv = (size_t)NB / 4;           // LdT units per dimension
-  const LdT* cp = reinterpret_cast<const LdT*>(
-      reinterpret_cast<const unsigned char*>(cent) + ((size_t)r * D * NB + (vj ? j0 : 0)) *
-                                                        (CF == 1 ? 2 : 4));
-  float acc[VW][G], acc2[VW][VD ? G : 1];
-#pragma unroll
-  for (int k = 0; k < VW; ++k) {
-#pragma unroll
-    for (int h = 0; h < G; ++h) acc[k][h] = 0.f;
-#pragma unroll
-    for (int h = 0; h < (VD ? G : 1); ++h) acc2[k][h] = 0.f;
-  }
-  const float4* vdp = VD ? reinterpret_cast<const float4*>(
-                               vardim + (size_t)r * D * NB + (vj ? j0 : 0))
-                         : nullptr;
-#pragma unroll 1
-  for (int d0 = 0; d0 < D; d0 += kLoadBatch) {
-    LdT cb[kLoadBatch];
-#pragma unroll
-    for (int u = 0; u < kLoadBatch; ++u)
-      cb[u] = vj ? __ldg(cp + (size_t)(d0 + u) * rowv) : LdT{};
-#pragma unroll
-    for (int u = 0; u < kLoadBatch; ++u) {
-      float cv[VW];
-      if constexpr (CF == 1) {
-        cv[0] = bf16_lo(cb[u].x); cv[1] = bf16_hi(cb[u].x); cv[2] = bf16_lo(cb[u].y);
-        cv[3] = bf16_hi(cb[u].y);
-      } else {
-        cv[0] = __uint_as_float(cb[u].x); cv[1] = __uint_as_float(cb[u].y);
-        cv[2] = __uint_as_float(cb[u].z); cv[3] = __uint_as_float(cb[u].w);
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float qv = qs[(d0 + u) * G + h];
-#pragma unroll
-        for (int k = 0; k < VW; ++k) acc[k][h] = fmaf(qv, cv[k], acc[k][h]);
-      }
-      if constexpr (VD) {
-        const float4 vv = vj ? __ldg(vdp + (size_t)(d0 + u) * (NB / 4))
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float vk[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float q2 = qs[(d0 + u) * G + h] * qs[(d0 + u) * G + h];
-#pragma unroll
-          for (int k = 0; k < VW; ++k) acc2[k][h] = fmaf(q2, vk[k], acc2[k][h]);
-        }
-      }
-    }
-  }
-  const size_t rj = (size_t)r * NB + j0;
-  float rad[VW];
-  int n[VW];
-#pragma unroll
-  for (int k = 0; k < VW; ++k) { rad[k] = 0.f; n[k] = 0; }
-  if (vj) {
-#pragma unroll
-    for (int v = 0; v < VW / 4; ++v) {
-      const float4 rr = __ldg(reinterpret_cast<const float4*>(rmax + rj) + v);
-      const int4 cc = __ldg(reinterpret_cast<const int4*>(cnt + rj) + v);
-      rad[4 * v] = rr.x; rad[4 * v + 1] = rr.y; rad[4 * v + 2] = rr.z; rad[4 * v + 3] = rr.w;
-      n[4 * v] = cc.x; n[4 * v + 1] = cc.y; n[4 * v + 2] = cc.z; n[4 * v + 3] = cc.w;
-      if (bound == ETA_BOUND_PROB) {
-        const float4 vv = __ldg(reinterpret_cast<const float4*>(var + rj) + v);
-        rad[4 * v] = fminf(rad[4 * v], z * sqrtf(vv.x / (float)D));
-        rad[4 * v + 1] = fminf(rad[4 * v + 1], z * sqrtf(vv.y / (float)D));
-        rad[4 * v + 2] = fminf(rad[4 * v + 2], z * sqrtf(vv.z / (float)D));
-        rad[4 * v + 3] = fminf(rad[4 * v + 3], z * sqrtf(vv.w / (float)D));
-      }
-    }
-  }
-  uint32_t uni = 0;
-  const int wsel = grp * VW + lane / LPW;        // word index of this lane's chunk
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    uint32_t bits = 0;
-    float ubv[VW];
-#pragma unroll
-    for (int k = 0; k < VW; ++k) {
-      if constexpr (VD)
-        ubv[k] = scale * (acc[k][h] + fminf(qn[h] * rad[k], z * sqrtf(acc2[k][h])));
-      else
-        ubv[k] = scale * fmaf(qn[h], rad[k], acc[k][h]);
-      if (vj && n[k] > 0 && ubv[k] >= ts[h]) bits |= 1u << k;
-    }
-    if (bounds_out && vj) {
-#pragma unroll
-      for (int v = 0; v < VW / 4; ++v)
-        reinterpret_cast<float4*>(bounds_out + (qhead0 + h) * NB + j0)[v] =
-            make_float4(ubv[4 * v], ubv[4 * v + 1], ubv[4 * v + 2], ubv[4 * v + 3]);
-    }
-    uint32_t word = bits << (VW * (lane % LPW));
-#pragma unroll
-    for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
-    if (lane % LPW == 0 && wsel < NW) head_mask[(qhead0 + h) * NW + wsel] = word;
-    uni |= word;
-  }
-  if (lane % LPW == 0 && wsel < NW) union_words[(size_t)r * NW + wsel] = uni;
+  if (grp * kScreenGroupBlocks >= NB) return;
+  screen_group<D, G, CF, VD, kScreenLoadBatch, false>(
+      NB, NW, grp, r, qhead0, qs, qn, ts, cent, rmax, var, vardim, cnt, bound, z, scale, NB,
+      head_mask, union_words, bounds_out);
 }
 
 __global__ void __launch_bounds__(kCompactThreads)

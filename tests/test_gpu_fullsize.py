@@ -132,3 +132,46 @@ def test_calibrated_256k_const_tau():
     torch.cuda.empty_cache()
     rep, dens = run_fullsize(w, rows=rows, tau_const=tau_const)
     print(rep, dens)
+
+
+def test_long_128k_fused_step_equals_separate_calls():
+    """The one-launch step at full size, in the launch configuration `bench.py --fused`
+    times: every output equals the separate calls' bit for bit; the sampled rows
+    against the oracle."""
+    w = synth.LONG128K
+    rows = [0, 63]
+    scale = 1.0 / math.sqrt(w.d)
+    g = synth.generate(w, "cuda")
+    bias = sampled_oracle_bias(w, g, rows, scale, "bf16")
+    bias_t = torch.full((w.Hq,), bias, device="cuda")
+    kw = dict(bound=w.bound, z=w.z, T=w.gate_T, cent_format="bf16")
+    sep = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, **kw)
+    fus = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, fused=True, **kw)
+    sep.build_meta()
+    fus.build_meta()
+    sep.step(g["q"], g["W"], bias_t)
+    fus.step(g["q"], g["W"], bias_t)
+    torch.cuda.synchronize()
+    sep.check_status()
+    fus.check_status()
+    for name in ("tau", "head_mask", "union_cnt", "head_cnt", "o", "lse", "cent", "rmax", "var",
+                 "cnt"):
+        assert torch.equal(getattr(sep, name), getattr(fus, name)), name
+    live = torch.arange(fus.NB, device="cuda") < fus.union_cnt[..., None]
+    assert torch.equal(sep.union_idx[live], fus.union_idx[live])
+    gpu = dict(tau=f64(fus.tau), head_mask=unpack_mask(fus.head_mask, fus.NB),
+               union_idx=fus.union_idx.cpu().numpy(), union_cnt=fus.union_cnt.cpu().numpy(),
+               head_cnt=fus.head_cnt.cpu().numpy(), o=f64(fus.o), lse=f64(fus.lse))
+    K64, V64, q64 = rows_f64(g["K"], rows), rows_f64(g["V"], rows), rows_f64(g["q"], rows)
+    L64 = g["lengths"][rows].cpu().numpy()
+    meta = O.cache_meta(K64, L64, w.blk, cent_format="bf16")
+    tau = O.predict_tau(q64, g["W"].double().cpu().numpy(), np.full(w.Hq, bias))
+    sc = O.screen(q64, tau, meta, scale, w.bound, w.z)
+    o, lse = O.decode(q64, tau, K64, V64, L64, sc["union_idx"], w.blk, scale, w.gate_T)
+    check_meta(gpu_meta(fus, rows), meta)
+    rep = compare_step(gpu, tau, sc, o, lse, q64, K64, V64, L64, w.blk, scale, w.gate_T, w.G,
+                       rows=rows)
+    print(rep)
+    del sep, fus, g
+    gc.collect()
+    torch.cuda.empty_cache()

@@ -5,16 +5,19 @@
 // (query, key) pair of a causal prefill, with beta = 1/T (T = 0: hard gate); the
 // inference-side counterpart of the paper's dense gated training forward.
 //
-// One CTA per (batch row, query head, 128-query tile), 192 threads:
-//   warp 4  TMA producer: the 128 x 128 query tile once, then 128-key K and V
+// One CTA per (batch row, query head, 128-query tile), 320 threads:
+//   warp 8  TMA producer: the 128 x 128 query tile once, then 128-key K and V
 //           tiles (two 64-dim boxes each, 128-byte swizzle) into a 2-stage ring
-//   warp 5  MMA issuer: S = Q K^T (M = 128 queries, N = 128 keys, K = d) into one of
+//   warp 9  MMA issuer: S = Q K^T (M = 128 queries, N = 128 keys, K = d) into one of
 //           two TMEM buffers, then O += P V (M = 128 queries, N = d, K = 128 keys,
 //           V read MN-major from its swizzled tile) into the TMEM accumulator
-//   warps 0-3 softmax, thread = query row = TMEM lane: causal mask, gate, running
-//           row max; O is rescaled in TMEM only when the row max grew by more than
-//           kRescale (FA-style conditional rescaling), P is written as bf16 into a
-//           swizzled shared tile (the A operand of P V).
+//   warps 0-7 softmax, two threads per query row (= TMEM lane): warps 0-3 take key
+//           columns 0-63 of the S tile, warps 4-7 columns 64-127, and the two halves
+//           of a row agree on the tile's row max through shared memory.  Causal mask,
+//           gate, running row max; O is rescaled in TMEM only when the row max grew by
+//           more than kRescale (FA-style conditional rescaling), each half rescaling its
+//           own 64 columns; P is written as bf16 into a swizzled shared tile (the A
+//           operand of P V), each half writing its own 64-key half.
 // TMEM: S 2 x 128 columns, O 128 columns (512 allocated).  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -45,7 +48,7 @@ constexpr int OFF_KV = 2 * HALF;                // stage s: K0 K1 V0 V1
 constexpr int KV_STAGE = 4 * HALF;              // 64 KB
 constexpr int OFF_P = OFF_KV + NKV * KV_STAGE;  // 2 buffers x 2 halves
 constexpr int OFF_MISC = OFF_P + 2 * 2 * HALF;
-constexpr int NWARP_SM = 4;
+constexpr int NWARP_SM = 8;                     // two warpgroups: key columns 0-63, 64-127
 constexpr int NT = (NWARP_SM + 2) * 32;
 constexpr int kTmemCols = 512;
 constexpr float kRescale = 8.0f;                // rescale O when the max grows by > 8 (e^8)
@@ -53,6 +56,7 @@ constexpr float kRescale = 8.0f;                // rescale O when the max grows 
 struct Misc {
   uint64_t q_full, kv_full[NKV], kv_empty[NKV];
   uint64_t s_full[2], s_free[2], p_full[2], o_done, o_final, fin;
+  float xch[2][TILE];      // per-half row maxima of a tile, then the final row sums
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -243,50 +247,67 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
   } else {
     // ------------------------------------------------------------------ softmax
-    const int row = threadIdx.x;                      // query row of the tile = TMEM lane
+    const int hh = warp >> 2;                         // key-column half of the tile
+    const int row = threadIdx.x & (TILE - 1);         // query row of the tile = TMEM lane
     const int tq = q0 + row;
-    const uint32_t lsel = (uint32_t)(warp * 32) << 16;
+    const uint32_t lsel = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t cb = (uint32_t)hh * 64;            // first column of this half
     const float tau = (tq < p.T_max) ? p.tau[((size_t)b * p.Hq + h) * p.T_max + tq] : 0.f;
     // l: row sum of the bf16-rounded weights (normalizes O, which the tensor core
-    // built from those weights); lx: row sum of the exact fp32 weights (for lse)
+    // built from those weights); lx: row sum of the exact fp32 weights (for lse);
+    // both over this half's columns until the end
     float m_used = -INFINITY, l = 0.f, lx = 0.f;
     bool ok = true;
-    float sv[TILE];
+    float sv[64];
     // every lane polls; the warp agrees on the outcome so collectives stay converged
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
+    // Both halves of a row pass the same named barriers in every tile, failed or
+    // not: a warp whose bounded wait ran out keeps looping with its work skipped,
+    // so its partner half never blocks on a barrier it will not reach.
+    auto halves_sync = [] { named_bar_sync(3, NWARP_SM * 32); };
+    const bool hard = p.invT < 0.f;
     for (int j = 0; j < nkv; ++j) {
       const int sb = j & 1, s = j % NKV;
-      if (!wwait(&ms->s_full[sb], (uint32_t)(j >> 1) & 1u)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < TILE / 32; ++c) tmem_ld32(tS + sb * 128 + c * 32 + lsel, sv + c * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms->s_free[sb]);
       const int k0 = j * TILE;
-      // 8 independent partial maxima: short dependency chains
-      float pm[8];
+      if (ok && !wwait(&ms->s_full[sb], (uint32_t)(j >> 1) & 1u)) ok = false;
+      float mxh = -INFINITY;
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(tS + sb * 128 + cb + lsel, sv);
+        tmem_ld32(tS + sb * 128 + cb + 32 + lsel, sv + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms->s_free[sb]);
+        // 8 independent partial maxima: short dependency chains
+        float pm[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
-      const bool hard = p.invT < 0.f;
-      const int lim = tq - k0;                         // keys c <= lim are causal
+        for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+        const int lim = tq - k0 - (int)cb;             // columns c <= lim are causal
 #pragma unroll
-      for (int c = 0; c < TILE; ++c) {
-        const float x = p.scale * sv[c];
-        float y;
-        if (hard) y = x >= tau ? x : 0.f;
-        else y = __fdividef(x, 1.f + __expf((tau - x) * p.invT));   // x * sigmoid
-        y = (c <= lim) ? y : -INFINITY;
-        sv[c] = y;
-        pm[c & 7] = fmaxf(pm[c & 7], y);
+        for (int c = 0; c < 64; ++c) {
+          const float x = p.scale * sv[c];
+          float y;
+          if (hard) y = x >= tau ? x : 0.f;
+          else y = __fdividef(x, 1.f + __expf((tau - x) * p.invT));   // x * sigmoid
+          y = (c <= lim) ? y : -INFINITY;
+          sv[c] = y;
+          pm[c & 7] = fmaxf(pm[c & 7], y);
+        }
+        mxh = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                    fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       }
-      const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                             fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      // the row max of the tile: this half's, then the other half's
+      ms->xch[hh][row] = mxh;
+      halves_sync();
+      const float mx = fmaxf(ms->xch[0][row], ms->xch[1][row]);
+      halves_sync();
+      if (!ok) continue;
       // running max: the first tile sets it; later tiles rescale O (in TMEM) only
-      // when the max grew by more than kRescale
+      // when the max grew by more than kRescale.  Both halves of a row take the
+      // same decision from the same values.
       float alpha = 1.f;
       bool resc = false;
       if (m_used == -INFINITY) {
@@ -299,32 +320,35 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       if (__any_sync(0xffffffffu, resc)) {
         // O holds tiles 0 .. j-1: wait for the last P V before touching it (P V of
         // tile j-2 is known complete: it was issued before Q K^T of tile j)
-        if (!wwait(&ms->o_done, (uint32_t)((j - 1) & 1))) { ok = false; break; }
+        if (!wwait(&ms->o_done, (uint32_t)((j - 1) & 1))) {
+          ok = false;
+          continue;
+        }
         tc_fence_after();
         float ov[32];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          tmem_ld32(tO + c * 32 + lsel, ov);
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(tO + cb + c * 32 + lsel, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-          tmem_st32(tO + c * 32 + lsel, ov);
+          tmem_st32(tO + cb + c * 32 + lsel, ov);
         }
         tmem_wait_st();
         tc_fence_before();
         l *= alpha;
         lx *= alpha;
       }
-      // P = exp(s' - m) as bf16, row `row` of the swizzled A tile (two 64-key halves)
-      unsigned char* pbuf = smem + OFF_P + sb * 2 * HALF;
+      // P = exp(s' - m) as bf16, row `row` of this half's swizzled 64-key A tile
+      unsigned char* pbuf = smem + OFF_P + sb * 2 * HALF + hh * HALF;
       float ls4[4] = {0.f, 0.f, 0.f, 0.f}, lx4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int cch = 0; cch < TILE / 8; ++cch) {
+      for (int c16 = 0; c16 < 8; ++c16) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p0 = __expf(sv[cch * 8 + 2 * e] - m_used);
-          const float p1 = __expf(sv[cch * 8 + 2 * e + 1] - m_used);
+          const float p0 = __expf(sv[c16 * 8 + 2 * e] - m_used);
+          const float p1 = __expf(sv[c16 * 8 + 2 * e + 1] - m_used);
           const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
           // the row sum uses the rounded weights the tensor core multiplies, so
           // O / l is an exact convex combination of them (a dominant weight's
@@ -334,20 +358,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           lx4[e] += p0 + p1;
           w[e] = *reinterpret_cast<const uint32_t*>(&pr);
         }
-        const int half = cch >> 3, c16 = cch & 7;
-        *reinterpret_cast<uint4*>(pbuf + half * HALF + row * 128 + ((c16 ^ (row & 7)) << 4)) =
+        *reinterpret_cast<uint4*>(pbuf + row * 128 + ((c16 ^ (row & 7)) << 4)) =
             make_uint4(w[0], w[1], w[2], w[3]);
       }
       l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
       lx += (lx4[0] + lx4[1]) + (lx4[2] + lx4[3]);
       // the last key tile: V rows past the sequence end must be finite for P V
       if (k0 + TILE > len && k0 + row >= len) {
-        unsigned char* vt = smem + OFF_KV + s * KV_STAGE + 2 * HALF;
+        unsigned char* vt = smem + OFF_KV + s * KV_STAGE + 2 * HALF + hh * HALF;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 8; ++c)
           *reinterpret_cast<uint4*>(vt + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(vt + HALF + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-        }
       }
       fence_async_smem();
       __syncwarp();
@@ -355,15 +376,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     }
     // every P V done (a single-phase barrier: no parity aliasing)
     if (ok && !wwait(&ms->o_final, 0u)) ok = false;
+    // the halves' row sums (every warp reaches this point, failed or not)
+    ms->xch[hh][row] = l;
+    halves_sync();
+    const float l_row = ms->xch[0][row] + ms->xch[1][row];
+    halves_sync();
+    ms->xch[hh][row] = lx;
+    halves_sync();
+    const float lx_row = ms->xch[0][row] + ms->xch[1][row];
     if (ok) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / l_row;
       const bool store = tq < len;
-      float* orow = p.O + (((size_t)b * p.Hq + h) * p.T_max + (store ? tq : 0)) * D;
+      float* orow = p.O + (((size_t)b * p.Hq + h) * p.T_max + (store ? tq : 0)) * D + cb;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float ov[32];
-        tmem_ld32(tO + c * 32 + lsel, ov);
+        tmem_ld32(tO + cb + c * 32 + lsel, ov);
         tmem_wait_ld();
         if (store) {
 #pragma unroll
@@ -372,7 +401,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
         }
       }
-      if (store) p.lse[((size_t)b * p.Hq + h) * p.T_max + tq] = m_used + logf(lx);
+      if (store && hh == 0) p.lse[((size_t)b * p.Hq + h) * p.T_max + tq] = m_used + logf(lx_row);
     } else {
       if (threadIdx.x == 0) set_status(p.status, ETA_DEVSTAT_TIMEOUT);
       *abort_flag = 1;

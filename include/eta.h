@@ -254,6 +254,24 @@ eta_status_t eta_decode_step(const eta_dims_t* dims, const eta_bf16_t* q, const 
                              int32_t* dev_status, void* stream);
 
 /*
+ * eta_lse_merge -- merges decode results computed over disjoint key sets into the
+ * result over their union: the log-sum-exp identity of a softmax split over key sets
+ * (Eq. 2-3 of the review make the decode a softmax over gated logits).  With a KV
+ * cache split into block-aligned sequence shards (one per GPU), eta_decode on each
+ * shard with the same thresholds followed by this merge of the gathered results is
+ * the decode of the whole cache: screening is per block, so each shard admits exactly
+ * the blocks of the whole cache's union that lie in its range.
+ *   M = max_p lse_p;  L = sum_p e^(lse_p - M);  o = sum_p e^(lse_p - M) o_p / L;
+ *   lse = M + log L;  parts with lse_p = -inf add nothing; all empty: o = 0, lse = -inf.
+ * o_parts fp32 [n_parts, n_rows, d], lse_parts fp32 [n_parts, n_rows] (device);
+ * o fp32 [n_rows, d], lse fp32 [n_rows] (device, may not alias the parts).
+ * n_rows = B * Hq; d in {64, 128}; n_parts >= 1 (else ETA_ERR_INVALID_ARG).
+ * No workspace, no device status.
+ */
+eta_status_t eta_lse_merge(int32_t n_parts, int32_t n_rows, int32_t d, const float* o_parts,
+                           const float* lse_parts, float* o, float* lse, void* stream);
+
+/*
  * eta_dense_decode -- the dense baseline the speedups are measured against (the
  * pages compare with FlashAttention-2 decode): standard softmax decode attention
  * over every valid key, no threshold, no gate, same split-KV pipeline as eta_decode.

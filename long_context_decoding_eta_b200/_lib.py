@@ -31,7 +31,7 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string",
            "eta_set_decode_engine", "eta_get_decode_engine", "eta_decode_static",
            "eta_decode_static_max_workspace", "eta_selftest_wait_timeout", "eta_prefill",
-           "eta_decode_step_workspace_size", "eta_decode_step")
+           "eta_decode_step_workspace_size", "eta_decode_step", "eta_lse_merge")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 
 
@@ -97,6 +97,8 @@ def lib() -> C.CDLL:
     L.eta_decode_step.argtypes = [DIMS, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P, I32, F32,
                                   F32, F32, P, P, P, P, P, P, P, P, C.c_size_t, P, P]
     L.eta_decode_step.restype = I32
+    L.eta_lse_merge.argtypes = [I32, I32, I32, P, P, P, P, P]
+    L.eta_lse_merge.restype = I32
     L.eta_selftest_wait_timeout.argtypes = [C.c_uint32, P, P, P]
     L.eta_selftest_wait_timeout.restype = I32
     L.eta_set_decode_engine.argtypes = [I32]
@@ -200,6 +202,15 @@ def eta_decode_step(dims: Dims, q, W, bias, tau_const, K, V, lengths, update_tai
         float(scale), _p(tau), _p(head_mask), _p(union_idx), _p(union_cnt), _p(head_cnt),
         _p(o), _p(lse), _p(ws), 0 if ws is None else ws.numel() * ws.element_size(),
         _p(dev_status), _stream(stream)))
+
+
+def eta_lse_merge(o_parts, lse_parts, o, lse, stream=None):
+    """o_parts fp32 [P, ..., d], lse_parts fp32 [P, ...] -> o [..., d], lse [...]
+    (see include/eta.h)."""
+    n_parts, d = int(o_parts.shape[0]), int(o_parts.shape[-1])
+    n_rows = int(lse_parts.numel() // n_parts)
+    _check("eta_lse_merge", lib().eta_lse_merge(
+        n_parts, n_rows, d, _p(o_parts), _p(lse_parts), _p(o), _p(lse), _stream(stream)))
 
 
 def eta_decode_static_max_workspace() -> int:

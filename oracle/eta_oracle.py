@@ -295,6 +295,28 @@ def decode(q: np.ndarray, tau: np.ndarray, K: np.ndarray, V: np.ndarray,
     return o, lse
 
 
+def lse_merge(o_parts: np.ndarray, lse_parts: np.ndarray):
+    """Softmax attention over the union of disjoint key sets from the results over
+    each set (the log-sum-exp identity behind split-KV decoding; Eq. 2-3's softmax
+    is a plain softmax over the gated logits).  Part p has lse_p = log sum e^{l_t}
+    and o_p = the e^{l_t}-weighted mean of its values, so over the union
+    o = sum_p e^{lse_p} o_p / sum_p e^{lse_p} and lse = log sum_p e^{lse_p}
+    (evaluated max-shifted).  Parts with lse = -inf (no keys) add nothing; all
+    empty gives o = 0, lse = -inf.  o_parts [P, ..., d], lse_parts [P, ...]."""
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    m = lse_parts.max(axis=0)
+    finite = np.isfinite(m)
+    shift = np.where(finite, m, 0.0)
+    w = np.where(np.isfinite(lse_parts), np.exp(lse_parts - shift[None]), 0.0)
+    den = w.sum(axis=0)
+    num = (w[..., None] * o_parts).sum(axis=0)
+    safe = np.where(den > 0, den, 1.0)
+    o = np.where((den > 0)[..., None], num / safe[..., None], 0.0)
+    lse = np.where(den > 0, shift + np.log(safe), -np.inf)
+    return o, lse
+
+
 def dense_gated(q_h: np.ndarray, tau_h: float, K_seq: np.ndarray, V_seq: np.ndarray,
                 n_valid: int, scale: float, T: float):
     """Gated attention over every valid key, no pruning (Eq. 2-3)."""

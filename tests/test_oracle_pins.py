@@ -579,3 +579,67 @@ def test_prefill_row_equals_gated_decode_over_its_prefix():
         sp = np.where(s >= tau[b, h, t], s, 0.0)
         p = np.exp(sp - sp.max())
         np.testing.assert_allclose(o[b, h, t], p @ V[b, h // G, :t + 1] / p.sum(), atol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# log-sum-exp merge of results over disjoint key sets (sequence-sharded decode)
+# ----------------------------------------------------------------------------
+def test_lse_merge_equals_softmax_over_the_union():
+    rng = np.random.default_rng(11)
+    n, d = 60, 8
+    logits = rng.normal(0, 3, n)
+    vals = rng.normal(0, 1, (n, d))
+    cut = [0, 17, 17, 41, n]                      # the second part is empty
+    o_parts, lse_parts = [], []
+    for a, b in zip(cut[:-1], cut[1:]):
+        l, v = logits[a:b], vals[a:b]
+        if b > a:
+            w = torch.softmax(torch.tensor(l), 0).numpy()
+            o_parts.append(w @ v)
+            lse_parts.append(float(torch.logsumexp(torch.tensor(l), 0)))
+        else:
+            o_parts.append(np.zeros(d))
+            lse_parts.append(-math.inf)
+    o, lse = O.lse_merge(np.stack(o_parts), np.array(lse_parts))
+    w = torch.softmax(torch.tensor(logits), 0).numpy()
+    np.testing.assert_allclose(o, w @ vals, rtol=0, atol=1e-12)
+    assert abs(lse - float(torch.logsumexp(torch.tensor(logits), 0))) < 1e-12
+    # one part: the identity; every part empty: o = 0, lse = -inf
+    o1, l1 = O.lse_merge(np.stack(o_parts[:1]), np.array(lse_parts[:1]))
+    np.testing.assert_array_equal(o1, o_parts[0])
+    assert l1 == lse_parts[0]
+    oe, le = O.lse_merge(np.zeros((3, d)), np.full(3, -math.inf))
+    assert np.all(oe == 0) and np.isneginf(le)
+
+
+@pytest.mark.parametrize("prune", [O.PRUNE_SKIP, O.PRUNE_FLOOR])
+def test_block_aligned_sequence_shards_merge_to_the_unsharded_decode(prune):
+    """Screening is per block and tau per query, so each shard of a block-aligned
+    split admits exactly the unsharded union's blocks in its range; merging the
+    shards' (o, lse) must give the unsharded decode."""
+    w = synth.TINY.with_(ctx=1024, seed=91)
+    g = synth.generate(w, "cpu", lengths=torch.tensor([1000], dtype=torch.int32))
+    K, V, q = (g[k].double().numpy() for k in ("K", "V", "q"))
+    L = g["lengths"].numpy().astype(np.int64)
+    scale = O.default_scale(w.d)
+    tau = O.predict_tau(q, g["W"].double().numpy(), np.full(w.Hq, 0.3))
+    meta = O.cache_meta(K, L, w.blk, V)
+    sc = O.screen(q, tau, meta, scale)
+    o_ref, lse_ref = O.decode(q, tau, K, V, L, sc["union_idx"], w.blk, scale, 0.05, prune, meta)
+    cuts = [0, 5 * w.blk, 9 * w.blk, w.ctx]       # three shards, the last partly empty
+    o_parts, lse_parts = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        Ls = np.clip(L - a, 0, b - a)
+        ms = O.cache_meta(K[:, :, a:b], Ls, w.blk, V[:, :, a:b])
+        ss = O.screen(q, tau, ms, scale)
+        o_s, l_s = O.decode(q, tau, K[:, :, a:b], V[:, :, a:b], Ls, ss["union_idx"], w.blk,
+                            scale, 0.05, prune, ms)
+        o_parts.append(o_s)
+        lse_parts.append(l_s)
+        # the shard admits exactly the unsharded union's blocks in its range
+        for gg in range(w.Hkv):
+            want = [j - a // w.blk for j in sc["union_idx"][0][gg] if a <= j * w.blk < b]
+            assert list(ss["union_idx"][0][gg]) == want
+    o, lse = O.lse_merge(np.stack(o_parts), np.stack(lse_parts))
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-10)

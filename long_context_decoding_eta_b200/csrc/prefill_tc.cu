@@ -102,6 +102,14 @@ ETA_DEV void tmem_st32(uint32_t taddr, const float* v) {
       : "memory");
 }
 
+// 2^x on the SFU (PTX ex2.approx; -inf gives 0)
+ETA_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
 ETA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 ETA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -285,16 +293,27 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         float pm[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
-        const int lim = tq - k0 - (int)cb;             // columns c <= lim are causal
+        auto gate = [&](float x) -> float {
+          if (hard) return x >= tau ? x : 0.f;
+          return __fdividef(x, 1.f + __expf((tau - x) * p.invT));      // x * sigmoid
+        };
+        if (j == nkv - 1) {
+          // the diagonal tile (k0 == q0): keys past the row's query are masked
+          const int lim = tq - k0 - (int)cb;           // columns c <= lim are causal
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float x = p.scale * sv[c];
-          float y;
-          if (hard) y = x >= tau ? x : 0.f;
-          else y = __fdividef(x, 1.f + __expf((tau - x) * p.invT));   // x * sigmoid
-          y = (c <= lim) ? y : -INFINITY;
-          sv[c] = y;
-          pm[c & 7] = fmaxf(pm[c & 7], y);
+          for (int c = 0; c < 64; ++c) {
+            const float y = (c <= lim) ? gate(p.scale * sv[c]) : -INFINITY;
+            sv[c] = y;
+            pm[c & 7] = fmaxf(pm[c & 7], y);
+          }
+        } else {
+          // every key of an earlier tile precedes every query of this one
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const float y = gate(p.scale * sv[c]);
+            sv[c] = y;
+            pm[c & 7] = fmaxf(pm[c & 7], y);
+          }
         }
         mxh = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
@@ -342,13 +361,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       // P = exp(s' - m) as bf16, row `row` of this half's swizzled 64-key A tile
       unsigned char* pbuf = smem + OFF_P + sb * 2 * HALF + hh * HALF;
       float ls4[4] = {0.f, 0.f, 0.f, 0.f}, lx4[4] = {0.f, 0.f, 0.f, 0.f};
+      const float nm = -m_used * kLog2e;               // e^(y - m) = 2^(y log2e - m log2e)
 #pragma unroll
       for (int c16 = 0; c16 < 8; ++c16) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p0 = __expf(sv[c16 * 8 + 2 * e] - m_used);
-          const float p1 = __expf(sv[c16 * 8 + 2 * e + 1] - m_used);
+          const float p0 = ex2_approx(fmaf(sv[c16 * 8 + 2 * e], kLog2e, nm));
+          const float p1 = ex2_approx(fmaf(sv[c16 * 8 + 2 * e + 1], kLog2e, nm));
           const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
           // the row sum uses the rounded weights the tensor core multiplies, so
           // O / l is an exact convex combination of them (a dominant weight's

@@ -245,9 +245,7 @@ def run_eta(args, rank, world, device):
         if args.graph:
             g_pre.replay()
         else:
-            dec.append_update()
-            dec.predict_tau(q, W, bias, tau_const)
-            dec.screen(q)
+            dec.prepare(q, W, bias, tau_const)
         if ev is not None:
             ev[0].record(stream)
         if args.graph:

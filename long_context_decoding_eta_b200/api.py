@@ -121,14 +121,22 @@ class EtaDecoder:
                           self.ws_step, self.dev_status, stream)
         return self.o, self.lse
 
-    def step(self, q, W=None, bias=None, tau_const=None, stream=None, append: bool = True):
-        """One decode step: tail-block metadata, tau, screening, gated decode."""
-        if self.fused:
-            return self.step_fused(q, W, bias, tau_const, stream, append)
+    def prepare(self, q, W=None, bias=None, tau_const=None, stream=None,
+                append: bool = True):
+        """Everything of the step before the decode: the tail-block metadata (on
+        append), the thresholds, the screening.  (Running the first two on two
+        streams was measured slower: the cross-stream wait costs more than they
+        overlap.)"""
         if append:
             self.append_update(stream)
         self.predict_tau(q, W, bias, tau_const, stream)
         self.screen(q, stream=stream)
+
+    def step(self, q, W=None, bias=None, tau_const=None, stream=None, append: bool = True):
+        """One decode step: tail-block metadata, tau, screening, gated decode."""
+        if self.fused:
+            return self.step_fused(q, W, bias, tau_const, stream, append)
+        self.prepare(q, W, bias, tau_const, stream, append)
         return self.decode(q, stream=stream)
 
     # -- CUDA graphs ----------------------------------------------------------
@@ -149,9 +157,7 @@ class EtaDecoder:
                     self.step_fused(q, W, bias, tau_const)
                     split = False
                 else:
-                    self.append_update()
-                    self.predict_tau(q, W, bias, tau_const)
-                    self.screen(q)
+                    self.prepare(q, W, bias, tau_const)
                     if not split:
                         self.decode(q)
             g_dec = None

@@ -182,19 +182,76 @@ struct FuseCtx {
   int token;
 };
 
+// The fused step: every CTA lays out the CTA shares itself (prefix sum of per-row
+// admitted counts, exactly as plan_kernel) into its shared memory: row_off[0..R], fs->plan = {total,
+// share length}, fs->cta_row = the row holding position blockIdx * share.  Every
+// thread of the CTA calls it.
+ETA_DEV void plan_local(const int32_t* counts, int R, int NB, int* row_off, FuseSmem* fs,
+                        int32_t* status) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int carry = 0;
+  for (int base = 0; base < R; base += NT) {
+    const int r = base + threadIdx.x;
+    int c = r < R ? __ldcg(counts + r) : 0;
+    if (c < 0 || c > NB) {
+      set_status(status, ETA_DEVSTAT_BAD_BLOCK);
+      c = min(max(c, 0), NB);
+    }
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) fs->wsum[warp] = incl;
+    __syncthreads();
+    int wpre = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+      const int v = fs->wsum[w];
+      if (w < warp) wpre += v;
+      total += v;
+    }
+    if (r < R) row_off[r] = carry + wpre + incl - c;
+    carry += total;
+    __syncthreads();
+  }
+  int chunk = (carry + gridDim.x - 1) / gridDim.x;
+  if (chunk < kMinChunk) chunk = kMinChunk;
+  if (threadIdx.x == 0) {
+    row_off[R] = carry;
+    fs->plan[0] = carry;
+    fs->plan[1] = chunk;
+    fs->cta_row = 0;
+  }
+  __syncthreads();
+  const int a = blockIdx.x * chunk;
+  for (int r = threadIdx.x; r < R; r += NT) {
+    const int off = row_off[r], c = row_off[r + 1] - off;
+    if (c > 0 && off <= a && a < off + c) fs->cta_row = r;
+  }
+  __syncthreads();
+}
+
 // The decode of one CTA share.  `smem` is the CTA's dynamic shared memory aligned
 // to 1024 bytes.  Every thread of the CTA calls it.
-// In the fused step the union list and tau were written by other CTAs of the same
-// grid before a grid barrier; plain (L1-cached) loads still see them, because no
-// SM reads those lines before the barrier (the screening reads tau with L2-only
-// loads).  The plan, the prefix sums and the CTA's first row are its own copy in
-// shared memory (p.cta_row points at that one entry).  The partial slots other
-// CTAs write during the decode are read with L2-only loads.
-template <int G, bool DENSE, bool FUSED>
+// LOCAL (the fused step): the plan, the prefix sums and the CTA's first row are the
+// CTA's own copy in shared memory (plan_local; p.cta_row points at that one entry),
+// and the partial results are merged in the kernel: a pair wholly inside one share
+// is written directly, otherwise the CTA writing the pair's last slot merges it (the
+// partial slots other CTAs write are read with L2-only loads).  For the standalone
+// decode this was measured slower than plan_kernel + decode + combine_kernel
+// (merges on the slowest CTAs' critical path), so decode_tc_kernel keeps LOCAL off.
+// FLAGS (the fused step): the union list and tau were written by other CTAs of the
+// same grid, and a row's union list is read once its compaction flag carries this
+// launch's token.  Plain (L1-cached) loads still see them, because no SM reads
+// those lines earlier in the launch (the screening reads tau with L2-only loads).
+template <int G, bool DENSE, bool LOCAL, bool FLAGS>
 ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const CUtensorMap* tmV,
                             const CUtensorMap* tmQ, const TcParams& p, const FuseCtx& fx) {
   static_assert(G >= 1 && G <= 8, "G");
-  static_assert(!(FUSED && DENSE), "the fused step is sparse");
+  static_assert(!(LOCAL && DENSE), "the in-kernel merge is for the sparse decode");
+  static_assert(!FLAGS || LOCAL, "flags come with the local plan");
   TcMisc* ms = reinterpret_cast<TcMisc*>(smem + SM_MISC);
   volatile int* abort_flag = &ms->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -245,7 +302,7 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
   if (warp == NWARP_SM) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      int r = FUSED ? p.cta_row[0] : p.cta_row[blockIdx.x];
+      int r = LOCAL ? p.cta_row[0] : p.cta_row[blockIdx.x];
       int roff = p.row_off[r], rend = p.row_off[r + 1];
       int it = 0;
       bool ok = true;
@@ -280,7 +337,7 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
       int ready_row = -1;
       bool rows_ok = true;
       auto row_ready = [&](int rr) -> bool {
-        if constexpr (FUSED) {
+        if constexpr (FLAGS) {
           if (rr == ready_row) return true;
           for (uint32_t w = 0; w < kWaitLimit; ++w) {
             if (ld_acquire_gpu(fx.ready + rr) == fx.token) {
@@ -441,13 +498,13 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
       }
       named_bar_sync(1, NWARP_SM * 32);
       int p0 = 0, ns = 0;
-      if constexpr (FUSED) {
+      if constexpr (LOCAL) {
         const int off = p.row_off[row], c = p.row_off[row + 1] - off;
         const int chunk = p.plan[1];
         p0 = off / chunk;
         ns = (off + c - 1) / chunk - p0 + 1;
       }
-      if (FUSED && ns == 1) {
+      if (LOCAL && ns == 1) {
         // the whole pair lies in this share: its partial is the merged result (the
         // one-slot merge written out: weight e^(m - m) = 1, or 0 for an empty softmax)
         const int b = row / p.Hkv, g = row % p.Hkv;
@@ -475,7 +532,7 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
           }
         }
         named_bar_sync(1, NWARP_SM * 32);
-        if constexpr (FUSED) {
+        if constexpr (LOCAL) {
           // this slot of the pair is written: count it; the CTA with the pair's last
           // slot merges all of them (threadFenceReduction pattern)
           FuseSmem* fs = reinterpret_cast<FuseSmem*>(smem + SM_FUSE);
@@ -625,7 +682,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  decode_tc_body<G, DENSE, false>(smem, &tmK, &tmV, &tmQ, p, FuseCtx{});
+  decode_tc_body<G, DENSE, false, false>(smem, &tmK, &tmV, &tmQ, p, FuseCtx{});
 }
 
 }  // namespace tc

@@ -415,54 +415,9 @@ step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
   }
 
   // ---------------------------------------------------------------- the share plan
-  // every CTA lays out the shares itself (prefix sum of the union counts over rows,
-  // as plan_kernel) into its shared memory; the counts are the screening's own
+  // every CTA lays out the shares itself, from the screening's own counts
   int* row_off = reinterpret_cast<int*>(smem + tc::SM_ROWOFF);
-  {
-    int carry = 0;
-    for (int base = 0; base < sp.R; base += tc::NT) {
-      const int r = base + threadIdx.x;
-      int c = r < sp.R ? __ldcg(adm_now + r) : 0;
-      if (c < 0 || c > sp.NB) {
-        set_status(sp.status, ETA_DEVSTAT_BAD_BLOCK);
-        c = min(max(c, 0), sp.NB);
-      }
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (lane == 31) fs->wsum[warp] = incl;
-      __syncthreads();
-      int wpre = 0, total = 0;
-#pragma unroll
-      for (int w = 0; w < tc::NT / 32; ++w) {
-        const int v = fs->wsum[w];
-        if (w < warp) wpre += v;
-        total += v;
-      }
-      if (r < sp.R) row_off[r] = carry + wpre + incl - c;
-      carry += total;
-      __syncthreads();
-    }
-    int chunk = (carry + gridDim.x - 1) / gridDim.x;
-    if (chunk < kMinChunk) chunk = kMinChunk;
-    if (threadIdx.x == 0) {
-      row_off[sp.R] = carry;
-      fs->plan[0] = carry;
-      fs->plan[1] = chunk;
-      fs->cta_row = 0;
-    }
-    __syncthreads();
-    // this CTA's first row: the row whose admitted range holds position blockIdx * chunk
-    const int a = blockIdx.x * chunk;
-    for (int r = threadIdx.x; r < sp.R; r += tc::NT) {
-      const int off = row_off[r], c = row_off[r + 1] - off;
-      if (c > 0 && off <= a && a < off + c) fs->cta_row = r;
-    }
-    __syncthreads();
-  }
+  tc::plan_local(adm_now, sp.R, sp.NB, row_off, fs, sp.status);
 
   // ---------------------------------------------------------------- C: decode + merge
   tc::TcParams tpl = tp;
@@ -475,7 +430,7 @@ step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
   fx.lse = sp.lse;
   fx.ready = sp.ready;
   fx.token = tok_compacted;
-  tc::decode_tc_body<G, false, true>(smem, &tmK, &tmV, &tmQ, tpl, fx);
+  tc::decode_tc_body<G, false, true, true>(smem, &tmK, &tmV, &tmQ, tpl, fx);
 }
 
 struct StepWs {

@@ -110,6 +110,13 @@ ETA_DEV float ex2_approx(float x) {
 }
 constexpr float kLog2e = 1.4426950408889634f;
 
+// tanh on the SFU (PTX tanh.approx)
+ETA_DEV float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 ETA_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 ETA_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -276,6 +283,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     // so its partner half never blocks on a barrier it will not reach.
     auto halves_sync = [] { named_bar_sync(3, NWARP_SM * 32); };
     const bool hard = p.invT < 0.f;
+    const float half_invT = 0.5f * p.invT;
     for (int j = 0; j < nkv; ++j) {
       const int sb = j & 1, s = j % NKV;
       const int k0 = j * TILE;
@@ -295,7 +303,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
         auto gate = [&](float x) -> float {
           if (hard) return x >= tau ? x : 0.f;
-          return __fdividef(x, 1.f + __expf((tau - x) * p.invT));      // x * sigmoid
+          // x * sigmoid((x - tau) / T) = hx + hx * tanh((x - tau) / 2T), hx = x / 2:
+          // one SFU op (tanh.approx) instead of an exponential and a reciprocal
+          const float hx = 0.5f * x;
+          return fmaf(hx, tanh_approx((x - tau) * half_invT), hx);
         };
         if (j == nkv - 1) {
           // the diagonal tile (k0 == q0): keys past the row's query are masked

@@ -38,7 +38,7 @@ from long_context_decoding_eta_b200 import synth  # noqa: E402
 METRIC = "decode attn steps/s and HBM GB/s on admitted KV bytes (% of B200 peak)"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
-LAUNCHES_PER_STEP = 7   # meta tail 1 + tau 1 + screen 2 + decode 3 (plan, decode, combine)
+LAUNCHES_PER_STEP = 6   # tail + tau 1 + screen 2 + decode 3 (plan, decode, combine)
 LAUNCHES_PER_FUSED_STEP = 1   # eta_decode_step: one persistent kernel
 
 
@@ -164,11 +164,13 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def setup(w: synth.Workload, device, rank: int, cent_format: str = "f32", fused: bool = False):
+def setup(w: synth.Workload, device, rank: int, cent_format: str = "f32", fused: bool = False,
+          merged_prologue: bool = True):
     from long_context_decoding_eta_b200.api import EtaDecoder
     g = synth.generate(w, device, seed=w.seed + 7919 * rank)
     dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, bound=w.bound, z=w.z,
-                     T=w.gate_T, keep_bounds=True, cent_format=cent_format, fused=fused)
+                     T=w.gate_T, keep_bounds=True, cent_format=cent_format, fused=fused,
+                     merged_prologue=merged_prologue)
     dec.build_meta()
     # workload calibration: bias so that tau hits the density target
     if w.tau_mode == "const":
@@ -219,7 +221,8 @@ def run_eta(args, rank, world, device):
     _lib.eta_set_decode_engine(args.engine)
     w = workload_by_name(args.workload, args.B)
     fused = bool(args.fused)
-    g, dec, W, bias, tau_const = setup(w, device, rank, args.cent, fused)
+    g, dec, W, bias, tau_const = setup(w, device, rank, args.cent, fused,
+                                       not args.separate_prologue)
     q = g["q"]
     stream = torch.cuda.current_stream()
     # one step to measure densities / bytes, then check status
@@ -344,6 +347,7 @@ def run_eta(args, rank, world, device):
             "context": w.ctx, "blk": w.blk, "bound": w.bound, "gate_T": w.gate_T,
             "tau_mode": w.tau_mode, "engine": args.engine, "centroids": args.cent,
             "cuda_graph": bool(args.graph), "fused_step": fused,
+            "prologue": "separate" if args.separate_prologue else "one launch",
             "density_target": f"{w.density:.2f} {w.density_kind}",
             "union_density": round(by["union_density"], 4),
             "head_density": round(by["head_density"], 4),
@@ -375,7 +379,8 @@ def run_eta(args, rank, world, device):
         "e2e": {"value": job_throughput(world, 1, e2e_ms), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host.numel() * 2,
                 "d2h_bytes_per_step": o_host.numel() * 4 + lse_host.numel() * 4},
-        "gpu_launches": (LAUNCHES_PER_FUSED_STEP if fused else LAUNCHES_PER_STEP) * args.steps,
+        "gpu_launches": (LAUNCHES_PER_FUSED_STEP if fused else
+                         LAUNCHES_PER_STEP + (1 if args.separate_prologue else 0)) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -559,6 +564,8 @@ def main():
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     ap.add_argument("--engine", default="auto", choices=["auto", "tcgen05", "fma"],
                     help="decode engine of libeta.so")
+    ap.add_argument("--separate-prologue", action="store_true",
+                    help="tail refresh and tau as two launches (default: one)")
     ap.add_argument("--fused", action="store_true",
                     help="run the step as one eta_decode_step launch (persistent kernel)")
     ap.add_argument("--graph", action="store_true",

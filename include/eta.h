@@ -149,6 +149,24 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  *   head_cnt   int32  [B, Hq] or NULL: popcount of the head's admit mask
  * ws/ws_bytes: scratch of at least eta_screen_workspace_size(dims) bytes.
  */
+/*
+ * eta_append_and_predict_tau -- eta_build_block_meta(..., ETA_TAIL_BLOCK, ...) and
+ * eta_predict_tau in one launch (the two parts of a step that precede the screening
+ * and do not depend on each other): one CTA per (batch row, KV head) refreshes the
+ * tail block's metadata with half its warps while the other half computes the
+ * group's thresholds.  Arguments and layouts as those two calls (vsum, vardim
+ * nullable as there; W / bias as eta_predict_tau, or tau_const non-NULL for the
+ * frozen constants).  Writes the same bits as the two calls.  dev_status:
+ * ETA_DEVSTAT_NONFINITE_Q.
+ */
+eta_status_t eta_append_and_predict_tau(const eta_dims_t* dims, const eta_bf16_t* K,
+                                        const eta_bf16_t* V, const int32_t* lengths,
+                                        eta_cent_format_t cent_format, void* cent, float* rmax,
+                                        float* var, int32_t* cnt, float* vsum, float* vardim,
+                                        const eta_bf16_t* q, const float* W, const float* bias,
+                                        const float* tau_const, float* tau,
+                                        int32_t* dev_status, void* stream);
+
 size_t eta_screen_workspace_size(const eta_dims_t* dims);
 eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                         eta_cent_format_t cent_format, const void* cent, const float* rmax,

@@ -31,7 +31,8 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_calibrate_const_tau", "eta_status_from_device", "eta_status_string",
            "eta_set_decode_engine", "eta_get_decode_engine", "eta_decode_static",
            "eta_decode_static_max_workspace", "eta_selftest_wait_timeout", "eta_prefill",
-           "eta_decode_step_workspace_size", "eta_decode_step", "eta_lse_merge")
+           "eta_decode_step_workspace_size", "eta_decode_step", "eta_lse_merge",
+           "eta_append_and_predict_tau")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 
 
@@ -97,6 +98,9 @@ def lib() -> C.CDLL:
     L.eta_decode_step.argtypes = [DIMS, P, P, P, P, P, P, P, I32, I32, P, P, P, P, P, I32, F32,
                                   F32, F32, P, P, P, P, P, P, P, P, C.c_size_t, P, P]
     L.eta_decode_step.restype = I32
+    L.eta_append_and_predict_tau.argtypes = [DIMS, P, P, P, I32, P, P, P, P, P, P, P, P, P, P,
+                                             P, P, P]
+    L.eta_append_and_predict_tau.restype = I32
     L.eta_lse_merge.argtypes = [I32, I32, I32, P, P, P, P, P]
     L.eta_lse_merge.restype = I32
     L.eta_selftest_wait_timeout.argtypes = [C.c_uint32, P, P, P]
@@ -144,6 +148,15 @@ def eta_predict_tau(dims: Dims, q, W, bias, tau_const, tau, dev_status=None, str
     _check("eta_predict_tau", lib().eta_predict_tau(
         C.byref(dims), _p(q), _p(W), _p(bias), _p(tau_const), _p(tau), _p(dev_status),
         _stream(stream)))
+
+
+def eta_append_and_predict_tau(dims: Dims, K, V, lengths, cent, rmax, var, cnt, vsum, vardim, q,
+                               W, bias, tau_const, tau, dev_status=None, stream=None):
+    """Tail-block metadata refresh and thresholds in one launch (see include/eta.h)."""
+    _check("eta_append_and_predict_tau", lib().eta_append_and_predict_tau(
+        C.byref(dims), _p(K), _p(V), _p(lengths), _cent_format(cent), _p(cent), _p(rmax),
+        _p(var), _p(cnt), _p(vsum), _p(vardim), _p(q), _p(W), _p(bias), _p(tau_const), _p(tau),
+        _p(dev_status), _stream(stream)))
 
 
 def eta_screen_workspace_size(dims: Dims) -> int:

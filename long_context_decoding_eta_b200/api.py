@@ -29,7 +29,8 @@ class EtaDecoder:
     def __init__(self, K: torch.Tensor, V: torch.Tensor, lengths: torch.Tensor, Hq: int,
                  blk: int, *, bound: str = "exact", z: float = 3.0, T: float = 0.0,
                  scale: float = 0.0, prune: str = "skip", keep_bounds: bool = False,
-                 cent_format: str = "f32", fused: bool = False):
+                 cent_format: str = "f32", fused: bool = False,
+                 merged_prologue: bool = True):
         if not K.is_cuda:
             raise ValueError("K/V must be CUDA tensors")
         if K.dtype != torch.bfloat16 or V.dtype != torch.bfloat16:
@@ -71,6 +72,7 @@ class EtaDecoder:
                                      dtype=torch.uint8, device=dev)
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
         self.fused = bool(fused)
+        self.merged_prologue = bool(merged_prologue)
         if self.fused and prune != "skip":
             raise ValueError("the fused step offers SKIP pruning only")
         # the fused step's workspace holds self-resetting counters: zero it once
@@ -124,12 +126,17 @@ class EtaDecoder:
     def prepare(self, q, W=None, bias=None, tau_const=None, stream=None,
                 append: bool = True):
         """Everything of the step before the decode: the tail-block metadata (on
-        append), the thresholds, the screening.  (Running the first two on two
-        streams was measured slower: the cross-stream wait costs more than they
-        overlap.)"""
-        if append:
-            self.append_update(stream)
-        self.predict_tau(q, W, bias, tau_const, stream)
+        append) and the thresholds (one launch, eta_append_and_predict_tau, unless
+        merged_prologue is off), then the screening."""
+        if append and self.merged_prologue:
+            L.eta_append_and_predict_tau(self.dims, self.K, self.V, self.lengths, self.cent,
+                                         self.rmax, self.var, self.cnt, self.vsum, self.vardim,
+                                         q, W, bias, tau_const, self.tau, self.dev_status,
+                                         stream)
+        else:
+            if append:
+                self.append_update(stream)
+            self.predict_tau(q, W, bias, tau_const, stream)
         self.screen(q, stream=stream)
 
     def step(self, q, W=None, bias=None, tau_const=None, stream=None, append: bool = True):

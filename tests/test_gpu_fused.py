@@ -164,3 +164,31 @@ def test_rejects_unsupported():
     with pytest.raises(ValueError):
         EtaDecoder(g["K"].to(DEV), g["V"].to(DEV), g["lengths"].to(DEV), w.Hq, w.blk,
                    fused=True, prune="floor")
+
+
+@pytest.mark.parametrize("cent_format,bound,tau_mode", [("f32", "exact", "predictor"),
+                                                         ("bf16", "prob_dim", "predictor"),
+                                                         ("bf16", "exact", "const")])
+def test_append_and_predict_tau_equals_the_two_calls(cent_format, bound, tau_mode):
+    """eta_append_and_predict_tau writes the same bits as eta_build_block_meta on the tail
+    block plus eta_predict_tau, after a token was appended to each row with room."""
+    w = synth.MID.with_(B=4, ctx=4096, needles=0, seed=420)
+    lengths = torch.tensor([4096, 0, 1, 2000], dtype=torch.int32)
+    g = synth.generate(w, "cpu", lengths=lengths)
+    K, V, q, W = (g[k].to(DEV) for k in ("K", "V", "q", "W"))
+    lens = g["lengths"].to(DEV)
+    kw = dict(bound=bound, cent_format=cent_format, prune="floor")
+    a = EtaDecoder(K, V, lens, w.Hq, w.blk, merged_prologue=False, **kw)
+    b = EtaDecoder(K, V, lens, w.Hq, w.blk, merged_prologue=True, **kw)
+    a.build_meta()
+    b.build_meta()
+    _append_token(K, V, a.lengths, torch.Generator().manual_seed(421))
+    bias = torch.full((w.Hq,), 0.7, device=DEV)
+    tc = torch.linspace(1.0, 2.0, w.Hq, device=DEV) if tau_mode == "const" else None
+    Wp = None if tc is not None else W
+    a.prepare(q, Wp, bias, tc)
+    b.prepare(q, Wp, bias, tc)
+    torch.cuda.synchronize()
+    a.check_status()
+    b.check_status()
+    _assert_identical(_outputs(a), _outputs(b))

@@ -55,6 +55,14 @@ ETA_DEV void combine_merge(const float* part_ml, const float* part_o, int r, int
   if (ns > 0) {
     const int np = G * ns;                 // pair k = slot * G + h
     if (np <= kCombineMaxPairs) {
+      // the first batch of partial outputs is loaded with the (m, l) pairs: it does not
+      // depend on them, so their latencies overlap
+      float v0[kMergeBatch];
+#pragma unroll
+      for (int u = 0; u < kMergeBatch; ++u) {
+        const size_t sl = ((size_t)(p0 + u / G) + r) * G + (u % G);
+        v0[u] = u < np ? ld_part<CG>(part_o + sl * D + dd) : 0.f;
+      }
       for (int k = dd; k < np; k += D) {
         const size_t sl = ((size_t)(p0 + k / G) + r) * G + (k % G);
         sc.m[k] = ld_part<CG>(part_ml + sl * 2);
@@ -82,7 +90,7 @@ ETA_DEV void combine_merge(const float* part_ml, const float* part_o, int r, int
         for (int u = 0; u < kMergeBatch; ++u) {
           const int k = k0 + u;
           const size_t sl = ((size_t)(p0 + k / G) + r) * G + (k % G);
-          v[u] = k < np ? ld_part<CG>(part_o + sl * D + dd) : 0.f;
+          v[u] = k0 == 0 ? v0[u] : k < np ? ld_part<CG>(part_o + sl * D + dd) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kMergeBatch; ++u) {

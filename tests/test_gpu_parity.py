@@ -94,6 +94,28 @@ def test_ragged_lengths_empty_and_single_token_rows():
         assert np.all(gpu["o"][1] == 0) and np.all(np.isneginf(gpu["lse"][1]))
 
 
+@pytest.mark.parametrize("B,Hkv", [(8, 4), (11, 3), (1, 1)])
+def test_batch_shapes_and_repeat_determinism(B, Hkv):
+    """Batches of 32, 33 and 1 (batch row, KV head) pairs, with empty, single-token,
+    single-block and ragged rows, against the oracle; repeated steps on one decoder
+    are bit-identical (the split plan and the combine order depend only on the
+    admitted counts)."""
+    w = synth.MID.with_(B=B, Hkv=Hkv, Hq=4 * Hkv, ctx=4096, needles=2, seed=90 + B)
+    lens = [4096, 0, 64, 4031, 1, 3000, 128, 2049, 4096, 777, 3333][:B]
+    lengths = torch.tensor(lens, dtype=torch.int32)
+    rep, gpu, sc = full_parity(w, lengths=lengths, density=0.4)
+    if B > 1:
+        assert np.all(gpu["o"][1] == 0) and np.all(np.isneginf(gpu["lse"][1]))
+    gd = to_dev(make(w, lengths))
+    dec = EtaDecoder(gd["K"], gd["V"], gd["lengths"], w.Hq, w.blk, T=w.gate_T)
+    dec.build_meta()
+    bias = torch.full((w.Hq,), 1.5, device=DEV)
+    first = run_cuda(dec, gd["q"], gd["W"], bias)
+    for _ in range(2):
+        again = run_cuda(dec, gd["q"], gd["W"], bias)
+        assert np.array_equal(again["o"], first["o"]) and np.array_equal(again["lse"], first["lse"])
+
+
 @pytest.mark.parametrize("d,G,blk", [(64, 1, 64), (64, 8, 128), (128, 2, 128), (128, 8, 64),
                                      (128, 4, 128)])
 def test_shapes(d, G, blk):

@@ -38,7 +38,8 @@ from long_context_decoding_eta_b200 import synth  # noqa: E402
 METRIC = "decode attn steps/s and HBM GB/s on admitted KV bytes (% of B200 peak)"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
-LAUNCHES_PER_STEP = 6   # tail + tau 1 + screen 2 + decode 3 (plan, decode, combine)
+PROLOGUE_LAUNCHES = 1   # tail-block metadata + tau in one launch (2 when separate)
+DECODE_LAUNCHES = 3     # plan, split-KV decode, combine
 LAUNCHES_PER_FUSED_STEP = 1   # eta_decode_step: one persistent kernel
 
 
@@ -380,7 +381,9 @@ def run_eta(args, rank, world, device):
                 "h2d_bytes_per_step": q_host.numel() * 2,
                 "d2h_bytes_per_step": o_host.numel() * 4 + lse_host.numel() * 4},
         "gpu_launches": (LAUNCHES_PER_FUSED_STEP if fused else
-                         LAUNCHES_PER_STEP + (1 if args.separate_prologue else 0)) * args.steps,
+                         PROLOGUE_LAUNCHES + (1 if args.separate_prologue else 0) +
+                         _lib.eta_screen_launches(dec.dims, args.cent) + DECODE_LAUNCHES)
+                        * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -148,6 +148,10 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  *   bounds_out fp32   [B, Hq, NB] or NULL (calibration, near-tie logging)
  *   head_cnt   int32  [B, Hq] or NULL: popcount of the head's admit mask
  * ws/ws_bytes: scratch of at least eta_screen_workspace_size(dims) bytes.
+ * Kernel launches: one (screening and compaction together, one CTA per (row, KV
+ * head) pair: batches of at most two CTAs per SM whose rows fit two rounds of the
+ * CTA's group buffers, NB a multiple of 8 for bf16 centroids or 4 for fp32) or two
+ * (screening, then compaction); eta_screen_launches says which.
  */
 /*
  * eta_append_and_predict_tau -- eta_build_block_meta(..., ETA_TAIL_BLOCK, ...) and
@@ -168,6 +172,10 @@ eta_status_t eta_append_and_predict_tau(const eta_dims_t* dims, const eta_bf16_t
                                         int32_t* dev_status, void* stream);
 
 size_t eta_screen_workspace_size(const eta_dims_t* dims);
+/* Kernel launches eta_screen makes on the current device for these dims and centroid
+ * format when every pointer argument is 16-byte aligned (1 or 2; 2 without a
+ * device), or -1 for invalid dims. */
+int32_t eta_screen_launches(const eta_dims_t* dims, eta_cent_format_t cent_format);
 eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                         eta_cent_format_t cent_format, const void* cent, const float* rmax,
                         const float* var, const float* vardim,

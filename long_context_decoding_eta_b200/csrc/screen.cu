@@ -15,7 +15,10 @@
 
 #include "eta_common.cuh"
 #include "eta_host.h"
+#include "compact_dev.cuh"
+#include "decode_tc.cuh"   // tc::tma_load_2d
 #include "screen_dev.cuh"
+#include "tma_host.h"
 
 namespace eta {
 
@@ -142,53 +145,124 @@ compact_kernel(int Hq, int Hkv, int G, int NB, int NW, const uint32_t* __restric
                const uint32_t* __restrict__ head_mask, int32_t* __restrict__ union_idx,
                int32_t* __restrict__ union_cnt, int32_t* __restrict__ head_cnt) {
   ETA_PDL_ENTRY();
-  __shared__ uint32_t wbuf[kCompactThreads];
-  __shared__ int woff[kCompactThreads];
-  __shared__ int wsum[kCompactThreads / 32];
-  const int r = blockIdx.x;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int carry = 0;
-  for (int base = 0; base < NW; base += kCompactThreads) {
-    const int w = base + tid;
-    const uint32_t word = w < NW ? union_words[(size_t)r * NW + w] : 0u;
-    const int c = __popc(word);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int wpre = 0, total = 0;
-#pragma unroll
-    for (int i = 0; i < kCompactThreads / 32; ++i) {
-      const int v = wsum[i];
-      if (i < warp) wpre += v;
-      total += v;
-    }
-    wbuf[tid] = word;
-    woff[tid] = carry + wpre + incl - c;
-    __syncthreads();
-    for (int i = warp; i < kCompactThreads && base + i < NW; i += kCompactThreads / 32) {
-      const uint32_t wd = wbuf[i];
-      if ((wd >> lane) & 1u)
-        union_idx[(size_t)r * NB + woff[i] + __popc(wd & ((1u << lane) - 1u))] =
-            (base + i) * 32 + lane;
-    }
-    carry += total;
-    __syncthreads();
+  __shared__ CompactScratch<kCompactThreads> cs;
+  compact_row<kCompactThreads>(blockIdx.x, Hq, Hkv, G, NB, NW, union_words, head_mask, union_idx,
+                               union_cnt, head_cnt, cs);
+}
+
+// Small batches: one CTA per (row, KV head) pair screens the whole row and compacts
+// it in the same launch.  Each warp owns one shared-memory buffer and screens the
+// groups warp, warp + NBUF, ...; a group's [D][128] dimension-major centroid tile
+// arrives by one TMA tensor copy and its rmax / var / cnt slices by 1-D bulk copies,
+// so a group costs one memory round trip instead of D / kScreenLoadBatch dependent
+// ones.  The arithmetic is screen_group_from's, as in screen_vec_kernel and the
+// fused step: the masks and bounds are bit-identical to theirs.
+template <int D, int CF>
+struct RowScreenCfg {
+  static constexpr int CENT = D * kScreenGroupBlocks * (CF == 1 ? 2 : 4);
+  static constexpr int OFF_RMAX = CENT;
+  static constexpr int OFF_VAR = CENT + 4 * kScreenGroupBlocks;
+  static constexpr int OFF_CNT = CENT + 8 * kScreenGroupBlocks;
+  static constexpr int SB = (CENT + 12 * kScreenGroupBlocks + 1023) / 1024 * 1024;
+  static constexpr int NBUF_FIT = (192 * 1024) / SB;
+  static constexpr int NBUF = NBUF_FIT > 8 ? 8 : NBUF_FIT;   // = warps per CTA
+  static constexpr int NT = NBUF * 32;
+  static constexpr int SMEM = NBUF * SB + 1024;               // + alignment slack
+  static_assert(NBUF >= 2, "two group buffers must fit");
+};
+// At most this many rounds of NBUF groups per row take the one-launch path.
+constexpr int kRowScreenMaxRounds = 2;
+
+template <int D, int G, int CF, bool VD>
+__global__ void __launch_bounds__(RowScreenCfg<D, CF>::NT, 1)
+screen_row_kernel(const __grid_constant__ CUtensorMap tmC, int Hq, int Hkv, int NB, int NW,
+                  const eta_bf16_t* __restrict__ q, const float* __restrict__ tau,
+                  const float* __restrict__ rmax, const float* __restrict__ var,
+                  const float* __restrict__ vardim, const int32_t* __restrict__ cnt, int bound,
+                  float z, float scale, uint32_t* head_mask, uint32_t* union_words,
+                  float* __restrict__ bounds_out, int32_t* __restrict__ union_idx,
+                  int32_t* __restrict__ union_cnt, int32_t* __restrict__ head_cnt,
+                  int32_t* status) {
+  using C = RowScreenCfg<D, CF>;
+  ETA_PDL_ENTRY();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(16) float qs[D * G];
+  __shared__ float qn[G], ts[G];
+  __shared__ __align__(8) uint64_t full[C::NBUF];
+  __shared__ CompactScratch<C::NT> cs;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x, b = r / Hkv, g = r % Hkv;
+  const size_t qhead0 = (size_t)b * Hq + (size_t)g * G;
+  const int ngrp = (NB + kScreenGroupBlocks - 1) / kScreenGroupBlocks;
+  const bool pv = bound == ETA_BOUND_PROB;
+
+  auto issue = [&](int buf, int grp) {
+    unsigned char* st = smem + buf * C::SB;
+    const int j0 = grp * kScreenGroupBlocks;
+    const uint32_t nb4 = (uint32_t)min(kScreenGroupBlocks, NB - j0) * 4u;
+    mbar_arrive_expect_tx(&full[buf], (uint32_t)C::CENT + nb4 * (pv ? 3u : 2u));
+    tc::tma_load_2d(st, &tmC, j0, r * D, &full[buf]);
+    const size_t rj = (size_t)r * NB + j0;
+    bulk_g2s(st + C::OFF_RMAX, rmax + rj, nb4, &full[buf]);
+    if (pv) bulk_g2s(st + C::OFF_VAR, var + rj, nb4, &full[buf]);
+    bulk_g2s(st + C::OFF_CNT, cnt + rj, nb4, &full[buf]);
+  };
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NBUF; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+    for (int i = 0; i < C::NBUF && i < ngrp; ++i) issue(i, i);   // first round in flight
   }
-  if (tid == 0) union_cnt[r] = carry;
-  if (head_cnt && warp < G) {
-    const int b = r / Hkv, g = r % Hkv;
-    const size_t hq = (size_t)b * Hq + (size_t)g * G + warp;
-    int s = 0;
-    for (int w = lane; w < NW; w += 32) s += __popc(head_mask[hq * NW + w]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) head_cnt[hq] = s;
+  for (int i = threadIdx.x; i < G * D; i += C::NT) {
+    const int h = i / D, k = i % D;
+    qs[k * G + h] = bf16_to_f(q[(qhead0 + h) * D + k]);
   }
+  __syncthreads();
+  for (int h = warp; h < G; h += C::NBUF) {
+    const float nrm = query_norm<D, G>(qs, h);
+    if (lane == 0) {
+      qn[h] = nrm;
+      ts[h] = tau[qhead0 + h];
+    }
+  }
+  __syncthreads();
+
+  bool ok = true;
+  int round = 0;
+  for (int grp = warp; grp < ngrp && ok; grp += C::NBUF, ++round) {
+    if (round > 0) {
+      // the buffer's previous tile was read by this warp's generic loads
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) issue(warp, grp);
+    }
+    if (!mbar_wait(&full[warp], (uint32_t)round & 1u, nullptr)) {
+      if (lane == 0) set_status(status, ETA_DEVSTAT_TIMEOUT);
+      ok = false;
+      break;
+    }
+    const unsigned char* st = smem + warp * C::SB;
+    SmemMeta<CF, VD> src;
+    src.tile = st;
+    const int jl = min(grp * kScreenGroupBlocks + lane * kScreenVW, NB - kScreenVW);
+    src.vdp = VD ? reinterpret_cast<const float4*>(vardim + (size_t)r * D * NB + jl) : nullptr;
+    src.rowvd = (size_t)NB / 4;
+    src.rmax = reinterpret_cast<const float*>(st + C::OFF_RMAX);
+    src.var = reinterpret_cast<const float*>(st + C::OFF_VAR);
+    src.cnt = reinterpret_cast<const int32_t*>(st + C::OFF_CNT);
+    src.lane = lane;
+    screen_group_from<D, G, CF, VD, kScreenLoadBatch>(src, NB, NW, grp, r, qhead0, qs, qn, ts,
+                                                      bound, z, scale, NB, head_mask,
+                                                      union_words, bounds_out);
+    __syncwarp();
+  }
+  // a warp that gave up leaves its copy in flight: wait for it (bounded) before the
+  // CTA's shared memory can be released
+  if (!ok && lane == 0) mbar_wait(&full[warp], (uint32_t)round & 1u, nullptr);
+  __syncthreads();
+  compact_row<C::NT>(r, Hq, Hkv, G, NB, NW, union_words, head_mask, union_idx, union_cnt,
+                     head_cnt, cs);
 }
 
 template <int D, int CF, bool VD>
@@ -214,6 +288,43 @@ static eta_status_t launch_screen(bool vec, int G, dim3 grid, cudaStream_t s, in
                   bound, z, scale, head_mask, uw, bounds_out);
 }
 
+template <int D, int CF, bool VD>
+static eta_status_t launch_screen_row(int G, const CUtensorMap& mc, int R, cudaStream_t s, int Hq,
+                                      int Hkv, int NB, int NW, const eta_bf16_t* q,
+                                      const float* tau, const float* rmax, const float* var,
+                                      const float* vardim, const int32_t* cnt, int bound, float z,
+                                      float scale, uint32_t* head_mask, uint32_t* uw,
+                                      float* bounds_out, int32_t* union_idx, int32_t* union_cnt,
+                                      int32_t* head_cnt, int32_t* status) {
+  using C = RowScreenCfg<D, CF>;
+#define ETA_ROW_LAUNCH(GG)                                                                     \
+  do {                                                                                         \
+    if (!set_smem_once<screen_row_kernel<D, GG, CF, VD>>(C::SMEM)) return ETA_ERR_CUDA;        \
+    return launch_k(screen_row_kernel<D, GG, CF, VD>, dim3(R), dim3(C::NT), C::SMEM, s, mc, Hq, \
+                    Hkv, NB, NW, q, tau, rmax, var, vardim, cnt, bound, z, scale, head_mask,   \
+                    uw, bounds_out, union_idx, union_cnt, head_cnt, status);                   \
+  } while (0)
+  switch (G) {
+    case 1: ETA_ROW_LAUNCH(1);
+    case 2: ETA_ROW_LAUNCH(2);
+    case 4: ETA_ROW_LAUNCH(4);
+    case 8: ETA_ROW_LAUNCH(8);
+  }
+#undef ETA_ROW_LAUNCH
+  return ETA_ERR_UNSUPPORTED;
+}
+
+// Whether the one-launch screen takes this call: few pairs (at most two waves of
+// CTAs), rows of at most kRowScreenMaxRounds rounds of group buffers, and the
+// alignment its bulk copies need.
+template <int D, int CF>
+static bool row_screen_fits(int R, int NB) {
+  using C = RowScreenCfg<D, CF>;
+  const int ngrp = (NB + kScreenGroupBlocks - 1) / kScreenGroupBlocks;
+  return R <= 2 * sm_count() && ngrp <= kRowScreenMaxRounds * C::NBUF &&
+         NB % (CF == 1 ? 8 : 4) == 0;
+}
+
 }  // namespace eta
 
 using namespace eta;
@@ -223,6 +334,17 @@ extern "C" size_t eta_screen_workspace_size(const eta_dims_t* dims) {
   return align_up((size_t)dims->B * dims->Hkv * num_words(dims) * sizeof(uint32_t), 256);
 }
 
+extern "C" int32_t eta_screen_launches(const eta_dims_t* dims, eta_cent_format_t cent_format) {
+  if (check_dims(dims) != ETA_OK) return -1;
+  const int NB = num_blocks(dims), R = dims->B * dims->Hkv;
+  const bool bf = cent_format == ETA_CENT_BF16;
+  if (NB % 4 != 0) return 2;
+  bool row;
+  if (dims->d == 128) row = bf ? row_screen_fits<128, 1>(R, NB) : row_screen_fits<128, 0>(R, NB);
+  else row = bf ? row_screen_fits<64, 1>(R, NB) : row_screen_fits<64, 0>(R, NB);
+  return row ? 1 : 2;
+}
+
 extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                                    eta_cent_format_t cent_format, const void* cent,
                                    const float* rmax, const float* var, const float* vardim,
@@ -230,7 +352,6 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
                                    uint32_t* head_mask, int32_t* union_idx, int32_t* union_cnt,
                                    float* bounds_out, int32_t* head_cnt, void* ws,
                                    size_t ws_bytes, int32_t* dev_status, void* stream) {
-  (void)dev_status;
   eta_status_t st = check_dims(dims);
   if (st != ETA_OK) return st;
   if (!q || !tau || !cent || !rmax || !cnt || !head_mask || !union_idx || !union_cnt)
@@ -252,6 +373,33 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   const bool vec = (NB % VW == 0) && aligned16(cent) && aligned16(rmax) && aligned16(cnt) &&
                    (!var || aligned16(var)) && (!vardim || aligned16(vardim)) &&
                    (!bounds_out || aligned16(bounds_out));
+  bool row = vec;
+  if (row) {
+    if (dims->d == 128) row = bf ? row_screen_fits<128, 1>(R, NB) : row_screen_fits<128, 0>(R, NB);
+    else row = bf ? row_screen_fits<64, 1>(R, NB) : row_screen_fits<64, 0>(R, NB);
+  }
+  if (row) {
+    CUtensorMap mc;
+    if (!make_map_plain(&mc, cent, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                        NB, (uint64_t)R * dims->d, (uint64_t)NB * (bf ? 2 : 4),
+                        kScreenGroupBlocks, dims->d))
+      return ETA_ERR_CUDA;
+#define ETA_ROW_ARGS G, mc, R, s, dims->Hq, dims->Hkv, NB, NW, q, tau, rmax, var, vardim, cnt, \
+                     (int)bound, z, scale, head_mask, uw, bounds_out, union_idx, union_cnt,   \
+                     head_cnt, dev_status
+    if (dims->d == 128) {
+      if (vd) return bf ? launch_screen_row<128, 1, true>(ETA_ROW_ARGS)
+                        : launch_screen_row<128, 0, true>(ETA_ROW_ARGS);
+      return bf ? launch_screen_row<128, 1, false>(ETA_ROW_ARGS)
+                : launch_screen_row<128, 0, false>(ETA_ROW_ARGS);
+    }
+    if (vd) return bf ? launch_screen_row<64, 1, true>(ETA_ROW_ARGS)
+                      : launch_screen_row<64, 0, true>(ETA_ROW_ARGS);
+    return bf ? launch_screen_row<64, 1, false>(ETA_ROW_ARGS)
+              : launch_screen_row<64, 0, false>(ETA_ROW_ARGS);
+#undef ETA_ROW_ARGS
+  }
   dim3 grid;
   if (vec) {
     const int ngroups = (NB + 32 * VW - 1) / (32 * VW);

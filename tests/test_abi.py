@@ -88,6 +88,9 @@ def test_argument_validation_without_gpu():
     assert lib.eta_predict_tau(ctypes.byref(g3), *([None] * 7)) == 2
     assert L.eta_screen_workspace_size(dims) == 256       # 2*4 rows x 2 words, 256-aligned
     assert L.eta_screen_workspace_size(bad) == 0
+    # launch-count query: invalid dims are refused; without a device the two-launch form
+    assert lib.eta_screen_launches(ctypes.byref(bad), 1) == -1
+    assert lib.eta_screen_launches(ctypes.byref(dims), 1) in (1, 2)
 
 
 def test_engine_selection_host_only():

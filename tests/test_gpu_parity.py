@@ -103,6 +103,9 @@ def test_batch_shapes_and_repeat_determinism(B, Hkv):
     w = synth.MID.with_(B=B, Hkv=Hkv, Hq=4 * Hkv, ctx=4096, needles=2, seed=90 + B)
     lens = [4096, 0, 64, 4031, 1, 3000, 128, 2049, 4096, 777, 3333][:B]
     lengths = torch.tensor(lens, dtype=torch.int32)
+    from long_context_decoding_eta_b200 import _lib as L
+    # these small batches take the one-launch screen (screening + compaction)
+    assert L.eta_screen_launches(L.Dims.of(B, w.Hq, w.Hkv, w.d, w.blk, w.T_max), "f32") == 1
     rep, gpu, sc = full_parity(w, lengths=lengths, density=0.4)
     if B > 1:
         assert np.all(gpu["o"][1] == 0) and np.all(np.isneginf(gpu["lse"][1]))

@@ -246,7 +246,9 @@ ETA_DEV void plan_local(const int32_t* counts, int R, int NB, int* row_off, Fuse
 // same grid, and a row's union list is read once its compaction flag carries this
 // launch's token.  Plain (L1-cached) loads still see them, because no SM reads
 // those lines earlier in the launch (the screening reads tau with L2-only loads).
-template <int G, bool DENSE, bool LOCAL, bool FLAGS>
+// PDL_IN (the standalone kernel): the shared-memory and TMEM setup runs before the
+// wait for the previous grid, so it overlaps that grid's tail; the plan is read after.
+template <int G, bool DENSE, bool LOCAL, bool FLAGS, bool PDL_IN = false>
 ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const CUtensorMap* tmV,
                             const CUtensorMap* tmQ, const TcParams& p, const FuseCtx& fx) {
   static_assert(G >= 1 && G <= 8, "G");
@@ -256,10 +258,13 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
   volatile int* abort_flag = &ms->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int Ntot = p.plan[0], chunk = p.plan[1];
-  const int a = blockIdx.x * chunk;
-  if (a >= Ntot) return;  // uniform, before any barrier
-  const int e = min(a + chunk, Ntot);
+  int a = 0, e = 0;
+  if constexpr (!PDL_IN) {
+    const int Ntot = p.plan[0], chunk = p.plan[1];
+    a = blockIdx.x * chunk;
+    if (a >= Ntot) return;  // uniform, before any barrier
+    e = min(a + chunk, Ntot);
+  }
 
   // zero the V halves and the P buffers once: every row the PV MMA reads is then
   // finite (TMA only overwrites them with cache rows, and rows past a sequence's
@@ -298,6 +303,18 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
   tc_fence_after();
   const uint32_t tmem = ms->tmem_base;
   const uint32_t tS0 = tmem, tO0 = tmem + 32;   // column offsets; lane field added per warp
+  if constexpr (PDL_IN) {
+    ETA_PDL_ENTRY();
+    const int Ntot = p.plan[0], chunk = p.plan[1];
+    a = blockIdx.x * chunk;
+    if (a >= Ntot) {   // uniform: no share, release TMEM (nothing was issued) and leave
+      if (warp == NWARP_SM + 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols));
+      return;
+    }
+    e = min(a + chunk, Ntot);
+  }
 
   if (warp == NWARP_SM) {
     // ---------------------------------------------------------------- producer
@@ -604,7 +621,7 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
         float x = sc;
         if constexpr (!DENSE) {
           if (p.invT < 0.f) x = sc >= tau_h[h] ? sc : 0.f;
-          else x = sc * __frcp_rn(1.f + __expf((tau_h[h] - sc) * p.invT));
+          else x = __fdividef(sc, 1.f + __expf((tau_h[h] - sc) * p.invT));   // 0 once exp overflows
         }
         sp[h] = valid ? x : -INFINITY;
         const float wm = warp_max(sp[h]);
@@ -678,11 +695,10 @@ template <int G, bool DENSE>
 __global__ void __launch_bounds__(NT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const TcParams p) {
-  ETA_PDL_ENTRY();
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  decode_tc_body<G, DENSE, false, false>(smem, &tmK, &tmV, &tmQ, p, FuseCtx{});
+  decode_tc_body<G, DENSE, false, false, true>(smem, &tmK, &tmV, &tmQ, p, FuseCtx{});
 }
 
 }  // namespace tc

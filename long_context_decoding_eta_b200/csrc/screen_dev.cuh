@@ -101,13 +101,16 @@ ETA_DEV int screen_group_from(const Src& src, int NB, int NW, int grp, int r, si
   const int lane = threadIdx.x & 31;
   const int j0 = grp * kScreenGroupBlocks + lane * VW;
   const bool vj = j0 < NB;                      // NB % VW == 0: all VW valid or none
-  float acc[VW][G], acc2[VW][VD ? G : 1];
+  // accumulators of blocks (2p, 2p+1) side by side: one packed fp32x2 FMA per pair,
+  // each component an ordinary round-to-nearest fp32 FMA
+  static_assert(VW % 2 == 0, "VW");
+  float2 acc[VW / 2][G], acc2[VW / 2][VD ? G : 1];
 #pragma unroll
-  for (int k = 0; k < VW; ++k) {
+  for (int k = 0; k < VW / 2; ++k) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc[k][h] = 0.f;
+    for (int h = 0; h < G; ++h) acc[k][h] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int h = 0; h < (VD ? G : 1); ++h) acc2[k][h] = 0.f;
+    for (int h = 0; h < (VD ? G : 1); ++h) acc2[k][h] = make_float2(0.f, 0.f);
   }
 #pragma unroll 1
   for (int d0 = 0; d0 < D; d0 += LB) {
@@ -128,7 +131,9 @@ ETA_DEV int screen_group_from(const Src& src, int NB, int NW, int grp, int r, si
       for (int h = 0; h < G; ++h) {
         const float qv = qs[(d0 + u) * G + h];
 #pragma unroll
-        for (int k = 0; k < VW; ++k) acc[k][h] = fmaf(qv, cv[k], acc[k][h]);
+        for (int k = 0; k < VW / 2; ++k)
+          acc[k][h] = __ffma2_rn(make_float2(qv, qv), make_float2(cv[2 * k], cv[2 * k + 1]),
+                                 acc[k][h]);
       }
       if constexpr (VD) {
         const float4 vv = vj ? src.vd(d0 + u) : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -137,7 +142,9 @@ ETA_DEV int screen_group_from(const Src& src, int NB, int NW, int grp, int r, si
         for (int h = 0; h < G; ++h) {
           const float q2 = qs[(d0 + u) * G + h] * qs[(d0 + u) * G + h];
 #pragma unroll
-          for (int k = 0; k < VW; ++k) acc2[k][h] = fmaf(q2, vk[k], acc2[k][h]);
+          for (int k = 0; k < VW / 2; ++k)
+            acc2[k][h] = __ffma2_rn(make_float2(q2, q2), make_float2(vk[2 * k], vk[2 * k + 1]),
+                                    acc2[k][h]);
         }
       }
     }
@@ -167,10 +174,13 @@ ETA_DEV int screen_group_from(const Src& src, int NB, int NW, int grp, int r, si
     float ubv[VW];
 #pragma unroll
     for (int k = 0; k < VW; ++k) {
-      if constexpr (VD)
-        ubv[k] = scale * (acc[k][h] + fminf(qn[h] * rad[k], z * sqrtf(acc2[k][h])));
-      else
-        ubv[k] = scale * fmaf(qn[h], rad[k], acc[k][h]);
+      const float dot = (k & 1) ? acc[k >> 1][h].y : acc[k >> 1][h].x;
+      if constexpr (VD) {
+        const float qv2 = (k & 1) ? acc2[k >> 1][h].y : acc2[k >> 1][h].x;
+        ubv[k] = scale * (dot + fminf(qn[h] * rad[k], z * sqrtf(qv2)));
+      } else {
+        ubv[k] = scale * fmaf(qn[h], rad[k], dot);
+      }
       if (vj && n[k] > 0 && j0 + k < nvalid && ubv[k] >= ts[h]) bits |= 1u << k;
     }
     if (bounds_out && vj)

@@ -39,7 +39,6 @@ METRIC = "decode attn steps/s and HBM GB/s on admitted KV bytes (% of B200 peak)
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0
 PROLOGUE_LAUNCHES = 1   # tail-block metadata + tau in one launch (2 when separate)
-DECODE_LAUNCHES = 3     # plan, split-KV decode, combine
 LAUNCHES_PER_FUSED_STEP = 1   # eta_decode_step: one persistent kernel
 
 
@@ -361,7 +360,8 @@ def run_eta(args, rank, world, device):
                            "total": by["step"], "dense_kv": by["dense_kv"]},
         "roofline": {"kernel": ("eta_decode_step (one persistent kernel: tail metadata, tau, "
                                 "screen, decode, merge)") if fused else
-                               "eta_decode (plan + split-KV decode + combine)", "bound": "hbm",
+                               "eta_decode (split-KV decode with its share plan + combine)",
+                     "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
                      "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
@@ -382,7 +382,8 @@ def run_eta(args, rank, world, device):
                 "d2h_bytes_per_step": o_host.numel() * 4 + lse_host.numel() * 4},
         "gpu_launches": (LAUNCHES_PER_FUSED_STEP if fused else
                          PROLOGUE_LAUNCHES + (1 if args.separate_prologue else 0) +
-                         _lib.eta_screen_launches(dec.dims, args.cent) + DECODE_LAUNCHES)
+                         _lib.eta_screen_launches(dec.dims, args.cent) +
+                         _lib.eta_decode_launches(dec.dims))
                         * args.steps,
         "clocks": clk.summary(),
     }

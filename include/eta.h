@@ -205,6 +205,10 @@ eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float
  * current device).  dev_status bits: TIMEOUT, NONFINITE_Q, BAD_BLOCK, BAD_LENGTH.
  */
 size_t eta_decode_workspace_size(const eta_dims_t* dims);
+/* Kernel launches eta_decode makes for these dims with the current engine: 2 (the
+ * tensor-core decode lays out its CTA shares itself, then the combine: 128 to 2048
+ * (row, KV head) pairs) or 3 (plan, decode, combine); -1 for invalid dims. */
+int32_t eta_decode_launches(const eta_dims_t* dims);
 eta_status_t eta_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                         const eta_bf16_t* K, const eta_bf16_t* V, const int32_t* lengths,
                         const int32_t* union_idx, const int32_t* union_cnt, float T,

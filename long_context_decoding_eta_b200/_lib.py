@@ -32,7 +32,7 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_set_decode_engine", "eta_get_decode_engine", "eta_decode_static",
            "eta_decode_static_max_workspace", "eta_selftest_wait_timeout", "eta_prefill",
            "eta_decode_step_workspace_size", "eta_decode_step", "eta_lse_merge",
-           "eta_append_and_predict_tau", "eta_screen_launches")
+           "eta_append_and_predict_tau", "eta_screen_launches", "eta_decode_launches")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 
 
@@ -77,6 +77,8 @@ def lib() -> C.CDLL:
     L.eta_screen_workspace_size.restype = C.c_size_t
     L.eta_screen_launches.argtypes = [DIMS, I32]
     L.eta_screen_launches.restype = I32
+    L.eta_decode_launches.argtypes = [DIMS]
+    L.eta_decode_launches.restype = I32
     L.eta_screen.argtypes = [DIMS, P, P, I32, P, P, P, P, P, I32, F32, F32, P, P, P, P, P, P,
                              C.c_size_t, P, P]
     L.eta_decode_workspace_size.argtypes = [DIMS]
@@ -163,6 +165,13 @@ def eta_append_and_predict_tau(dims: Dims, K, V, lengths, cent, rmax, var, cnt, 
 
 def eta_screen_workspace_size(dims: Dims) -> int:
     return int(lib().eta_screen_workspace_size(C.byref(dims)))
+
+
+def eta_decode_launches(dims: Dims) -> int:
+    n = int(lib().eta_decode_launches(C.byref(dims)))
+    if n < 0:
+        raise EtaError("eta_decode_launches", 1)
+    return n
 
 
 def eta_screen_launches(dims: Dims, cent_format: str = "f32") -> int:

@@ -170,6 +170,13 @@ struct TcParams {
   float* part_o;
   float* part_ml;
   int32_t* status;
+  // plan in the kernel (standalone decode): the R per-pair admitted counts it is laid
+  // out from, and where CTA 0 publishes row_off[0..R] and {total, share} for the
+  // combine launch that follows
+  int R;
+  const int32_t* counts;
+  int32_t* row_off_g;
+  int32_t* plan_g;
 };
 
 // In-kernel merge of the fused step: the CTA that writes the last partial slot of
@@ -248,19 +255,26 @@ ETA_DEV void plan_local(const int32_t* counts, int R, int NB, int* row_off, Fuse
 // those lines earlier in the launch (the screening reads tau with L2-only loads).
 // PDL_IN (the standalone kernel): the shared-memory and TMEM setup runs before the
 // wait for the previous grid, so it overlaps that grid's tail; the plan is read after.
-template <int G, bool DENSE, bool LOCAL, bool FLAGS, bool PDL_IN = false>
+// PLAN_IN (with PDL_IN, sparse): no plan launch; every CTA lays the shares out itself
+// (plan_local, from the admitted counts) and CTA 0 publishes row_off and the plan
+// for the combine launch.
+template <int G, bool DENSE, bool LOCAL, bool FLAGS, bool PDL_IN = false, bool PLAN_IN = false>
 ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const CUtensorMap* tmV,
                             const CUtensorMap* tmQ, const TcParams& p, const FuseCtx& fx) {
   static_assert(G >= 1 && G <= 8, "G");
   static_assert(!(LOCAL && DENSE), "the in-kernel merge is for the sparse decode");
   static_assert(!FLAGS || LOCAL, "flags come with the local plan");
+  static_assert(!PLAN_IN || (PDL_IN && !DENSE && !LOCAL), "plan in the standalone sparse decode");
   TcMisc* ms = reinterpret_cast<TcMisc*>(smem + SM_MISC);
+  const int32_t* plan = p.plan;
+  const int32_t* row_off = p.row_off;
+  const int32_t* cta_row = p.cta_row;
   volatile int* abort_flag = &ms->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   int a = 0, e = 0;
   if constexpr (!PDL_IN) {
-    const int Ntot = p.plan[0], chunk = p.plan[1];
+    const int Ntot = plan[0], chunk = plan[1];
     a = blockIdx.x * chunk;
     if (a >= Ntot) return;  // uniform, before any barrier
     e = min(a + chunk, Ntot);
@@ -305,7 +319,22 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
   const uint32_t tS0 = tmem, tO0 = tmem + 32;   // column offsets; lane field added per warp
   if constexpr (PDL_IN) {
     ETA_PDL_ENTRY();
-    const int Ntot = p.plan[0], chunk = p.plan[1];
+    if constexpr (PLAN_IN) {
+      FuseSmem* fs = reinterpret_cast<FuseSmem*>(smem + SM_FUSE);
+      int* ro = reinterpret_cast<int*>(smem + SM_ROWOFF);
+      plan_local(p.counts, p.R, p.NB, ro, fs, p.status);
+      if (blockIdx.x == 0) {
+        for (int r = threadIdx.x; r <= p.R; r += NT) p.row_off_g[r] = ro[r];
+        if (threadIdx.x == 0) {
+          p.plan_g[0] = fs->plan[0];
+          p.plan_g[1] = fs->plan[1];
+        }
+      }
+      plan = fs->plan;
+      row_off = ro;
+      cta_row = &fs->cta_row;
+    }
+    const int Ntot = plan[0], chunk = plan[1];
     a = blockIdx.x * chunk;
     if (a >= Ntot) {   // uniform: no share, release TMEM (nothing was issued) and leave
       if (warp == NWARP_SM + 1)
@@ -319,8 +348,8 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
   if (warp == NWARP_SM) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      int r = LOCAL ? p.cta_row[0] : p.cta_row[blockIdx.x];
-      int roff = p.row_off[r], rend = p.row_off[r + 1];
+      int r = (LOCAL || PLAN_IN) ? cta_row[0] : cta_row[blockIdx.x];
+      int roff = row_off[r], rend = row_off[r + 1];
       int it = 0;
       bool ok = true;
       int pend_row = -1, pend_t0 = 0, pend_nv = 0;   // a lone sub-tile waiting for a partner
@@ -375,7 +404,7 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
         while (pos >= re) {
           ++rr;
           ro = re;
-          re = p.row_off[rr + 1];
+          re = row_off[rr + 1];
         }
         if (DENSE) return pos - ro;
         if (!row_ready(rr)) {
@@ -516,8 +545,8 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
       named_bar_sync(1, NWARP_SM * 32);
       int p0 = 0, ns = 0;
       if constexpr (LOCAL) {
-        const int off = p.row_off[row], c = p.row_off[row + 1] - off;
-        const int chunk = p.plan[1];
+        const int off = row_off[row], c = row_off[row + 1] - off;
+        const int chunk = plan[1];
         p0 = off / chunk;
         ns = (off + c - 1) / chunk - p0 + 1;
       }
@@ -691,14 +720,14 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
   }
 }
 
-template <int G, bool DENSE>
+template <int G, bool DENSE, bool PLAN_IN = false>
 __global__ void __launch_bounds__(NT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const TcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  decode_tc_body<G, DENSE, false, false, true>(smem, &tmK, &tmV, &tmQ, p, FuseCtx{});
+  decode_tc_body<G, DENSE, false, false, true, PLAN_IN>(smem, &tmK, &tmV, &tmQ, p, FuseCtx{});
 }
 
 }  // namespace tc

@@ -91,6 +91,8 @@ def test_argument_validation_without_gpu():
     # launch-count query: invalid dims are refused; without a device the two-launch form
     assert lib.eta_screen_launches(ctypes.byref(bad), 1) == -1
     assert lib.eta_screen_launches(ctypes.byref(dims), 1) in (1, 2)
+    assert lib.eta_decode_launches(ctypes.byref(bad)) == -1
+    assert lib.eta_decode_launches(ctypes.byref(dims)) in (2, 3)
 
 
 def test_engine_selection_host_only():

@@ -94,7 +94,14 @@ def test_long_128k_b64_union16(engine, cent):
     w = synth.LONG128K
     from long_context_decoding_eta_b200 import _lib as L
     # 16 groups of 128 blocks per row: the two-launch screen (screening, compaction)
-    assert L.eta_screen_launches(L.Dims.of(w.B, w.Hq, w.Hkv, w.d, w.blk, w.T_max), cent) == 2
+    dims = L.Dims.of(w.B, w.Hq, w.Hkv, w.d, w.blk, w.T_max)
+    assert L.eta_screen_launches(dims, cent) == 2
+    # the tensor-core decode lays out its shares itself: decode + combine
+    L.eta_set_decode_engine(engine)
+    try:
+        assert L.eta_decode_launches(dims) == (2 if engine != "fma" else 3)
+    finally:
+        L.eta_set_decode_engine("auto")
     rep, dens = run_fullsize(w, rows=[0, 37, 63], engine=engine, cent_format=cent)
     # the density target is set on the 3 sampled rows only; across the batch it
     # varies with the rows' thresholds: require real pruning and real admission

@@ -94,18 +94,22 @@ def test_ragged_lengths_empty_and_single_token_rows():
         assert np.all(gpu["o"][1] == 0) and np.all(np.isneginf(gpu["lse"][1]))
 
 
-@pytest.mark.parametrize("B,Hkv", [(8, 4), (11, 3), (1, 1)])
-def test_batch_shapes_and_repeat_determinism(B, Hkv):
-    """Batches of 32, 33 and 1 (batch row, KV head) pairs, with empty, single-token,
+@pytest.mark.parametrize("B,Hkv", [(8, 4), (11, 3), (1, 1), (32, 4)])
+def test_batch_shapes_and_repeat_determinism(B, Hkv, engine):
+    """Batches of 32, 33, 1 and 128 (batch row, KV head) pairs, with empty, single-token,
     single-block and ragged rows, against the oracle; repeated steps on one decoder
     are bit-identical (the split plan and the combine order depend only on the
     admitted counts)."""
     w = synth.MID.with_(B=B, Hkv=Hkv, Hq=4 * Hkv, ctx=4096, needles=2, seed=90 + B)
-    lens = [4096, 0, 64, 4031, 1, 3000, 128, 2049, 4096, 777, 3333][:B]
+    lens = ([4096, 0, 64, 4031, 1, 3000, 128, 2049, 4096, 777, 3333] * 3)[:B]
     lengths = torch.tensor(lens, dtype=torch.int32)
     from long_context_decoding_eta_b200 import _lib as L
+    dims = L.Dims.of(B, w.Hq, w.Hkv, w.d, w.blk, w.T_max)
     # these small batches take the one-launch screen (screening + compaction)
-    assert L.eta_screen_launches(L.Dims.of(B, w.Hq, w.Hkv, w.d, w.blk, w.T_max), "f32") == 1
+    assert L.eta_screen_launches(dims, "f32") == 1
+    # 128 pairs and more: the tensor-core decode plans its own shares
+    if engine == "tcgen05":
+        assert L.eta_decode_launches(dims) == (2 if B * Hkv >= 128 else 3)
     rep, gpu, sc = full_parity(w, lengths=lengths, density=0.4)
     if B > 1:
         assert np.all(gpu["o"][1] == 0) and np.all(np.isneginf(gpu["lse"][1]))

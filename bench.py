@@ -384,11 +384,12 @@ def run_eta(args, rank, world, device):
         "e2e": {"value": job_throughput(world, 1, e2e_ms), "unit": "steps/s",
                 "h2d_bytes_per_step": q_host.numel() * 2,
                 "d2h_bytes_per_step": o_host.numel() * 4 + lse_host.numel() * 4},
+        # all ranks' launches in the timed region (each rank runs the same steps)
         "gpu_launches": (LAUNCHES_PER_FUSED_STEP if fused else
                          PROLOGUE_LAUNCHES + (1 if args.separate_prologue else 0) +
                          _lib.eta_screen_launches(dec.dims, args.cent) +
                          _lib.eta_decode_launches(dec.dims))
-                        * args.steps,
+                        * args.steps * world,
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -550,7 +551,7 @@ def run_prefill(args, rank, world, device):
             "roofline": {"kernel": "prefill_tc_kernel", "bound": "tensor", "achieved": tf,
                          "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
                          "peak_kind": "measured cuBLAS bf16 burst"},
-            "gpu_launches": args.steps, "clocks": clk.summary()}
+            "gpu_launches": args.steps * world, "clocks": clk.summary()}
 
 
 def main():

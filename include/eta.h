@@ -152,6 +152,8 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  * head) pair: batches of at most two CTAs per SM whose rows fit two rounds of the
  * CTA's group buffers, NB a multiple of 8 for bf16 centroids or 4 for fp32) or two
  * (screening, then compaction); eta_screen_launches says which.
+ * dev_status (may be NULL): ETA_DEVSTAT_TIMEOUT if the one-launch form's bounded wait
+ * for a staged group tile ran out (the outputs are then incomplete).
  */
 /*
  * eta_append_and_predict_tau -- eta_build_block_meta(..., ETA_TAIL_BLOCK, ...) and

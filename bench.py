@@ -25,6 +25,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -38,6 +39,8 @@ from long_context_decoding_eta_b200 import synth  # noqa: E402
 METRIC = "decode attn steps/s and HBM GB/s on admitted KV bytes (% of B200 peak)"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 1000 * 1000
+# where the nvidia-smi clock samples of the timed region go (--clock-log-dir)
+CLOCK_LOG_DIR = tempfile.gettempdir()
 NOMINAL_HBM_GBS = 8000.0
 PROLOGUE_LAUNCHES = 1   # tail-block metadata + tau in one launch (2 when separate)
 LAUNCHES_PER_FUSED_STEP = 1   # eta_decode_step: one persistent kernel
@@ -121,9 +124,10 @@ class Clocks:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = os.path.join(CLOCK_LOG_DIR, f"eta_bench_clocks_rank{index}.csv")
 
     def __enter__(self):
+        self.fh = None
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
@@ -133,6 +137,8 @@ class Clocks:
                                          stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            if self.fh is not None:
+                self.fh.close()
         return self
 
     def __exit__(self, *a):
@@ -555,6 +561,7 @@ def run_prefill(args, rank, world, device):
 
 
 def main():
+    global CLOCK_LOG_DIR
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -568,6 +575,8 @@ def main():
     ap.add_argument("--pf-gate-T", type=float, default=0.0)
     ap.add_argument("--cpu-rows", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log-dir", default="",
+                    help="keep the raw clock samples (CSV per rank) in this folder")
     ap.add_argument("--clock-soak-s", type=float, default=1.0,
                     help="untimed steps run under the clock sampler before the timed region")
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
@@ -582,6 +591,8 @@ def main():
     ap.add_argument("--cent", default="bf16", choices=["f32", "bf16"],
                     help="storage of the block centroids the screen reads")
     args = ap.parse_args()
+    if args.clock_log_dir:
+        CLOCK_LOG_DIR = args.clock_log_dir
     if args.warmup < 3:
         args.warmup = 3
 

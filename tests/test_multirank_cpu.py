@@ -130,3 +130,14 @@ def test_shard_range_and_lengths():
         assert torch.equal(tot, lens.to(torch.int64))
     with pytest.raises(ValueError):
         shard_range(100, 64, 2, 0)
+
+
+def test_clock_sampler_without_nvidia_smi_reports_unavailable(tmp_path, monkeypatch):
+    """On a host without nvidia-smi the sampler records nothing and says so."""
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setattr(bench, "CLOCK_LOG_DIR", str(tmp_path))
+    monkeypatch.setenv("PATH", str(tmp_path))          # no nvidia-smi on this PATH
+    with bench.Clocks(0) as clk:
+        pass
+    assert clk.summary()["reasons"] == ["unavailable"]

@@ -3,13 +3,15 @@
 // evolve.pub review, Methodology Assessment Eq. 2-3: m = sigmoid(beta (S - tau)),
 // gated logits S * m; review FAQ: a sub-threshold logit goes to 0, weight e^0 = 1).
 //
-// Pipeline per step (three launches on one stream):
+// Pipeline per step (three launches on one stream; two when the tensor-core decode
+// plans its own shares, at 128 to 2048 pairs):
 //   plan_kernel    prefix sum of admitted blocks over (row, KV head) pairs, and the
 //                  first pair of every CTA's share.  The admitted blocks of all pairs,
 //                  laid end to end, are cut into equal contiguous shares, one per CTA
 //                  (persistent grid = SM count), so every SM streams the same bytes
 //                  whatever the per-pair density.
-//   decode_kernel  one producer warp issues 1-D TMA bulk copies (cp.async.bulk) of
+//   decode         decode_tc_kernel (tcgen05 engine, d = 128: decode_tc.cuh) or
+//   decode_kernel  (this file, the CUDA-core engine): one producer warp issues 1-D TMA bulk copies (cp.async.bulk) of
 //                  64-key K and V tiles into a ring of shared-memory stages guarded by
 //                  mbarriers; NCW consumer warps compute, for the G query heads of the
 //                  group, q.k on CUDA cores (lane = d/32 dims, transposed butterfly

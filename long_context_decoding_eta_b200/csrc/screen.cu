@@ -4,13 +4,18 @@
 // coarse GPU block selection"; evolve.pub review FAQ: blocks whose best possible
 // score falls below the threshold are skipped entirely).
 //
-// screen_kernel: lane = block.  Centroids are stored dimension-major per (row, KV
-//   head), so each of the d loads of a warp is one 128-byte line covering 32
+// screen_vec_kernel (the default when NB % 4 == 0 and the metadata is 16-byte
+//   aligned): a warp screens 128 consecutive blocks, lane = 4 blocks, through
+//   screen_group_from (screen_dev.cuh), the arithmetic the fused step shares.
+// screen_kernel (otherwise): lane = block.  Centroids are stored dimension-major per
+//   (row, KV head), so each of the d loads of a warp is one 128-byte line covering 32
 //   consecutive blocks; the G query heads of the group sit in shared memory as
 //   [d][G] fp32 and are read as broadcasts.  One ballot per head gives the
 //   head's 32-bit admit word directly; the union word is their OR.
 // compact_kernel: one CTA per (row, KV head) turns union words into the ascending
 //   list of admitted block indices (popcount prefix over words, lane = bit).
+// screen_row_kernel (small batches): screening from TMA-staged group tiles and the
+//   compaction of its row in one launch.
 #include <type_traits>
 
 #include "eta_common.cuh"

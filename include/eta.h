@@ -176,7 +176,8 @@ eta_status_t eta_append_and_predict_tau(const eta_dims_t* dims, const eta_bf16_t
 size_t eta_screen_workspace_size(const eta_dims_t* dims);
 /* Kernel launches eta_screen makes on the current device for these dims and centroid
  * format when every pointer argument is 16-byte aligned (1 or 2; 2 without a
- * device), or -1 for invalid dims. */
+ * device), or -1 for invalid dims.  A packaging query with no counterpart in the
+ * pages; host only, launches nothing. */
 int32_t eta_screen_launches(const eta_dims_t* dims, eta_cent_format_t cent_format);
 eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                         eta_cent_format_t cent_format, const void* cent, const float* rmax,
@@ -209,7 +210,8 @@ eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float
 size_t eta_decode_workspace_size(const eta_dims_t* dims);
 /* Kernel launches eta_decode makes for these dims with the current engine: 2 (the
  * tensor-core decode lays out its CTA shares itself, then the combine: 128 to 2048
- * (row, KV head) pairs) or 3 (plan, decode, combine); -1 for invalid dims. */
+ * (row, KV head) pairs) or 3 (plan, decode, combine); -1 for invalid dims.  A
+ * packaging query with no counterpart in the pages; host only, launches nothing. */
 int32_t eta_decode_launches(const eta_dims_t* dims);
 eta_status_t eta_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                         const eta_bf16_t* K, const eta_bf16_t* V, const int32_t* lengths,

@@ -54,6 +54,22 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def with_overrides(w: synth.Workload, args) -> synth.Workload:
+    """The workload with the operating point asked for on the command line (the
+    density sweep and the threshold mode of the long-context configurations)."""
+    kw = {}
+    if getattr(args, "density", None):
+        kw["density"] = float(args.density)
+    if getattr(args, "density_kind", None):
+        kw["density_kind"] = args.density_kind
+    if getattr(args, "tau_mode", None):
+        kw["tau_mode"] = args.tau_mode
+    if not kw:
+        return w
+    tag = "-".join(f"{k}{v}" for k, v in sorted(kw.items()))
+    return w.with_(name=f"{w.name}-{tag}", **kw)
+
+
 def workload_by_name(name: str, B: int = 0) -> synth.Workload:
     for w in synth.WORKLOADS.values():
         if w.name == name or w.name.startswith(name):
@@ -226,7 +242,7 @@ def step_bytes(dec, w):
 def run_eta(args, rank, world, device):
     from long_context_decoding_eta_b200 import _lib
     _lib.eta_set_decode_engine(args.engine)
-    w = workload_by_name(args.workload, args.B)
+    w = with_overrides(workload_by_name(args.workload, args.B), args)
     fused = bool(args.fused)
     g, dec, W, bias, tau_const = setup(w, device, rank, args.cent, fused,
                                        not args.separate_prologue)
@@ -455,7 +471,7 @@ def run_reference(args, rank, world, device):
     The threshold bias is set by the oracle itself on the sampled rows, with the
     same density rule as the eta arm; no CUDA kernel of this package runs."""
     from oracle import eta_oracle as O
-    w = workload_by_name(args.workload, args.B)
+    w = with_overrides(workload_by_name(args.workload, args.B), args)
     g = synth.generate(w, device, seed=w.seed)
     rows = list(range(max(1, min(args.cpu_rows, w.B))))
     K64 = g["K"][rows].double().cpu().numpy()
@@ -575,6 +591,12 @@ def main():
     ap.add_argument("--pf-gate-T", type=float, default=0.0)
     ap.add_argument("--cpu-rows", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--density", type=float, default=0.0,
+                    help="override the workload's density target (e.g. 0.38)")
+    ap.add_argument("--density-kind", default="", choices=["", "head", "union"],
+                    help="override what the density target counts: per head or union")
+    ap.add_argument("--tau-mode", default="", choices=["", "predictor", "const"],
+                    help="override the threshold mode (the calibrated workload's comparison)")
     ap.add_argument("--clock-log-dir", default="",
                     help="keep the raw clock samples (CSV per rank) in this folder")
     ap.add_argument("--clock-soak-s", type=float, default=1.0,

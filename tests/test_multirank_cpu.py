@@ -141,3 +141,19 @@ def test_clock_sampler_without_nvidia_smi_reports_unavailable(tmp_path, monkeypa
     with bench.Clocks(0) as clk:
         pass
     assert clk.summary()["reasons"] == ["unavailable"]
+
+
+def test_operating_point_overrides():
+    """--density / --density-kind / --tau-mode change only what they name, and the
+    default run keeps the workload as defined."""
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+    base = bench.workload_by_name("long")
+    none = types.SimpleNamespace(density=0.0, density_kind="", tau_mode="")
+    assert bench.with_overrides(base, none) is base
+    pt = types.SimpleNamespace(density=0.38, density_kind="head", tau_mode="")
+    w = bench.with_overrides(base, pt)
+    assert (w.density, w.density_kind, w.tau_mode) == (0.38, "head", base.tau_mode)
+    assert (w.B, w.ctx, w.blk, w.seed) == (base.B, base.ctx, base.blk, base.seed)
+    assert w.name != base.name

@@ -30,12 +30,15 @@ union semantics, pruned-block semantics, tie-breaks); each function says which.
 Everything is float64.  bf16 inputs are passed in already widened (exactly).
 Pure numpy; no blocking, fusion or reordering beyond the definitions.
 
-Parity unpinned: the two probabilistic bounds of block_bounds (BOUND_PROB,
-BOUND_PROB_DIM).  The pages name a "probabilistic" bound from cached variance
-but print no formula; the tests pin only the properties the reading implies
-(never looser than the exact bound, equal to it as z grows, the closed forms of
-the variance terms), not the formula itself.  Every other function is pinned
-by closed forms, brute force or library routines in tests/test_oracle_pins.py.
+The two probabilistic bounds of block_bounds (BOUND_PROB, BOUND_PROB_DIM) are
+readings: the pages name a "probabilistic" bound from cached variance but print
+no formula.  Each is pinned to the property that defines a z-sigma bound: on
+blocks of keys with Gaussian deviations from their centre (isotropic for the
+scalar form, one spread per dimension for the per-dimension form) the fraction
+of keys scoring above the bound is the one-sided normal tail 1 - Phi(z), within
+a binomial tolerance; besides, neither is ever looser than the exact bound, and
+both equal it as z grows.  Every function is pinned by closed forms, brute
+force, library routines or those statistics in tests/test_oracle_pins.py.
 """
 from __future__ import annotations
 
@@ -160,7 +163,8 @@ def block_bounds(q_h: np.ndarray, cent: np.ndarray, rmax: np.ndarray, var: np.nd
     prob  (variance):        scale * (q.c + ||q|| * min(rmax, z * sqrt(var / d)))
     prob_dim (per-dimension variance, vardim [NB, d]):
                              scale * (q.c + min(||q|| * rmax, z * sqrt(sum_i q_i^2 vardim_i)))
-    The two probabilistic forms are readings (parity unpinned, see the module note).
+    The two probabilistic forms are readings of a z-sigma bound (see the module
+    note): for Gaussian key deviations a fraction 1 - Phi(z) of keys exceeds them.
     """
     d = q_h.shape[0]
     qc = cent @ q_h

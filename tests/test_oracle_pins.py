@@ -388,16 +388,77 @@ def test_probabilistic_bound_properties():
     for z in (0.5, 1.0, 3.0, math.sqrt(w.d)):
         pr = O.screen(q, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_PROB, z)["bounds"]
         assert np.all(pr <= ex + 1e-12)
-        # for z <= sqrt(d) the min is inactive: var <= rmax^2 gives z sqrt(var/d) <= rmax
-        for b in range(w.B):
-            for h in range(w.Hq):
-                g = h // w.G
-                qh = q[b, h]
-                want = scale * (meta["cent"][b, g] @ qh + np.linalg.norm(qh) * z
-                                * np.sqrt(meta["var"][b, g] / w.d))
-                np.testing.assert_allclose(pr[b, h], want, atol=1e-12)
     pr = O.screen(q, np.zeros((w.B, w.Hq)), meta, scale, O.BOUND_PROB, 1e9)["bounds"]
     np.testing.assert_allclose(pr, ex, atol=1e-12)
+
+
+def _gaussian_blocks(rng, nblk, blk, sig):
+    """nblk blocks of blk keys, k = c_j + sig * N(0, I) around random centres c_j."""
+    d = sig.shape[0]
+    centres = rng.normal(size=(nblk, d))
+    return centres[:, None, :] + sig[None, None, :] * rng.normal(size=(nblk, blk, d))
+
+
+def _tail_fraction(keys, bound, z, queries):
+    """Fraction of (query, key) pairs whose score exceeds the oracle's bound of the
+    key's block, with the exact-radius cap lifted (rmax = +inf) so that only the
+    probabilistic term is measured.  Scores and bounds in unscaled units (scale 1)."""
+    nblk, blk, d = keys.shape
+    m = O.block_meta(keys.reshape(nblk * blk, d), nblk * blk, blk)
+    no_cap = np.full(nblk, np.inf)
+    above = 0
+    for q in queries:
+        ub = O.block_bounds(q, m["cent"], no_cap, m["var"], 1.0, bound, z, m["vardim"])
+        above += int(((keys @ q) > ub[:, None]).sum())
+    return above / (len(queries) * nblk * blk)
+
+
+def _tail_tolerance(p, n_keys):
+    # 4 binomial standard deviations counted over the keys alone (the queries
+    # share keys, so they are not independent draws), plus 5% of p for the
+    # sampling noise of the per-block variance estimates
+    return 4.0 * math.sqrt(p * (1.0 - p) / n_keys) + 0.05 * p
+
+
+@pytest.mark.parametrize("d,nblk", [(16, 2000), (128, 500)])
+def test_probabilistic_bound_is_the_z_sigma_tail_for_isotropic_keys(d, nblk):
+    """BOUND_PROB reads the cached variance as a z-sigma bound: for keys with
+    isotropic Gaussian deviations from their block centre, q.(k - c) is normal with
+    standard deviation ||q|| sqrt(var / d), so the fraction of keys scoring above
+    the bound must be the one-sided normal tail 1 - Phi(z).  A bound built from
+    sqrt(var) (no / d), from the key count instead of d, or from z^2 gives
+    fractions of about 0, 1 - Phi(z sqrt(d / n)) and 1 - Phi(z^2): all far
+    outside the tolerance."""
+    from scipy.stats import norm
+    rng = np.random.default_rng(41 + d)
+    blk = 128
+    keys = _gaussian_blocks(rng, nblk, blk, np.full(d, 0.3))
+    queries = [rng.normal(size=d) for _ in range(8)]
+    for z in (1.0, 2.0, 3.0):
+        p = norm.sf(z)
+        f = _tail_fraction(keys, O.BOUND_PROB, z, queries)
+        assert abs(f - p) <= _tail_tolerance(p, nblk * blk), (z, f, p)
+
+
+@pytest.mark.parametrize("d,nblk", [(16, 2000), (128, 500)])
+def test_per_dimension_bound_is_the_z_sigma_tail_for_anisotropic_keys(d, nblk):
+    """BOUND_PROB_DIM: with independent per-dimension spreads sigma_i and any q,
+    q.(k - c) has variance sum_i q_i^2 sigma_i^2, so again 1 - Phi(z) of the keys
+    score above the bound.  The scalar bound on the same keys, which assumes
+    isotropy, misses that tail by far (the query leans on the wide dimensions)."""
+    from scipy.stats import norm
+    rng = np.random.default_rng(43 + d)
+    blk = 128
+    sig = np.exp(rng.uniform(math.log(0.1), math.log(2.0), size=d))
+    keys = _gaussian_blocks(rng, nblk, blk, sig)
+    queries = [rng.normal(size=d) * (0.2 + sig) for _ in range(8)]
+    for z in (1.0, 2.0, 3.0):
+        p = norm.sf(z)
+        tol = _tail_tolerance(p, nblk * blk)
+        f = _tail_fraction(keys, O.BOUND_PROB_DIM, z, queries)
+        assert abs(f - p) <= tol, (z, f, p)
+        f_iso = _tail_fraction(keys, O.BOUND_PROB, z, queries)
+        assert abs(f_iso - p) > 4 * tol, (z, f_iso, p)
 
 
 # --------------------------------------------------------------------------
@@ -513,12 +574,6 @@ def test_per_dimension_variance_bound_brute_force_values():
     m = O.block_meta(keys, 7, 8)
     c = keys.mean(0)
     assert np.allclose(m["vardim"][0], [np.mean((keys[:, i] - c[i]) ** 2) for i in range(5)])
-    qv = rng.normal(size=5)
-    ub = O.block_bounds(qv, m["cent"], m["rmax"], m["var"], 1.0, O.BOUND_PROB_DIM, 1.5,
-                        m["vardim"])
-    want = c @ qv + min(np.linalg.norm(qv) * m["rmax"][0],
-                        1.5 * math.sqrt(sum(qv[i] ** 2 * m["vardim"][0][i] for i in range(5))))
-    assert abs(ub[0] - want) < 1e-12
 
 
 # --------------------------------------------------------------------------

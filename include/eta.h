@@ -15,7 +15,8 @@
  * Conventions (all entry points):
  *  - Every tensor argument is a caller-owned DEVICE pointer unless said otherwise.
  *    The library never allocates, frees or retains memory.  Scratch comes from a
- *    caller-provided workspace whose size the *_workspace_size query returns.
+ *    caller-provided workspace whose size the *_workspace_size query returns (the
+ *    one exception, eta_decode_static, uses a fixed array reserved at load time).
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
  *    legacy default stream) and never synchronize the host.
  *  - Host-side argument errors are returned immediately as ETA_ERR_* and nothing is
@@ -233,11 +234,14 @@ eta_status_t eta_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float
  * 4 MiB until the process exits.  It calls no cudaMalloc, cudaFree or other
  * allocating routine.
  *  - Limit: returns ETA_ERR_WORKSPACE when eta_decode_workspace_size(dims) would
- *    exceed eta_decode_static_max_workspace() (4 MiB; enough for B * Hkv up to
- *    about 900 pairs at G = 4, d = 128 on a 148-SM GPU).
- *  - Set-up: the first call made on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current).  Make that first call
- *    before any stream capture.
+ *    exceed eta_decode_static_max_workspace() (4 MiB).  On a 148-SM GPU with
+ *    d = 128 that admits B * Hkv up to 1864 (row, KV head) pairs at G = 4 and 859
+ *    at G = 8 (the per-CTA and per-pair partial results dominate the scratch).
+ *  - Set-up: the first call made in a device's context looks up the array's device
+ *    address (cudaGetSymbolAddress, with that device current).  Make that first
+ *    call before any stream capture.  A device reset (or any re-creation of the
+ *    context) makes the next call look the address up again, so that first call
+ *    after a reset should also come before any capture.
  *  - All calls share the one array and it keeps the last call's contents; nothing
  *    in it needs to start at zero.  Calls that overlap on the GPU (other streams,
  *    other host threads) race on it: serialize them.

@@ -24,6 +24,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "combine_dev.cuh"
 #include "decode_tc.cuh"
@@ -714,20 +715,33 @@ namespace eta {
 constexpr size_t kStaticScratchBytes = size_t(4) << 20;   // 4 MiB
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-// Device address of g_static_scratch per device, looked up once per device (with
-// that device current) on the first call made on it.
+// Device address of g_static_scratch, looked up with cudaGetSymbolAddress (the
+// array's name is only a host-side stand-in in host code) on the first call made in
+// a device's context, with that device current, and cached per device together with
+// the id of the context it belongs to.  A call in a new context (after a device
+// reset) looks the address up again: the module, and the array with it, may then sit
+// elsewhere.
 constexpr int kMaxDevices = 64;
-static std::atomic<void*> g_static_scratch_ptr[kMaxDevices];
+struct StaticScratchSlot {
+  unsigned long long ctx = 0;
+  void* ptr = nullptr;
+};
+static StaticScratchSlot g_static_scratch_slot[kMaxDevices];
+static std::mutex g_static_scratch_mu;
 
 inline eta_status_t static_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ETA_ERR_CUDA;
-  void* ptr = g_static_scratch_ptr[dev].load();
-  if (!ptr) {
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  StaticScratchSlot& slot = g_static_scratch_slot[dev];
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0 || slot.ctx != ctx || !slot.ptr) {
+    void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return ETA_ERR_CUDA;
-    g_static_scratch_ptr[dev].store(ptr);
+    slot.ptr = ptr;
+    slot.ctx = ctx != 0 ? ctx : current_context_id();
   }
-  *out = ptr;
+  *out = slot.ptr;
   return ETA_OK;
 }
 

@@ -2,9 +2,11 @@
 // properties, launch-error mapping.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "../../include/eta.h"
@@ -54,18 +56,51 @@ inline eta_status_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size
              : ETA_ERR_CUDA;
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device (so that calls made
-// during stream capture issue no attribute change).  One flag set per kernel.
+// Unique identifier of the CUDA context current on the calling thread, or 0 when
+// none is current (or the driver cannot say).  Per-device caches key on it rather
+// than on the device ordinal: after cudaDeviceReset, or any destruction and
+// re-creation of the primary context, the library's module is loaded again, so
+// symbol addresses and function attributes cached for the old context are stale.
+inline unsigned long long current_context_id() {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static const std::pair<GetCurrentFn, GetIdFn> fns = [] {
+    void* cur = nullptr;
+    void* gid = nullptr;
+    cudaDriverEntryPointQueryResult q1, q2;
+    const bool ok =
+        cudaGetDriverEntryPoint("cuCtxGetCurrent", &cur, cudaEnableDefault, &q1) ==
+            cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &gid, cudaEnableDefault, &q2) == cudaSuccess &&
+        q2 == cudaDriverEntryPointSuccess;
+    return ok ? std::make_pair(reinterpret_cast<GetCurrentFn>(cur),
+                               reinterpret_cast<GetIdFn>(gid))
+              : std::make_pair(GetCurrentFn(nullptr), GetIdFn(nullptr));
+  }();
+  if (!fns.first || !fns.second) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (fns.first(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (fns.second(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device context (so that
+// calls made during stream capture issue no attribute change).  The context id is
+// remembered per device; a new context (after a device reset) sets it again.
 template <auto Kern>
 inline bool set_smem_once(int bytes) {
-  static bool done[64] = {};
+  static std::atomic<unsigned long long> done_ctx[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (done[dev]) return true;
+  const unsigned long long ctx = current_context_id();
+  if (ctx != 0 && done_ctx[dev].load() == ctx) return true;
   if (cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
       cudaSuccess)
     return false;
-  done[dev] = true;
+  // the attribute call made the primary context current if none was yet
+  done_ctx[dev].store(ctx != 0 ? ctx : current_context_id());
   return true;
 }
 

@@ -7,9 +7,12 @@ One step = the whole hot path for one batch of decode queries of one layer:
   eta_screen           (O(1) block screening, per-head masks, union compaction)
   eta_decode           (gated split-KV attention over admitted blocks + LSE combine)
 
-Default workload: batch 64, 16 query / 4 KV heads, d = 128, 128K context, KV
-block 64, bf16 clustered-key cache (256 clusters, segments of 384-640 tokens),
-threshold bias calibrated for 16% union density, exact bound, hard gate.
+Default workload: batch 64, 16 query / 4 KV heads, d = 128, 512K context (68.7 GB
+of K/V), KV block 128, bf16 clustered-key cache (256 clusters, segments of 384-640
+tokens), threshold bias calibrated for 16% union density, probabilistic variance
+bound with z = 3 (the exact bound's union density at the same thresholds and the
+keys scoring above tau that z = 3 prunes are reported beside it), hard gate.
+`--workload long-b64...` selects the 128K / block-64 / exact-bound configuration.
 
 Prints ONE JSON line (rank 0).  `--impl reference` times the float64 CPU oracle
 on a bounded sample of the same workload instead (rank 0 only).
@@ -64,6 +67,10 @@ def with_overrides(w: synth.Workload, args) -> synth.Workload:
         kw["density_kind"] = args.density_kind
     if getattr(args, "tau_mode", None):
         kw["tau_mode"] = args.tau_mode
+    if getattr(args, "bound", None):
+        kw["bound"] = args.bound
+    if getattr(args, "ctx", 0):
+        kw["ctx"] = int(args.ctx)
     if not kw:
         return w
     tag = "-".join(f"{k}{v}" for k, v in sorted(kw.items()))
@@ -81,7 +88,8 @@ def density_offset(bounds: np.ndarray, tau0: np.ndarray, valid: np.ndarray, dens
                    G: int, kind: str) -> float:
     """Common threshold offset that admits the target fraction of (head, block)
     pairs ("head") or (KV group, block) pairs ("union"): a quantile of the
-    margins bound - tau.  Workload calibration only (host numpy)."""
+    margins bound - tau, placed halfway to the next lower margin so that no bound
+    sits exactly on a threshold.  Workload calibration only (host numpy)."""
     B, Hq, NB = bounds.shape
     m = np.where(valid, bounds - tau0[:, :, None], -np.inf)
     if kind == "union":
@@ -89,7 +97,10 @@ def density_offset(bounds: np.ndarray, tau0: np.ndarray, valid: np.ndarray, dens
     v = m[np.isfinite(m)]
     k = int(math.floor((1.0 - density) * v.size))
     k = min(max(k, 0), v.size - 1)
-    return float(np.partition(v, k)[k])
+    part = np.partition(v, [k - 1, k] if k > 0 else [k])
+    if k == 0:
+        return float(part[0]) - 1.0
+    return 0.5 * (float(part[k - 1]) + float(part[k]))
 
 
 def decode_traffic(admitted_kv: int, engine_tc: bool, record: str = "decode_tc_traffic.json"):
@@ -212,6 +223,95 @@ def setup(w: synth.Workload, device, rank: int, cent_format: str = "f32", fused:
         bias = torch.full((w.Hq,), off, dtype=torch.float32, device=device)
     dec.bounds = None
     return g, dec, W, bias, tau_const
+
+
+def workload_config(w: synth.Workload, args) -> dict:
+    """The workload keys of the JSON line, identical in the eta and reference arms
+    (what was measured about the run goes elsewhere in the line)."""
+    dense_kv = w.B * w.Hkv * w.ctx * w.d * 2 * 2
+    nb_total = w.B * w.Hkv * ((w.ctx + w.blk - 1) // w.blk)
+    cb = 2 if args.cent == "bf16" else 4
+    est = w.density * dense_kv + nb_total * (cb * w.d + 12)
+    return {
+        "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+        "context": w.ctx, "blk": w.blk, "bound": w.bound,
+        "z": w.z if w.bound != "exact" else None, "gate_T": w.gate_T,
+        "tau_mode": w.tau_mode, "density_target": f"{w.density:.2f} {w.density_kind}",
+        "centroids": args.cent, "engine": args.engine, "cuda_graph": bool(args.graph),
+        "fused_step": bool(args.fused),
+        "prologue": "separate" if args.separate_prologue else "one launch",
+        "l2": (f"no flush: a step reads about {est / 1e9:.2f} GB (admitted K/V at the density "
+               "target + screened metadata), more than the 126 MB L2" if est > L2_BYTES else
+               f"no flush: a step's ~{est / 1e6:.1f} MB stay L2-resident (a launch-latency "
+               "figure, not a bandwidth one)"),
+        "parallelism": "single GPU",
+    }
+
+
+def unpack_admit(words: torch.Tensor, NB: int) -> torch.Tensor:
+    """uint32 mask words [..., NW] (held as int32) -> bool [..., NB] on the device."""
+    j = torch.arange(NB, device=words.device)
+    w = words[..., j // 32].to(torch.int64) & 0xFFFFFFFF
+    return ((w >> (j % 32)) & 1).bool()
+
+
+def screen_diagnostics(dec, q, w) -> dict:
+    """Statistics of the step's screening, taken after the timed region:
+    - near_tie_blocks: (query head, block) pairs whose bound lies within 1e-5 of
+      tau (relative, floored at 1), where fp32 rounding may flip the admit bit;
+    - empty_unions: (row, KV head) pairs that admitted no block;
+    - keys scoring s >= tau (s = scale q.k over every valid key, fp32, computed with
+      torch over all rows) and how many of them sit in blocks the screening pruned
+      for their head, or pruned from their group's union (the union is what the
+      decode reads).  The exact bound never prunes such a key (up to fp32 ties);
+      for a probabilistic bound the ratio is its measured miss rate;
+    - for a probabilistic bound, the union density the exact bound admits at the
+      same thresholds."""
+    from long_context_decoding_eta_b200 import _lib
+    B, Hq, Hkv, NB, G, blk = dec.B, dec.Hq, dec.Hkv, dec.NB, dec.Hq // dec.Hkv, dec.blk
+    dev = dec.K.device
+    bounds = torch.empty(B, Hq, NB, dtype=torch.float32, device=dev)
+    hm = torch.empty_like(dec.head_mask)
+    ui, uc, hc = (torch.empty_like(dec.union_idx), torch.empty_like(dec.union_cnt),
+                  torch.empty_like(dec.head_cnt))
+    _lib.eta_screen(dec.dims, q, dec.tau, dec.cent, dec.rmax, dec.var, dec.cnt, dec.bound,
+                    dec.z, dec.scale, hm, ui, uc, bounds, hc, dec.ws_screen, dec.dev_status,
+                    None, dec.vardim)
+    valid_blk = dec.cnt > 0
+    nonempty = int(valid_blk.sum())
+    tau = dec.tau
+    near = ((bounds - tau[..., None]).abs() <= 1e-5 * tau.abs().clamp(min=1.0)[..., None])
+    near &= valid_blk.repeat_interleave(G, dim=1)
+    out = {"near_tie_blocks": int(near.sum()), "screened_pairs": int(nonempty * G),
+           "empty_unions": int((uc == 0).sum()),
+           "union_density": float(uc.sum()) / max(1, nonempty)}
+    if dec.bound != "exact":
+        uc_ex = torch.empty_like(uc)
+        _lib.eta_screen(dec.dims, q, dec.tau, dec.cent, dec.rmax, dec.var, dec.cnt, "exact",
+                        dec.z, dec.scale, torch.empty_like(hm), torch.empty_like(ui), uc_ex,
+                        None, torch.empty_like(hc), dec.ws_screen, dec.dev_status, None,
+                        dec.vardim)
+        out["union_density_exact_bound_same_tau"] = float(uc_ex.sum()) / max(1, nonempty)
+    admit = unpack_admit(hm, NB)                                   # [B, Hq, NB]
+    above = missed_head = missed_union = 0
+    for b in range(B):
+        n = int(dec.lengths[b])
+        if n == 0:
+            continue
+        s = torch.einsum("gtd,ghd->ght", dec.K[b, :, :n].float(),
+                         q[b].float().view(Hkv, G, dec.d)) * dec.scale    # [Hkv, G, n]
+        hi = s >= tau[b].view(Hkv, G, 1)
+        blk_of = torch.arange(n, device=dev) // blk
+        adm = admit[b].view(Hkv, G, NB)[:, :, blk_of]                     # [Hkv, G, n]
+        uni = admit[b].view(Hkv, G, NB).any(dim=1)[:, None, blk_of]
+        above += int(hi.sum())
+        missed_head += int((hi & ~adm).sum())
+        missed_union += int((hi & ~uni).sum())
+    out.update({"keys_scoring_above_tau": above, "of_which_pruned_for_their_head": missed_head,
+                "of_which_outside_the_union": missed_union,
+                "miss_rate_head": (missed_head / above) if above else None,
+                "miss_rate_union": (missed_union / above) if above else None})
+    return out
 
 
 def step_bytes(dec, w):
@@ -347,6 +447,10 @@ def run_eta(args, rank, world, device):
     torch.cuda.synchronize()
     e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, device)
 
+    diag = screen_diagnostics(dec, q, w)
+    torch.cuda.synchronize()
+    dec.check_status()
+
     peak, peak_kind = peaks()
     ms_step = ms / args.steps
     # the dominant kernel: eta_decode's three launches, or the fused step's one launch
@@ -365,21 +469,11 @@ def run_eta(args, rank, world, device):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {
-            "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-            "context": w.ctx, "blk": w.blk, "bound": w.bound, "gate_T": w.gate_T,
-            "tau_mode": w.tau_mode, "engine": args.engine, "centroids": args.cent,
-            "cuda_graph": bool(args.graph), "fused_step": fused,
-            "prologue": "separate" if args.separate_prologue else "one launch",
-            "density_target": f"{w.density:.2f} {w.density_kind}",
-            "union_density": round(by["union_density"], 4),
-            "head_density": round(by["head_density"], 4),
-            "l2": (f"no flush: the step's {by['step'] / 1e6:.0f} MB (admitted K/V + screened "
-                   "metadata) exceed the 126 MB L2" if by["step"] > L2_BYTES else
-                   f"no flush: the step's {by['step'] / 1e6:.1f} MB stay L2-resident "
-                   "(a launch-latency-bound configuration, not a bandwidth figure)"),
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-        },
+        "config": dict(workload_config(w, args),
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "density": {"union": round(by["union_density"], 4),
+                    "head": round(by["head_density"], 4)},
+        "screening": diag,
         "hbm_gbs": by["step"] / (ms_step * 1e-3) / 1e9,
         "hbm_frac_of_nominal_8tbs": by["step"] / (ms_step * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
         "bytes_per_step": {"admitted_kv": by["admitted_kv"], "metadata": by["meta"],
@@ -415,70 +509,74 @@ def run_eta(args, rank, world, device):
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, g, dec, W, bias, tau_const, rows=args.cpu_rows)
+        res["cpu_baseline"] = cpu_baseline(w, g, rows=args.cpu_rows)
     return res
 
 
-def oracle_sample_step(w, g, W, bias, tau_const, rows):
-    """Float64 oracle over a sample of batch rows (all heads of those rows).
-    Returns (seconds for one step of the sample, threads used)."""
-    from oracle import eta_oracle as O
-    sel = list(rows)
-    K64 = g["K"][sel].double().cpu().numpy()
-    V64 = g["V"][sel].double().cpu().numpy()
-    q64 = g["q"][sel].double().cpu().numpy()
-    L = g["lengths"][sel].cpu().numpy()
-    meta = O.cache_meta(K64, L, w.blk)           # prefill (not timed)
+class OracleSample:
+    """The float64 oracle's decode step over a bounded sample of batch rows (all
+    heads of those rows), on the same cache bytes the GPU reads.  The widened
+    cache and its block metadata (the prefill) are prepared once, untimed; each
+    step() times one oracle step: the tail-block metadata of every sampled
+    (row, KV head), the thresholds, the screening and the gated decode."""
+
+    def __init__(self, w, g, rows):
+        from oracle import eta_oracle as O
+        self.O, self.w = O, w
+        self.rows = list(rows)
+        self.K64 = g["K"][self.rows].double().cpu().numpy()
+        self.V64 = g["V"][self.rows].double().cpu().numpy()
+        self.q64 = g["q"][self.rows].double().cpu().numpy()
+        self.L = g["lengths"][self.rows].cpu().numpy()
+        self.meta = O.cache_meta(self.K64, self.L, w.blk)
+        self.scale = 1.0 / math.sqrt(w.d)
+
+    def step(self, W64, b64, tc) -> float:
+        O, w, K64, L, meta = self.O, self.w, self.K64, self.L, self.meta
+        t = time.perf_counter()
+        for i in range(len(self.rows)):
+            j = (int(L[i]) - 1) // w.blk
+            for h in range(w.Hkv):
+                m = O.block_meta(K64[i, h, j * w.blk:(j + 1) * w.blk], int(L[i]) - j * w.blk,
+                                 w.blk)
+                for k in ("cent", "rmax", "var", "cnt", "vardim"):
+                    meta[k][i, h, j] = m[k][0]
+        tau = (O.predict_tau(self.q64, W64, b64) if tc is None
+               else O.const_tau(len(self.rows), tc))
+        sc = O.screen(self.q64, tau, meta, self.scale, w.bound, w.z)
+        O.decode(self.q64, tau, K64, self.V64, L, sc["union_idx"], w.blk, self.scale, w.gate_T)
+        return time.perf_counter() - t
+
+    def union_density(self, W64, b64, tc) -> float:
+        O = self.O
+        tau = (O.predict_tau(self.q64, W64, b64) if tc is None
+               else O.const_tau(len(self.rows), tc))
+        sc = O.screen(self.q64, tau, self.meta, self.scale, self.w.bound, self.w.z)
+        return float(sc["union"].sum()) / max(1, int((self.meta["cnt"] > 0).sum()))
+
+
+def time_oracle(sample: OracleSample, W, bias, tau_const, warmup: int, reps: int):
+    """Per-step seconds of `reps` oracle steps after `warmup` untimed ones, with
+    numpy's BLAS held to one thread (the oracle is single-threaded Python loops
+    over rows and heads; the thread count reported is the one used)."""
+    from threadpoolctl import threadpool_limits
     W64 = None if W is None else W.double().cpu().numpy()
     b64 = None if bias is None else bias.double().cpu().numpy()
     tc = None if tau_const is None else tau_const.double().cpu().numpy()
-    scale = 1.0 / math.sqrt(w.d)
-    t = time.perf_counter()
-    # tail-block metadata of every sampled (row, KV head)
-    for i in range(len(sel)):
-        j = (int(L[i]) - 1) // w.blk
-        for h in range(w.Hkv):
-            m = O.block_meta(K64[i, h, j * w.blk:(j + 1) * w.blk], int(L[i]) - j * w.blk, w.blk)
-            for k in ("cent", "rmax", "var", "cnt"):
-                meta[k][i, h, j] = m[k][0]
-    tau = O.predict_tau(q64, W64, b64) if tc is None else O.const_tau(len(sel), tc)
-    sc = O.screen(q64, tau, meta, scale, w.bound, w.z)
-    O.decode(q64, tau, K64, V64, L, sc["union_idx"], w.blk, scale, w.gate_T)
-    dt = time.perf_counter() - t
-    return dt, threads_used()
+    with threadpool_limits(limits=1):
+        for _ in range(warmup):
+            sample.step(W64, b64, tc)
+        return [sample.step(W64, b64, tc) for _ in range(reps)]
 
 
-def threads_used():
-    try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:
-        return os.cpu_count() or 1
-
-
-def cpu_baseline(w, g, dec, W, bias, tau_const, rows=2):
-    rows = max(1, min(rows, w.B))
-    dt, cores = oracle_sample_step(w, g, W, bias, tau_const, range(rows))
-    per_step = dt * w.B / rows
-    return {"value": 1.0 / per_step, "unit": "steps/s", "cores": cores, "kind": "oracle",
-            "sample": f"{rows} of {w.B} batch rows (all {w.Hq} heads), float64 numpy oracle, "
-                      f"{dt:.2f} s measured, scaled by B/{rows}"}
-
-
-def run_reference(args, rank, world, device):
-    """The float64 CPU oracle as the reference arm, on a bounded sample per step.
-    The threshold bias is set by the oracle itself on the sampled rows, with the
-    same density rule as the eta arm; no CUDA kernel of this package runs."""
+def oracle_sample_inputs(w, g, rows):
+    """The oracle's sample of `rows` batch rows and its threshold inputs: the
+    predictor's W with a bias the oracle sets itself on those rows by the workload's
+    density rule, or (calibrated workloads) per-head constants from the calibration
+    rule on them.  Both arms time the oracle on exactly these inputs."""
     from oracle import eta_oracle as O
-    w = with_overrides(workload_by_name(args.workload, args.B), args)
-    g = synth.generate(w, device, seed=w.seed)
-    rows = list(range(max(1, min(args.cpu_rows, w.B))))
-    K64 = g["K"][rows].double().cpu().numpy()
-    q64 = g["q"][rows].double().cpu().numpy()
-    L = g["lengths"][rows].cpu().numpy()
-    scale = 1.0 / math.sqrt(w.d)
-    meta = O.cache_meta(K64, L, w.blk)
+    sample = OracleSample(w, g, rows)
+    meta, q64, scale = sample.meta, sample.q64, sample.scale
     W = bias = tau_const = None
     if w.tau_mode == "const":
         qc = synth.calibration_queries(w, g["mu"]).double().cpu().numpy()
@@ -500,26 +598,59 @@ def run_reference(args, rank, world, device):
         off = O.offset_for_density(ub, tau0, np.repeat(meta["cnt"] > 0, w.G, axis=1),
                                    w.density, w.G, w.density_kind)
         bias = torch.full((w.Hq,), off, dtype=torch.float64)
-    del K64
-    for _ in range(args.warmup):
-        oracle_sample_step(w, g, W, bias, tau_const, rows)
-    times = []
-    cores = 1
-    for _ in range(args.steps):
-        dt, cores = oracle_sample_step(w, g, W, bias, tau_const, rows)
-        times.append(dt * w.B / len(rows))
+    return sample, W, bias, tau_const
+
+
+def cpu_baseline(w, g, rows=2, warmup=1, reps=3):
+    """The oracle timed as the reference arm times it (same sample, same threshold
+    inputs, one thread), inside the eta arm's line."""
+    rows = list(range(max(1, min(rows, w.B))))
+    sample, W, bias, tau_const = oracle_sample_inputs(w, g, rows)
+    times = time_oracle(sample, W, bias, tau_const, warmup, reps)
+    per = statistics.median(times)
+    n = len(rows)
+    return {"value": n / w.B / per, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {w.B} batch rows (all {w.Hq} heads) per oracle step, float64 "
+                      f"numpy oracle on one thread, threshold offset set by the oracle on "
+                      f"those rows; median of {reps} steps after {warmup} warm-up ({per:.2f} s "
+                      f"each), steps/s scaled by {n}/{w.B}"}
+
+
+def run_reference(args, rank, world, device):
+    """The float64 CPU oracle as the reference arm.  Each step is the oracle's step
+    over a bounded sample of batch rows (all heads), timed on one host thread; the
+    line's value is whole-batch steps/s, scaled from the sample by rows / B, and
+    ms_per_step is the measured time of one sampled step (so that steps x ms_per_step
+    is the run's timed work).  The threshold bias is set by the oracle itself on the
+    sampled rows with the eta arm's density rule; no CUDA kernel of this package
+    runs (torch only draws the seeded inputs)."""
+    w = with_overrides(workload_by_name(args.workload, args.B), args)
+    g = synth.generate(w, device, seed=w.seed)
+    rows = list(range(max(1, min(args.cpu_rows, w.B))))
+    sample, W, bias, tau_const = oracle_sample_inputs(w, g, rows)
+    del g
+    times = time_oracle(sample, W, bias, tau_const, args.warmup, args.steps)
     per = sum(times) / len(times)
-    v = 1.0 / per
+    v = len(rows) / w.B / per
+    dens = sample.union_density(None if W is None else W.double().cpu().numpy(),
+                                None if bias is None else bias.double().cpu().numpy(),
+                                None if tau_const is None else tau_const.double().numpy())
     return {
         "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
-                   "context": w.ctx, "blk": w.blk},
-        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{len(rows)} of {w.B} batch rows per step (all heads), "
-                                   f"scaled by B/{len(rows)}"},
+        "value_basis": (f"each step runs the oracle on {len(rows)} of {w.B} batch rows; value = "
+                        f"whole-batch steps/s = ({len(rows)}/{w.B}) / measured seconds per "
+                        f"sampled step; ms_per_step = measured time of one sampled step"),
+        "ms_per_full_step_extrapolated": per * 1e3 * w.B / len(rows),
+        "config": workload_config(w, args),
+        "density": {"union": round(dens, 4), "rows": len(rows)},
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{len(rows)} of {w.B} batch rows (all {w.Hq} heads) per "
+                                   f"step, float64 numpy oracle on one thread, threshold "
+                                   f"offset set by the oracle on those rows, steps/s scaled "
+                                   f"by {len(rows)}/{w.B}"},
         "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -582,7 +713,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default=synth.LONG128K.name)
+    ap.add_argument("--workload", default=synth.EXTREME512K.name,
+                    help="workload name or prefix (tiny, mid, long, extreme, calibrated)")
     ap.add_argument("--impl", default="eta", choices=["eta", "reference"])
     ap.add_argument("--mode", default="decode", choices=["decode", "prefill"],
                     help="decode: the ETA decode step (default); prefill: eta_prefill")
@@ -602,6 +734,10 @@ def main():
     ap.add_argument("--clock-soak-s", type=float, default=1.0,
                     help="untimed steps run under the clock sampler before the timed region")
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
+    ap.add_argument("--ctx", type=int, default=0,
+                    help="override the context length (small profiling captures)")
+    ap.add_argument("--bound", default="", choices=["", "exact", "prob", "prob_dim"],
+                    help="override the screening bound (the extreme workload's exact arm)")
     ap.add_argument("--engine", default="auto", choices=["auto", "tcgen05", "fma"],
                     help="decode engine of libeta.so")
     ap.add_argument("--separate-prologue", action="store_true",

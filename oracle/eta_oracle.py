@@ -401,7 +401,9 @@ def offset_for_density(bounds: np.ndarray, tau: np.ndarray, valid: np.ndarray,
                        density: float, G: int, kind: str = "head") -> float:
     """Common offset delta such that thresholds tau + delta admit (at least) the
     target fraction of (query head, block) pairs ("head") or of (KV group,
-    block) pairs in the union ("union").  Input-synthesis helper for tests."""
+    block) pairs in the union ("union").  Input-synthesis helper for tests.
+    delta lies halfway between the k-th margin and the one below it, so that no
+    bound sits exactly on a threshold (a tie the test would have to skip)."""
     B, Hq, NB = bounds.shape
     margin = np.where(valid, bounds - tau[:, :, None], -np.inf)
     if kind == "union":
@@ -409,4 +411,6 @@ def offset_for_density(bounds: np.ndarray, tau: np.ndarray, valid: np.ndarray,
     vals = np.sort(margin[np.isfinite(margin)])
     k = int(math.floor((1.0 - density) * vals.size))
     k = min(max(k, 0), vals.size - 1)
-    return float(vals[k])
+    if k == 0:
+        return float(vals[0]) - 1.0
+    return 0.5 * (float(vals[k - 1]) + float(vals[k]))

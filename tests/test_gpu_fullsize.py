@@ -53,10 +53,14 @@ def whole_batch_properties(dec, gpu, w):
     return un.mean()
 
 
-def run_fullsize(w, rows, tau_const=None, engine="auto", cent_format="f32"):
+def run_fullsize(w, rows, tau_const=None, engine="auto", cent_format="f32", g=None,
+                 keep=False):
+    """The whole batch through the CUDA path; the oracle on `rows`.  With keep=True
+    the decoder is returned too (the caller frees it)."""
     L.eta_set_decode_engine(engine)
     scale = 1.0 / math.sqrt(w.d)
-    g = synth.generate(w, "cuda")
+    own = g is None
+    g = synth.generate(w, "cuda") if own else g
     dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, bound=w.bound, z=w.z,
                      T=w.gate_T, keep_bounds=True, cent_format=cent_format)
     dec.build_meta()
@@ -82,10 +86,14 @@ def run_fullsize(w, rows, tau_const=None, engine="auto", cent_format="f32"):
     check_meta(gpu_meta(dec, rows), meta)
     rep = compare_step(gpu, tau, sc, o, lse, q64, K64, V64, L64, w.blk, scale, w.gate_T, w.G,
                        rows=rows)
-    del dec, g
+    L.eta_set_decode_engine("auto")
+    if keep:
+        return rep, union_density, dec, gpu
+    del dec
+    if own:
+        del g
     gc.collect()
     torch.cuda.empty_cache()
-    L.eta_set_decode_engine("auto")
     return rep, union_density
 
 
@@ -109,21 +117,55 @@ def test_long_128k_b64_union16(engine, cent):
     print(rep, dens)
 
 
-def test_extreme_512k_b64_prob_bound_blk128():
-    w = synth.EXTREME512K
-    rep, dens = run_fullsize(w, rows=[5, 60])
-    assert 0.01 < dens < 0.6, dens
+@pytest.mark.parametrize("density,kind", [(0.38, "head"), (0.51, "union")])
+def test_long_128k_b64_trained_operating_points(density, kind):
+    """The 128K configuration at the pages' trained operating point: about 38% of
+    blocks per head, or 51% in the union (review Summary: 51.2% union density at
+    B = 64)."""
+    w = synth.LONG128K.with_(density=density, density_kind=kind)
+    rep, dens = run_fullsize(w, rows=[1, 50], cent_format="bf16")
+    lo, hi = (0.3, 0.95) if kind == "head" else (0.35, 0.7)
+    assert lo < dens < hi, dens
     print(rep, dens)
 
 
-def test_calibrated_256k_const_tau():
-    # per-head constants from the calibration rule on the oracle, with the
-    # calibration queries paired with the sampled rows (the full-batch pairing
-    # would need the oracle's metadata of all 64 rows)
-    w = synth.CALIB256K
-    rows = [3, 42]
-    scale = 1.0 / math.sqrt(w.d)
+def test_extreme_512k_b64_prob_and_exact_bound_blk128():
+    """512K context, block 128: the probabilistic bound (z = 3) and the exact bound,
+    each with its threshold offset set for 16% union density on the sampled rows, on
+    the same cache; and at the probabilistic arm's thresholds, every block the z = 3
+    bound admits is one the exact bound admits too (its bound is never larger), on
+    every row of the batch."""
+    w = synth.EXTREME512K
     g = synth.generate(w, "cuda")
+    rep, dens, dec, gpu = run_fullsize(w, rows=[5, 60], g=g, keep=True)
+    assert 0.01 < dens < 0.6, dens
+    ex_mask = torch.empty_like(dec.head_mask)
+    ex_cnt = torch.empty_like(dec.union_cnt)
+    L.eta_screen(dec.dims, g["q"], dec.tau, dec.cent, dec.rmax, dec.var, dec.cnt, "exact",
+                 w.z, dec.scale, ex_mask, torch.empty_like(dec.union_idx), ex_cnt, None,
+                 torch.empty_like(dec.head_cnt), dec.ws_screen, dec.dev_status)
+    torch.cuda.synchronize()
+    dec.check_status()
+    ex = unpack_mask(ex_mask, dec.NB)
+    assert not np.any(gpu["head_mask"] & ~ex), "z = 3 admitted a block the exact bound pruned"
+    nonempty = int((dec.cnt > 0).sum())
+    dens_exact = float(ex_cnt.sum()) / nonempty
+    assert dens_exact >= dens
+    print(rep, "union density z=3:", dens, "exact bound at the same tau:", dens_exact)
+    del dec, gpu
+    gc.collect()
+    rep_ex, dens_ex = run_fullsize(w.with_(bound="exact"), rows=[5, 60], g=g)
+    assert 0.01 < dens_ex < 0.6, dens_ex
+    print(rep_ex, "exact-bound arm union density:", dens_ex)
+    del g
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+def calibrated_tau_const(w, g, rows, scale):
+    """Per-head constants from the calibration rule on the oracle, with the
+    calibration queries paired with the sampled rows (the full-batch pairing would
+    need the oracle's metadata of every row)."""
     K64 = rows_f64(g["K"], rows)
     L64 = g["lengths"][rows].cpu().numpy()
     meta = O.cache_meta(K64, L64, w.blk)
@@ -136,12 +178,39 @@ def test_calibrated_256k_const_tau():
         mrow = {k: v[r:r + 1] for k, v in meta.items()}
         bounds[i] = O.screen(qc[i:i + 1], np.zeros((1, w.Hq)), mrow, scale)["bounds"][0]
         valid[i] = np.repeat(meta["cnt"][r] > 0, w.G, axis=0)
-    tau_const = O.calibrate_const_tau(bounds, valid, w.density)
-    del g, K64
+    return O.calibrate_const_tau(bounds, valid, w.density)
+
+
+def test_calibrated_256k_const_tau_and_predictor_same_inputs():
+    """256K, B = 64: frozen per-head constants from the calibration rule, then the
+    predictor (Eq. 1, offset for the same 38% per-head target) on the same inputs."""
+    w = synth.CALIB256K
+    rows = [3, 42]
+    scale = 1.0 / math.sqrt(w.d)
+    g = synth.generate(w, "cuda")
+    tau_const = calibrated_tau_const(w, g, rows, scale)
+    rep, dens = run_fullsize(w, rows=rows, tau_const=tau_const, g=g)
+    print("const tau:", rep, dens)
+    rep_p, dens_p = run_fullsize(w.with_(tau_mode="predictor"), rows=rows, g=g)
+    print("predictor:", rep_p, dens_p)
+    del g
     gc.collect()
     torch.cuda.empty_cache()
-    rep, dens = run_fullsize(w, rows=rows, tau_const=tau_const)
+
+
+def test_calibrated_256k_b32_const_tau():
+    """The calibrated configuration at B = 32 (the pages report ETA slower than
+    FlashAttention-2 there on H100)."""
+    w = synth.CALIB256K.with_(B=32, name="calibrated-b32-h16x4-d128-ctx256k-blk64")
+    rows = [0, 31]
+    scale = 1.0 / math.sqrt(w.d)
+    g = synth.generate(w, "cuda")
+    tau_const = calibrated_tau_const(w, g, rows, scale)
+    rep, dens = run_fullsize(w, rows=rows, tau_const=tau_const, g=g)
     print(rep, dens)
+    del g
+    gc.collect()
+    torch.cuda.empty_cache()
 
 
 def test_long_128k_fused_step_equals_separate_calls():

@@ -46,8 +46,8 @@ constexpr int NKV = 2;                          // KV ring stages
 constexpr int OFF_Q = 0;                        // 2 halves
 constexpr int OFF_KV = 2 * HALF;                // stage s: K0 K1 V0 V1
 constexpr int KV_STAGE = 4 * HALF;              // 64 KB
-constexpr int OFF_P = OFF_KV + NKV * KV_STAGE;  // 2 buffers x 2 halves
-constexpr int OFF_MISC = OFF_P + 2 * 2 * HALF;
+constexpr int OFF_P = OFF_KV + NKV * KV_STAGE;  // one P tile: 2 halves (see the softmax)
+constexpr int OFF_MISC = OFF_P + 2 * HALF;
 constexpr int NWARP_SM = 8;                     // two warpgroups: key columns 0-63, 64-127
 constexpr int NT = (NWARP_SM + 2) * 32;
 constexpr int kTmemCols = 512;
@@ -56,7 +56,8 @@ constexpr float kRescale = 8.0f;                // rescale O when the max grows 
 struct Misc {
   uint64_t q_full, kv_full[NKV], kv_empty[NKV];
   uint64_t s_full[2], s_free[2], p_full[2], o_done, o_final, fin;
-  float xch[2][TILE];      // per-half row maxima of a tile, then the final row sums
+  float xch[2][2][TILE];   // per tile parity, per half: the row maxima of a tile
+  float2 xsum[2][TILE];    // per half: the final row sums (rounded weights, exact weights)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -220,7 +221,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         const int s = k % NKV, pb = k & 1;
         if (!mbar_wait(&ms->p_full[pb], (uint32_t)(k >> 1) & 1u, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(smem + OFF_P + pb * 2 * HALF);
+        const uint32_t pa = smem_u32(smem + OFF_P);
         const uint32_t v0 = smem_u32(smem + OFF_KV + s * KV_STAGE + 2 * HALF);
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) {
@@ -268,22 +269,36 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     const uint32_t lsel = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t cb = (uint32_t)hh * 64;            // first column of this half
     const float tau = (tq < p.T_max) ? p.tau[((size_t)b * p.Hq + h) * p.T_max + tq] : 0.f;
+    // Gated logits in raw units u (the gated logit is scale * u), so that the scale
+    // folds into the constants: the hard gate keeps s iff scale * s >= tau, i.e.
+    // s >= tau / scale (scale > 0); the soft gate is
+    //   scale * s * sigmoid((scale * s - tau) / T) = scale * (hs + hs * tanh(s * ta - tb)),
+    // hs = s / 2, ta = scale / 2T, tb = tau / 2T; and e^(scale * (u - m)) is
+    // 2^(u * c1 - m * c1), c1 = scale * log2(e): one FFMA and one ex2 per key.
+    const bool hard = p.invT < 0.f;
+    const float tau_raw = tau / p.scale;
+    const float ta = 0.5f * p.scale * p.invT, tb = 0.5f * tau * p.invT;
+    const float c1 = p.scale * kLog2e;
+    const float resc_raw = kRescale / p.scale;
     // l: row sum of the bf16-rounded weights (normalizes O, which the tensor core
     // built from those weights); lx: row sum of the exact fp32 weights (for lse);
-    // both over this half's columns until the end
-    float m_used = -INFINITY, l = 0.f, lx = 0.f;
+    // both over this half's columns until the end, two columns per packed add
+    float m_used = -INFINITY;                         // raw units
+    float2 l2 = make_float2(0.f, 0.f), lx2 = make_float2(0.f, 0.f);
     bool ok = true;
     float sv[64];
     // every lane polls; the warp agrees on the outcome so collectives stay converged
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
-    // Both halves of a row pass the same named barriers in every tile, failed or
-    // not: a warp whose bounded wait ran out keeps looping with its work skipped,
-    // so its partner half never blocks on a barrier it will not reach.
-    auto halves_sync = [] { named_bar_sync(3, NWARP_SM * 32); };
-    const bool hard = p.invT < 0.f;
-    const float half_invT = 0.5f * p.invT;
+    // The two warps that share these TMEM lanes (warp w and w + 4: the two halves of
+    // the same rows) exchange through shared memory behind their own 64-thread
+    // barrier.  Both pass it in every tile, failed or not: a warp whose bounded wait
+    // ran out keeps looping with its work skipped, so its partner never blocks on a
+    // barrier it will not reach.  The exchange buffer alternates with the tile's
+    // parity, so one barrier per tile suffices.
+    const int pair_bar = 4 + (warp & 3);
+    auto pair_sync = [&] { named_bar_sync(pair_bar, 64); };
     for (int j = 0; j < nkv; ++j) {
       const int sb = j & 1, s = j % NKV;
       const int k0 = j * TILE;
@@ -302,18 +317,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 #pragma unroll
         for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
         auto gate = [&](float x) -> float {
-          if (hard) return x >= tau ? x : 0.f;
-          // x * sigmoid((x - tau) / T) = hx + hx * tanh((x - tau) / 2T), hx = x / 2:
-          // one SFU op (tanh.approx) instead of an exponential and a reciprocal
-          const float hx = 0.5f * x;
-          return fmaf(hx, tanh_approx((x - tau) * half_invT), hx);
+          if (hard) return x >= tau_raw ? x : 0.f;
+          const float hs = 0.5f * x;
+          return fmaf(hs, tanh_approx(fmaf(x, ta, -tb)), hs);
         };
         if (j == nkv - 1) {
           // the diagonal tile (k0 == q0): keys past the row's query are masked
           const int lim = tq - k0 - (int)cb;           // columns c <= lim are causal
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            const float y = (c <= lim) ? gate(p.scale * sv[c]) : -INFINITY;
+            const float y = (c <= lim) ? gate(sv[c]) : -INFINITY;
             sv[c] = y;
             pm[c & 7] = fmaxf(pm[c & 7], y);
           }
@@ -321,7 +334,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           // every key of an earlier tile precedes every query of this one
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
-            const float y = gate(p.scale * sv[c]);
+            const float y = gate(sv[c]);
             sv[c] = y;
             pm[c & 7] = fmaxf(pm[c & 7], y);
           }
@@ -330,30 +343,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
       }
       // the row max of the tile: this half's, then the other half's
-      ms->xch[hh][row] = mxh;
-      halves_sync();
-      const float mx = fmaxf(ms->xch[0][row], ms->xch[1][row]);
-      halves_sync();
+      ms->xch[sb][hh][row] = mxh;
+      pair_sync();
+      const float mx = fmaxf(ms->xch[sb][0][row], ms->xch[sb][1][row]);
       if (!ok) continue;
       // running max: the first tile sets it; later tiles rescale O (in TMEM) only
-      // when the max grew by more than kRescale.  Both halves of a row take the
-      // same decision from the same values.
+      // when the max grew by more than kRescale (in logit units).  Both halves of a
+      // row take the same decision from the same values.
       float alpha = 1.f;
       bool resc = false;
       if (m_used == -INFINITY) {
         m_used = mx;
-      } else if (mx > m_used + kRescale) {
-        alpha = __expf(m_used - mx);
+      } else if (mx > m_used + resc_raw) {
+        alpha = ex2_approx((m_used - mx) * c1);
         m_used = mx;
         resc = true;
       }
+      // P of this tile goes into the one P buffer, and a rescale touches O: both
+      // wait until P V of the previous tile is done (it was issued when the previous
+      // tile's P was complete, so it has usually finished by now)
+      if (j > 0 && !wwait(&ms->o_done, (uint32_t)((j - 1) & 1))) {
+        ok = false;
+        continue;
+      }
       if (__any_sync(0xffffffffu, resc)) {
-        // O holds tiles 0 .. j-1: wait for the last P V before touching it (P V of
-        // tile j-2 is known complete: it was issued before Q K^T of tile j)
-        if (!wwait(&ms->o_done, (uint32_t)((j - 1) & 1))) {
-          ok = false;
-          continue;
-        }
         tc_fence_after();
         float ov[32];
 #pragma unroll
@@ -366,34 +379,31 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         }
         tmem_wait_st();
         tc_fence_before();
-        l *= alpha;
-        lx *= alpha;
+        l2.x *= alpha; l2.y *= alpha;
+        lx2.x *= alpha; lx2.y *= alpha;
       }
-      // P = exp(s' - m) as bf16, row `row` of this half's swizzled 64-key A tile
-      unsigned char* pbuf = smem + OFF_P + sb * 2 * HALF + hh * HALF;
-      float ls4[4] = {0.f, 0.f, 0.f, 0.f}, lx4[4] = {0.f, 0.f, 0.f, 0.f};
-      const float nm = -m_used * kLog2e;               // e^(y - m) = 2^(y log2e - m log2e)
+      // P = e^(scale * (u - m)) as bf16, row `row` of this half's swizzled 64-key A tile
+      const float nm = -m_used * c1;
+      unsigned char* pbuf = smem + OFF_P + hh * HALF;
 #pragma unroll
       for (int c16 = 0; c16 < 8; ++c16) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2_approx(fmaf(sv[c16 * 8 + 2 * e], kLog2e, nm));
-          const float p1 = ex2_approx(fmaf(sv[c16 * 8 + 2 * e + 1], kLog2e, nm));
+          const float2 a = __ffma2_rn(make_float2(sv[c16 * 8 + 2 * e], sv[c16 * 8 + 2 * e + 1]),
+                                      make_float2(c1, c1), make_float2(nm, nm));
+          const float p0 = ex2_approx(a.x), p1 = ex2_approx(a.y);
           const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
           // the row sum uses the rounded weights the tensor core multiplies, so
           // O / l is an exact convex combination of them (a dominant weight's
           // rounding cancels between numerator and denominator)
-          const float2 pf = __bfloat1622float2(pr);
-          ls4[e] += pf.x + pf.y;
-          lx4[e] += p0 + p1;
+          l2 = __fadd2_rn(l2, __bfloat1622float2(pr));
+          lx2 = __fadd2_rn(lx2, make_float2(p0, p1));
           w[e] = *reinterpret_cast<const uint32_t*>(&pr);
         }
         *reinterpret_cast<uint4*>(pbuf + row * 128 + ((c16 ^ (row & 7)) << 4)) =
             make_uint4(w[0], w[1], w[2], w[3]);
       }
-      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
-      lx += (lx4[0] + lx4[1]) + (lx4[2] + lx4[3]);
       // the last key tile: V rows past the sequence end must be finite for P V
       if (k0 + TILE > len && k0 + row >= len) {
         unsigned char* vt = smem + OFF_KV + s * KV_STAGE + 2 * HALF + hh * HALF;
@@ -408,13 +418,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     // every P V done (a single-phase barrier: no parity aliasing)
     if (ok && !wwait(&ms->o_final, 0u)) ok = false;
     // the halves' row sums (every warp reaches this point, failed or not)
-    ms->xch[hh][row] = l;
-    halves_sync();
-    const float l_row = ms->xch[0][row] + ms->xch[1][row];
-    halves_sync();
-    ms->xch[hh][row] = lx;
-    halves_sync();
-    const float lx_row = ms->xch[0][row] + ms->xch[1][row];
+    ms->xsum[hh][row] = make_float2(l2.x + l2.y, lx2.x + lx2.y);
+    pair_sync();
+    const float2 s0 = ms->xsum[0][row], s1 = ms->xsum[1][row];
+    const float l_row = s0.x + s1.x, lx_row = s0.y + s1.y;
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l_row;
@@ -432,7 +439,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
         }
       }
-      if (store && hh == 0) p.lse[((size_t)b * p.Hq + h) * p.T_max + tq] = m_used + logf(lx_row);
+      if (store && hh == 0)
+        p.lse[((size_t)b * p.Hq + h) * p.T_max + tq] = p.scale * m_used + logf(lx_row);
     } else {
       if (threadIdx.x == 0) set_status(p.status, ETA_DEVSTAT_TIMEOUT);
       *abort_flag = 1;

@@ -307,3 +307,24 @@ def test_per_dimension_variance_bound(cent_format, ctx):
     w = synth.MID.with_(B=3, ctx=ctx, needles=4, q_scale=4.0, density=0.3, seed=310 + ctx)
     for z in (1.0, 3.0):
         full_parity(w, bound="prob_dim", z=z, cent_format=cent_format, T=0.0)
+
+
+@pytest.mark.parametrize("d,G,Hkv,bound", [(128, 4, 2, "exact"), (128, 4, 2, "prob"),
+                                           (128, 8, 1, "prob_dim"), (128, 1, 4, "exact"),
+                                           (64, 2, 2, "prob")])
+def test_bf16_screen_of_long_rows(d, G, Hkv, bound, engine):
+    """Rows longer than two rounds of the one-launch screen's group buffers take the
+    two-launch screen (vector screening, then compaction) with bf16 centroids, a
+    partial last group and one ragged row: masks, bounds and union lists against the
+    oracle."""
+    from long_context_decoding_eta_b200 import _lib as L
+    # more groups per row than two rounds of the one-launch screen's buffers (5 at
+    # d = 128, 8 at d = 64), and a partial last group
+    ctx = (96 if d == 128 else 160) * 1024 + 512
+    w = synth.Workload("bf16-long-rows", B=2, Hq=G * Hkv, Hkv=Hkv, d=d, ctx=ctx,
+                       blk=64, n_clusters=32, seg=(384, 640), needles=2, gate_T=0.0,
+                       density=0.3, density_kind="head", q_scale=2.0, seed=320 + d + G)
+    dims = L.Dims.of(w.B, w.Hq, w.Hkv, w.d, w.blk, w.T_max)
+    assert L.eta_screen_launches(dims, "bf16") == 2
+    lengths = torch.tensor([w.ctx, w.ctx - 7000], dtype=torch.int32)
+    full_parity(w, lengths=lengths, bound=bound, z=2.0, cent_format="bf16")

@@ -103,10 +103,13 @@ def density_offset(bounds: np.ndarray, tau0: np.ndarray, valid: np.ndarray, dens
     return 0.5 * (float(part[k - 1]) + float(part[k]))
 
 
-def decode_traffic(admitted_kv: int, engine_tc: bool, record: str = "decode_tc_traffic.json"):
-    """DRAM bytes per launch from a committed ncu capture (profiles/<record>), scaled
-    to this workload by its admitted K/V bytes; None when the kernel source changed
-    since the capture or the capture does not cover the engine that ran."""
+def decode_traffic(admitted_kv: int, engine_tc: bool, record: str = "decode_tc_traffic.json",
+                   pairs: int = 0, ctas: int = 0):
+    """DRAM bytes per launch from a committed ncu capture of a small case of the same
+    kernel (profiles/<record>), scaled to this workload: the reads by its admitted K/V
+    bytes, the writes (partial result slots, one per CTA and pair) by its slot count.
+    None when the kernel source changed since the capture or the capture does not
+    cover the engine that ran."""
     import hashlib
     p = os.path.join(ROOT, "profiles", record)
     if not engine_tc or not os.path.exists(p):
@@ -120,8 +123,9 @@ def decode_traffic(admitted_kv: int, engine_tc: bool, record: str = "decode_tc_t
         m.update(open(fp, "rb").read())
     if m.hexdigest() != rec["source_sha256"]:
         return None
-    per = (rec["dram_bytes_read"] + rec["dram_bytes_write"]) / rec["admitted_kv_bytes"]
-    return per * admitted_kv
+    reads = rec["dram_bytes_read"] / rec["admitted_kv_bytes"] * admitted_kv
+    slots = (ctas + pairs) / (rec["ctas"] + rec["pairs"]) if pairs and ctas else 1.0
+    return reads + rec["dram_bytes_write"] * slots
 
 
 def reduce_max(x: float, device) -> float:
@@ -489,11 +493,13 @@ def run_eta(args, rank, world, device):
                      "traffic": decode_traffic(
                          by["admitted_kv"], w.d == 128 and (fused or args.engine in
                                                             ("auto", "tcgen05")),
-                         "step_fused_traffic.json" if fused else "decode_tc_traffic.json"),
+                         "step_fused_traffic.json" if fused else "decode_tc_traffic.json",
+                         dec.B * dec.Hkv, torch.cuda.get_device_properties(device).multi_processor_count),
                      "traffic_source": ("profiles/step_fused_traffic.json" if fused else
                                         "profiles/decode_tc_traffic.json") +
-                                       " (ncu dram__bytes_read+write of one full-size launch, "
-                                       "scaled by admitted KV)"},
+                                       " (ncu dram__bytes_read+write of one launch of a small "
+                                       "case of the same kernel: reads scaled by admitted K/V "
+                                       "bytes, writes by partial-slot count)"},
         "dense_baseline": {"ms": dense_ms, "steps_per_s_decode_only": 1e3 / dense_ms,
                            "gbs": by["dense_kv"] / (dense_ms * 1e-3) / 1e9,
                            "speedup_of_eta_decode": dense_ms / dec_ms},

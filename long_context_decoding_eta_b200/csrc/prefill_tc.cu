@@ -19,6 +19,9 @@
 //           own 64 columns; P is written as bf16 into a swizzled shared tile (the A
 //           operand of P V), each half writing its own 64-key half.
 // TMEM: S 2 x 128 columns, O 128 columns (512 allocated).  Every wait is bounded.
+// This one-tile kernel serves the soft gate; the hard gate takes the two-tile kernel
+// further down (prefill_pp_kernel: two query tiles per CTA sharing every K/V tile,
+// P kept in tensor memory), which measured faster for it.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -455,6 +458,372 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   }
 }
 
+// ---------------------------------------------------------------------------------
+// Two query tiles per CTA ("ping-pong").  One CTA per (batch row, query head, pair of
+// 128-query tiles A = [q0, q0 + 128) and B = [q0 + 128, q0 + 256)), 576 threads:
+//   warps 0-7   softmax of tile A, warps 8-15 softmax of tile B (two threads per
+//               query row, 64 key columns each, as in prefill_tc_kernel)
+//   warp 16     TMA producer: both query tiles, then 128-key K and V tiles into a
+//               2-stage ring; each K/V tile serves both query tiles
+//   warp 17     MMA issuer: S_X = Q_X K^T and O_X += P_X V for X = A, B
+// TMEM (512 columns): S_A, S_B, O_A, O_B (128 each).  P_X is written by its softmax
+// threads into the S_X columns they have already read (half h of a row into columns
+// 64 h .. 64 h + 31 of S_X, two bf16 per column) and read from there by P V as the
+// A operand (tcgen05.mma with A in tensor memory).  While one tile's softmax runs,
+// the tensor core works on the other tile, so neither waits for the other's chain.
+// Tile X's chain per key tile: QK_X -> softmax_X -> P V_X -> QK_X of the next tile
+// (issued once P V_X has read P_X out of the S_X columns).  Every wait is bounded.
+namespace pp {
+
+constexpr int NWG = 8;                          // softmax warps per query tile
+constexpr int NT = (2 * NWG + 2) * 32;
+constexpr int OFF_QA = 0, OFF_QB = 2 * HALF;    // two halves each
+constexpr int OFF_KV = 4 * HALF;
+constexpr int OFF_MISC = OFF_KV + NKV * KV_STAGE;
+
+struct Misc {
+  uint64_t q_full, kv_full[NKV], kv_empty[NKV];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_final[2], fin;
+  float xch[2][2][2][TILE];   // [tile][parity][half][row]: the row maxima of a key tile
+  float2 xsum[2][2][TILE];    // [tile][half][row]: the final row sums
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr int SMEM_BYTES = OFF_MISC + (int)sizeof(Misc) + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "prefill ping-pong shared memory");
+
+ETA_DEV void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                        uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+ETA_DEV void tmem_st16u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15])
+      : "memory");
+}
+
+template <int G, bool HARD>
+__global__ void __launch_bounds__(NT, 1)
+prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  ETA_PDL_ENTRY();
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Misc* ms = reinterpret_cast<Misc*>(smem + OFF_MISC);
+  volatile int* abort_flag = &ms->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // heaviest tile pairs (most keys) first
+  const int qp = p.ntiles - 1 - (int)(blockIdx.x % p.ntiles);   // ntiles: tile pairs here
+  const int bh = blockIdx.x / p.ntiles;
+  const int b = bh / p.Hq, h = bh % p.Hq, g = h / G;
+  const int len = min(max(p.lengths[b], 0), p.T_max);
+  const int q0 = qp * 2 * TILE;
+  if (q0 >= len) return;                              // uniform, before any barrier
+  // key tiles of A: 0 .. q0 / 128 (its diagonal last); of B: one more, if B holds a
+  // valid query
+  const int nA = q0 / TILE + 1;
+  const int nB = (q0 + TILE < len) ? nA + 1 : 0;
+  const int nkv = nB > 0 ? nB : nA;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ms->q_full, 1);
+    for (int s = 0; s < NKV; ++s) {
+      mbar_init(&ms->kv_full[s], 1);
+      mbar_init(&ms->kv_empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&ms->s_full[x], 1);
+      mbar_init(&ms->p_full[x], NWG);
+      mbar_init(&ms->pv_done[x], 1);
+      mbar_init(&ms->o_final[x], 1);
+    }
+    mbar_init(&ms->fin, 1);
+    ms->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2 * NWG + 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&ms->tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ms->tmem_base;
+  const uint32_t tS[2] = {tmem, tmem + 128}, tO[2] = {tmem + 256, tmem + 384};
+
+  if (warp == 2 * NWG) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      bool ok = true;
+      const int qrow = (b * p.Hq + h) * p.T_max + q0;
+      mbar_arrive_expect_tx(&ms->q_full, (nB > 0 ? 4 : 2) * HALF);
+      tma_load_2d(smem + OFF_QA, &tmQ, 0, qrow, &ms->q_full);
+      tma_load_2d(smem + OFF_QA + HALF, &tmQ, 64, qrow, &ms->q_full);
+      if (nB > 0) {
+        tma_load_2d(smem + OFF_QB, &tmQ, 0, qrow + TILE, &ms->q_full);
+        tma_load_2d(smem + OFF_QB + HALF, &tmQ, 64, qrow + TILE, &ms->q_full);
+      }
+      int j = 0;
+      for (; j < nkv && ok; ++j) {
+        const int s = j % NKV;
+        if (!mbar_wait(&ms->kv_empty[s], ((uint32_t)(j / NKV) & 1u) ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        unsigned char* st = smem + OFF_KV + s * KV_STAGE;
+        const int krow = (b * p.Hkv + g) * p.T_max + j * TILE;
+        mbar_arrive_expect_tx(&ms->kv_full[s], 4 * HALF);
+        tma_load_2d(st, &tmK, 0, krow, &ms->kv_full[s]);
+        tma_load_2d(st + HALF, &tmK, 64, krow, &ms->kv_full[s]);
+        tma_load_2d(st + 2 * HALF, &tmV, 0, krow, &ms->kv_full[s]);
+        tma_load_2d(st + 3 * HALF, &tmV, 64, krow, &ms->kv_full[s]);
+      }
+      if (!ok) {
+        // wait (bounded) for every copy this thread issued before the CTA exits
+        set_status(p.status, ETA_DEVSTAT_TIMEOUT);
+        *abort_flag = 1;
+        mbar_wait(&ms->q_full, 0, nullptr);
+        for (int k = max(0, j - NKV); k < j; ++k)
+          mbar_wait(&ms->kv_full[k % NKV], (uint32_t)(k / NKV) & 1u, nullptr);
+      }
+    }
+  } else if (warp == 2 * NWG + 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(&ms->q_full, 0, abort_flag);
+      const int nX[2] = {nA, nB};
+      const uint32_t qa[2] = {smem_u32(smem + OFF_QA), smem_u32(smem + OFF_QB)};
+      auto issue_qk = [&](int x, int j) -> bool {     // S_X = Q_X K_j^T
+        const int s = j % NKV;
+        if (!mbar_wait(&ms->kv_full[s], (uint32_t)(j / NKV) & 1u, abort_flag)) return false;
+        // S_X's columns hold P_X of the previous key tile until P V has read them
+        if (j > 0 && !mbar_wait(&ms->pv_done[x], (uint32_t)((j - 1) & 1), abort_flag))
+          return false;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(smem + OFF_KV + s * KV_STAGE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * HALF + (uint32_t)(kk & 3) * 32;
+          mma_f16(tS[x], smem_desc(qa[x] + off, 16, 1024, tc::kSwizzle128),
+                  smem_desc(ka + off, 16, 1024, tc::kSwizzle128), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&ms->s_full[x]);
+        return true;
+      };
+      auto issue_pv = [&](int x, int j) -> bool {     // O_X += P_X V_j
+        const int s = j % NKV;
+        if (!mbar_wait(&ms->p_full[x], (uint32_t)(j & 1), abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(smem + OFF_KV + s * KV_STAGE + 2 * HALF);
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) {
+          // keys 16 kk .. 16 kk + 15: half kk / 4 of the row, 8 columns per 16 keys
+          const uint32_t pa = tS[x] + (uint32_t)(kk >> 2) * 64 + (uint32_t)(kk & 3) * 8;
+          mma_f16_ts(tO[x], pa, smem_desc(v0 + kk * 2048, HALF, 1024, tc::kSwizzle128),
+                     kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&ms->pv_done[x]);
+        if (j == nX[x] - 1) mma_commit(&ms->o_final[x]);
+        return true;
+      };
+      // QK of both tiles' first key tile, then per key tile: P V of A, the next QK
+      // of A, P V of B, the next QK of B; a K/V slot is released after its last P V
+      if (ok) ok = issue_qk(0, 0);
+      if (ok && nB > 0) ok = issue_qk(1, 0);
+      for (int j = 0; j < nkv && ok; ++j) {
+        if (j < nA) {
+          ok = issue_pv(0, j);
+          if (ok && j + 1 < nA) ok = issue_qk(0, j + 1);
+        }
+        if (ok && j < nB) ok = issue_pv(1, j);
+        if (ok) mma_commit(&ms->kv_empty[j % NKV]);   // after the last P V of key tile j
+        if (ok && j + 1 < nB) ok = issue_qk(1, j + 1);
+      }
+      if (!ok) {
+        set_status(p.status, ETA_DEVSTAT_TIMEOUT);
+        *abort_flag = 1;
+      }
+      mma_commit(&ms->fin);
+      mbar_wait(&ms->fin, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int x = warp >= NWG ? 1 : 0;                // query tile of this warp
+    const int wl = warp - x * NWG;                    // warp within the tile's group
+    const int hh = wl >> 2;                           // key-column half of the tile
+    const int row = threadIdx.x & (TILE - 1);         // query row of the tile = TMEM lane
+    const int nkx = x == 0 ? nA : nB;
+    const int qx = q0 + x * TILE;
+    const int tq = qx + row;
+    const uint32_t lsel = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t cb = (uint32_t)hh * 64;            // first column of this half
+    const float tau = (tq < p.T_max) ? p.tau[((size_t)b * p.Hq + h) * p.T_max + tq] : 0.f;
+    // raw-unit gate and exponent constants, as in prefill_tc_kernel
+    const float tau_raw = tau / p.scale;
+    const float ta = 0.5f * p.scale * p.invT, tb = 0.5f * tau * p.invT;
+    const float c1 = p.scale * kLog2e;
+    const float resc_raw = kRescale / p.scale;
+    float m_used = -INFINITY;
+    float2 l2 = make_float2(0.f, 0.f), lx2 = make_float2(0.f, 0.f);
+    bool ok = true;
+    auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+    };
+    // the two warps holding the halves of the same rows meet at their own barrier
+    const int pair_bar = 4 + x * 4 + (warp & 3);
+    auto pair_sync = [&] { named_bar_sync(pair_bar, 64); };
+    for (int j = 0; j < nkx; ++j) {
+      const int sb = j & 1, s = j % NKV;
+      const int k0 = j * TILE;
+      if (ok && !wwait(&ms->s_full[x], (uint32_t)(j & 1))) ok = false;
+      float mxh = -INFINITY;
+      if (ok) {
+        // the gated logits go back into the same S_X columns (32 at a time), so that
+        // no thread holds all 64 of them across the row-max exchange
+        tc_fence_after();
+        float pm[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+        auto gate = [&](float v) -> float {
+          if constexpr (HARD) return v >= tau_raw ? v : 0.f;
+          const float hs = 0.5f * v;
+          return fmaf(hs, tanh_approx(fmaf(v, ta, -tb)), hs);
+        };
+        const int lim = (j == nkx - 1) ? tq - k0 - (int)cb : 64;   // diagonal: causal mask
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          float sv[32];
+          tmem_ld32(tS[x] + cb + ch * 32 + lsel, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float y = (ch * 32 + c <= lim) ? gate(sv[c]) : -INFINITY;
+            sv[c] = y;
+            pm[c & 7] = fmaxf(pm[c & 7], y);
+          }
+          tmem_st32(tS[x] + cb + ch * 32 + lsel, sv);
+        }
+        mxh = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                    fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      }
+      ms->xch[x][sb][hh][row] = mxh;
+      pair_sync();
+      const float mx = fmaxf(ms->xch[x][sb][0][row], ms->xch[x][sb][1][row]);
+      if (!ok) continue;
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_used == -INFINITY) {
+        m_used = mx;
+      } else if (mx > m_used + resc_raw) {
+        alpha = ex2_approx((m_used - mx) * c1);
+        m_used = mx;
+        resc = true;
+      }
+      if (__any_sync(0xffffffffu, resc)) {
+        // P V of the previous key tile is complete: QK of this one waited for it
+        float ov[32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(tO[x] + cb + c * 32 + lsel, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+          tmem_st32(tO[x] + cb + c * 32 + lsel, ov);
+        }
+        l2.x *= alpha; l2.y *= alpha;
+        lx2.x *= alpha; lx2.y *= alpha;
+      }
+      // P = e^(scale * (u - m)) as bf16 pairs into the 32 S_X columns this half read,
+      // 16 columns (32 keys) at a time
+      const float nm = -m_used * c1;
+      tmem_wait_st();                                  // the gated logits are in TMEM
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        float sv[32];
+        tmem_ld32(tS[x] + cb + ch * 32 + lsel, sv);
+        tmem_wait_ld();
+        uint32_t pw[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c = 2 * e;
+          const float2 a = __ffma2_rn(make_float2(sv[c], sv[c + 1]), make_float2(c1, c1),
+                                      make_float2(nm, nm));
+          const float p0 = ex2_approx(a.x), p1 = ex2_approx(a.y);
+          const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
+          // the row sum uses the rounded weights the tensor core multiplies
+          l2 = __fadd2_rn(l2, __bfloat1622float2(pr));
+          lx2 = __fadd2_rn(lx2, make_float2(p0, p1));
+          pw[e] = *reinterpret_cast<const uint32_t*>(&pr);
+        }
+        tmem_st16u(tS[x] + cb + ch * 16 + lsel, pw);
+      }
+      // the query tile holding position len - 1 zeroes the V rows past it (its
+      // diagonal key tile is the only one that reaches past the sequence end)
+      if (k0 + TILE > len && k0 + row >= len) {
+        unsigned char* vt = smem + OFF_KV + s * KV_STAGE + 2 * HALF + hh * HALF;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(vt + row * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+        fence_async_smem();
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms->p_full[x]);
+    }
+    if (ok && nkx > 0 && !wwait(&ms->o_final[x], 0u)) ok = false;
+    ms->xsum[x][hh][row] = make_float2(l2.x + l2.y, lx2.x + lx2.y);
+    pair_sync();
+    const float2 s0 = ms->xsum[x][0][row], s1 = ms->xsum[x][1][row];
+    const float l_row = s0.x + s1.x, lx_row = s0.y + s1.y;
+    if (ok && nkx > 0) {
+      tc_fence_after();
+      const float inv = 1.f / l_row;
+      const bool store = tq < len;
+      float* orow = p.O + (((size_t)b * p.Hq + h) * p.T_max + (store ? tq : 0)) * D + cb;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float ov[32];
+        tmem_ld32(tO[x] + cb + c * 32 + lsel, ov);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(orow + c * 32 + i) =
+                make_float4(ov[i] * inv, ov[i + 1] * inv, ov[i + 2] * inv, ov[i + 3] * inv);
+        }
+      }
+      if (store && hh == 0)
+        p.lse[((size_t)b * p.Hq + h) * p.T_max + tq] = p.scale * m_used + logf(lx_row);
+    } else if (!ok) {
+      if (threadIdx.x == 0) set_status(p.status, ETA_DEVSTAT_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2 * NWG + 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
+  }
+}
+
+}  // namespace pp
+
 }  // namespace pf
 
 template <int G>
@@ -465,6 +834,22 @@ static eta_status_t launch_prefill(const CUtensorMap& mq, const CUtensorMap& mk,
   return launch_k(pf::prefill_tc_kernel<G>, dim3(ctas), dim3(pf::NT), pf::SMEM_BYTES, s, mq, mk,
                   mv, prm);
 }
+
+template <int G, bool HARD>
+static eta_status_t launch_prefill_pp(const CUtensorMap& mq, const CUtensorMap& mk,
+                                      const CUtensorMap& mv, pf::PrefillParams prm,
+                                      int B, cudaStream_t s) {
+  using namespace pf;
+  prm.ntiles = (prm.T_max + 2 * TILE - 1) / (2 * TILE);   // query tile pairs
+  const int64_t ctas = (int64_t)B * prm.Hq * prm.ntiles;
+  if (!set_smem_once<pp::prefill_pp_kernel<G, HARD>>(pp::SMEM_BYTES)) return ETA_ERR_CUDA;
+  return launch_k(pp::prefill_pp_kernel<G, HARD>, dim3((unsigned)ctas), dim3(pp::NT),
+                  pp::SMEM_BYTES, s, mq, mk, mv, prm);
+}
+
+// The hard gate takes the two-tile kernel (605 vs 580 TFLOP/s at B = 4, T = 8192 on
+// one B200); the soft gate's extra SFU work and registers make it slower there
+// (452 vs 558), so it keeps the one-tile kernel.
 
 }  // namespace eta
 
@@ -496,6 +881,15 @@ extern "C" eta_status_t eta_prefill(const eta_dims_t* dims, const eta_bf16_t* Q,
   prm.invT = T == 0.f ? -1.f : 1.f / T;
   prm.tau = tau; prm.lengths = lengths; prm.O = O; prm.lse = lse; prm.status = dev_status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (prm.invT < 0.f) {
+    switch (dims->Hq / dims->Hkv) {
+      case 1: return launch_prefill_pp<1, true>(mq, mk, mv, prm, dims->B, s);
+      case 2: return launch_prefill_pp<2, true>(mq, mk, mv, prm, dims->B, s);
+      case 4: return launch_prefill_pp<4, true>(mq, mk, mv, prm, dims->B, s);
+      case 8: return launch_prefill_pp<8, true>(mq, mk, mv, prm, dims->B, s);
+    }
+    return ETA_ERR_UNSUPPORTED;
+  }
   switch (dims->Hq / dims->Hkv) {
     case 1: return launch_prefill<1>(mq, mk, mv, prm, (int)ctas, s);
     case 2: return launch_prefill<2>(mq, mk, mv, prm, (int)ctas, s);

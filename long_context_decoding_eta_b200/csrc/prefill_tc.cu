@@ -114,6 +114,13 @@ ETA_DEV float ex2_approx(float x) {
 }
 constexpr float kLog2e = 1.4426950408889634f;
 
+// max of three values in one instruction (PTX max.f32 with three sources)
+ETA_DEV float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // tanh on the SFU (PTX tanh.approx)
 ETA_DEV float tanh_approx(float x) {
   float y;
@@ -702,19 +709,40 @@ prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
           const float hs = 0.5f * v;
           return fmaf(hs, tanh_approx(fmaf(v, ta, -tb)), hs);
         };
-        const int lim = (j == nkx - 1) ? tq - k0 - (int)cb : 64;   // diagonal: causal mask
+        if (j == nkx - 1) {
+          // the diagonal tile (k0 == qx): keys past the row's query are masked
+          const int lim = tq - k0 - (int)cb;           // columns c <= lim are causal
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          float sv[32];
-          tmem_ld32(tS[x] + cb + ch * 32 + lsel, sv);
-          tmem_wait_ld();
+          for (int ch = 0; ch < 2; ++ch) {
+            float sv[32];
+            tmem_ld32(tS[x] + cb + ch * 32 + lsel, sv);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float y = (ch * 32 + c <= lim) ? gate(sv[c]) : -INFINITY;
-            sv[c] = y;
-            pm[c & 7] = fmaxf(pm[c & 7], y);
+            for (int c = 0; c < 32; c += 2) {
+              const float y0 = (ch * 32 + c <= lim) ? gate(sv[c]) : -INFINITY;
+              const float y1 = (ch * 32 + c + 1 <= lim) ? gate(sv[c + 1]) : -INFINITY;
+              sv[c] = y0;
+              sv[c + 1] = y1;
+              pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], y0, y1);
+            }
+            tmem_st32(tS[x] + cb + ch * 32 + lsel, sv);
           }
-          tmem_st32(tS[x] + cb + ch * 32 + lsel, sv);
+        } else {
+          // every key of an earlier tile precedes every query of this one
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            float sv[32];
+            tmem_ld32(tS[x] + cb + ch * 32 + lsel, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float y0 = gate(sv[c]), y1 = gate(sv[c + 1]);
+              sv[c] = y0;
+              sv[c + 1] = y1;
+              pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], y0, y1);
+            }
+            tmem_st32(tS[x] + cb + ch * 32 + lsel, sv);
+          }
         }
         mxh = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));

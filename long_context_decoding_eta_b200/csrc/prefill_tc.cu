@@ -736,7 +736,20 @@ prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
-              const float y0 = gate(sv[c]), y1 = gate(sv[c + 1]);
+              float y0, y1;
+              if constexpr (HARD) {
+                // s * [s >= tau / scale]: a 1.0 / 0.0 flag per score (set.ge) and one
+                // packed multiply for two scores (S is finite)
+                float g0, g1;
+                asm("set.ge.f32.f32 %0, %1, %2;" : "=f"(g0) : "f"(sv[c]), "f"(tau_raw));
+                asm("set.ge.f32.f32 %0, %1, %2;" : "=f"(g1) : "f"(sv[c + 1]), "f"(tau_raw));
+                const float2 y = __fmul2_rn(make_float2(sv[c], sv[c + 1]), make_float2(g0, g1));
+                y0 = y.x;
+                y1 = y.y;
+              } else {
+                y0 = gate(sv[c]);
+                y1 = gate(sv[c + 1]);
+              }
               sv[c] = y0;
               sv[c + 1] = y1;
               pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], y0, y1);

@@ -708,7 +708,8 @@ def run_prefill(args, rank, world, device):
             "config": {"workload": f"prefill-b{B}-h{Hq}x{Hkv}-d{d}-T{T}-causal",
                        "gate_T": args.pf_gate_T},
             "roofline": {"kernel": ("prefill_pp_kernel (two query tiles per CTA)"
-                                    if args.pf_gate_T == 0.0 else "prefill_tc_kernel"),
+                                    if L.eta_prefill_kernel_for(dims, args.pf_gate_T) == "two_tile"
+                                    else "prefill_tc_kernel"),
                          "bound": "tensor", "achieved": tf,
                          "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
                          "peak_kind": "measured cuBLAS bf16 burst"},

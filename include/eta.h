@@ -355,6 +355,30 @@ eta_status_t eta_prefill(const eta_dims_t* dims, const eta_bf16_t* Q, const floa
                          void* stream);
 
 /*
+ * Prefill kernel (process-wide; both compute the same function, both are tested
+ * against the float64 oracle):
+ *   ETA_PREFILL_ONE_TILE -- one CTA per (row, query head, 128-query tile)
+ *   ETA_PREFILL_TWO_TILE -- one CTA per (row, query head, pair of 128-query tiles);
+ *                           every K/V tile serves both, P stays in tensor memory
+ *   ETA_PREFILL_AUTO     -- the default: the two-tile kernel once its tile pairs
+ *                           (B * Hq * ceil(T_max / 256)) exceed half the SM count with
+ *                           the hard gate, twice the SM count with the soft gate (the
+ *                           sizes from which this library measures it faster)
+ * eta_set_prefill_kernel returns ETA_ERR_INVALID_ARG for an unknown value.
+ * eta_prefill_kernel_for returns the kernel (ETA_PREFILL_ONE_TILE or _TWO_TILE) that
+ * eta_prefill would launch for these dims and gate temperature T under the current
+ * setting (host only, no device work; -1 for dims or T that eta_prefill refuses).
+ */
+typedef enum {
+  ETA_PREFILL_AUTO = 0,
+  ETA_PREFILL_ONE_TILE = 1,
+  ETA_PREFILL_TWO_TILE = 2
+} eta_prefill_kernel_t;
+eta_status_t eta_set_prefill_kernel(eta_prefill_kernel_t kernel);
+eta_prefill_kernel_t eta_get_prefill_kernel(void);
+int32_t eta_prefill_kernel_for(const eta_dims_t* dims, float T);
+
+/*
  * eta_calibrate_const_tau -- offline calibration of frozen per-head thresholds
  * (abstract: "an offline calibration algorithm ... that freezes per-head constant
  * thresholds").  HOST pointers.  The pages do not print the algorithm; the rule

@@ -32,8 +32,10 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_set_decode_engine", "eta_get_decode_engine", "eta_decode_static",
            "eta_decode_static_max_workspace", "eta_selftest_wait_timeout", "eta_prefill",
            "eta_decode_step_workspace_size", "eta_decode_step", "eta_lse_merge",
-           "eta_append_and_predict_tau", "eta_screen_launches", "eta_decode_launches")
+           "eta_append_and_predict_tau", "eta_screen_launches", "eta_decode_launches",
+           "eta_set_prefill_kernel", "eta_get_prefill_kernel", "eta_prefill_kernel_for")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
+PREFILL_KERNEL = {"auto": 0, "one_tile": 1, "two_tile": 2}
 
 
 class EtaError(RuntimeError):
@@ -113,6 +115,12 @@ def lib() -> C.CDLL:
     L.eta_set_decode_engine.restype = I32
     L.eta_get_decode_engine.argtypes = []
     L.eta_get_decode_engine.restype = I32
+    L.eta_set_prefill_kernel.argtypes = [I32]
+    L.eta_set_prefill_kernel.restype = I32
+    L.eta_get_prefill_kernel.argtypes = []
+    L.eta_get_prefill_kernel.restype = I32
+    L.eta_prefill_kernel_for.argtypes = [DIMS, F32]
+    L.eta_prefill_kernel_for.restype = I32
     for name in ("eta_build_block_meta", "eta_predict_tau", "eta_screen", "eta_decode",
                  "eta_dense_decode", "eta_calibrate_const_tau", "eta_status_from_device"):
         getattr(L, name).restype = I32
@@ -284,6 +292,26 @@ def eta_set_decode_engine(engine) -> None:
 def eta_get_decode_engine() -> str:
     v = int(lib().eta_get_decode_engine())
     return {k: n for n, k in ENGINE.items()}.get(v, str(v))
+
+
+def eta_set_prefill_kernel(kernel) -> None:
+    """kernel: "auto" | "one_tile" | "two_tile" (or the integer value)."""
+    _check("eta_set_prefill_kernel", lib().eta_set_prefill_kernel(
+        PREFILL_KERNEL[kernel] if isinstance(kernel, str) else int(kernel)))
+
+
+def eta_get_prefill_kernel() -> str:
+    v = int(lib().eta_get_prefill_kernel())
+    return {k: n for n, k in PREFILL_KERNEL.items()}.get(v, str(v))
+
+
+def eta_prefill_kernel_for(dims: Dims, T: float) -> str:
+    """The kernel eta_prefill would launch for these dims and gate T ("one_tile" or
+    "two_tile"); raises EtaError(INVALID_ARG) for dims or T that eta_prefill refuses."""
+    v = int(lib().eta_prefill_kernel_for(C.byref(dims), float(T)))
+    if v < 0:
+        raise EtaError("eta_prefill_kernel_for", 1)
+    return {k: n for n, k in PREFILL_KERNEL.items()}[v]
 
 
 def eta_selftest_wait_timeout(wait_limit: int, never_set, dev_status, stream=None) -> None:

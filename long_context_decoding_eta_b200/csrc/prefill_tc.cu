@@ -19,10 +19,12 @@
 //           own 64 columns; P is written as bf16 into a swizzled shared tile (the A
 //           operand of P V), each half writing its own 64-key half.
 // TMEM: S 2 x 128 columns, O 128 columns (512 allocated).  Every wait is bounded.
-// This one-tile kernel serves the soft gate; the hard gate takes the two-tile kernel
-// further down (prefill_pp_kernel: two query tiles per CTA sharing every K/V tile,
-// P kept in tensor memory), which measured faster for it.
+// The two-tile kernel further down (prefill_pp_kernel: two query tiles per CTA
+// sharing every K/V tile, P kept in tensor memory) is faster wherever its tile pairs
+// fill the SMs; this one-tile kernel takes the small launches (see eta_prefill).
 #include <cuda.h>
+#include <algorithm>
+#include <atomic>
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -888,9 +890,21 @@ static eta_status_t launch_prefill_pp(const CUtensorMap& mq, const CUtensorMap& 
                   pp::SMEM_BYTES, s, mq, mk, mv, prm);
 }
 
-// The hard gate takes the two-tile kernel (605 vs 580 TFLOP/s at B = 4, T = 8192 on
-// one B200); the soft gate's extra SFU work and registers make it slower there
-// (452 vs 558), so it keeps the one-tile kernel.
+std::atomic<int> g_prefill_kernel{ETA_PREFILL_AUTO};
+
+// Which kernel eta_prefill launches.  Measured on one B200 (16 / 4 heads, d = 128):
+// the two-tile kernel is faster once its tile pairs fill the SMs (B = 4, T = 8192:
+// 742 vs 580 TFLOP/s hard gate, 626 vs 559 soft), but it has half as many CTAs, each
+// twice as long, so on small launches idle SMs and the longest pair decide: at 64
+// pairs (B = 1, T = 1024) it takes 32 vs 22 us; at 256 pairs (B = 1, T = 4096) it still
+// wins with the hard gate (158 vs 164 us) and loses with the soft gate (186 vs 170 us).
+inline bool prefill_two_tile(const eta_dims_t* d, bool hard) {
+  const int k = g_prefill_kernel.load();
+  if (k != ETA_PREFILL_AUTO) return k == ETA_PREFILL_TWO_TILE;
+  const int64_t pairs = (int64_t)d->B * d->Hq * ((d->T_max / pf::TILE + 1) / 2);
+  const int64_t n = std::max(sm_count(), 1);
+  return hard ? pairs > n / 2 : pairs > 2 * n;
+}
 
 }  // namespace eta
 
@@ -922,12 +936,17 @@ extern "C" eta_status_t eta_prefill(const eta_dims_t* dims, const eta_bf16_t* Q,
   prm.invT = T == 0.f ? -1.f : 1.f / T;
   prm.tau = tau; prm.lengths = lengths; prm.O = O; prm.lse = lse; prm.status = dev_status;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (prm.invT < 0.f) {
-    switch (dims->Hq / dims->Hkv) {
+  const bool hard = prm.invT < 0.f;
+  if (prefill_two_tile(dims, hard)) {
+    switch ((dims->Hq / dims->Hkv) * (hard ? 1 : -1)) {
       case 1: return launch_prefill_pp<1, true>(mq, mk, mv, prm, dims->B, s);
       case 2: return launch_prefill_pp<2, true>(mq, mk, mv, prm, dims->B, s);
       case 4: return launch_prefill_pp<4, true>(mq, mk, mv, prm, dims->B, s);
       case 8: return launch_prefill_pp<8, true>(mq, mk, mv, prm, dims->B, s);
+      case -1: return launch_prefill_pp<1, false>(mq, mk, mv, prm, dims->B, s);
+      case -2: return launch_prefill_pp<2, false>(mq, mk, mv, prm, dims->B, s);
+      case -4: return launch_prefill_pp<4, false>(mq, mk, mv, prm, dims->B, s);
+      case -8: return launch_prefill_pp<8, false>(mq, mk, mv, prm, dims->B, s);
     }
     return ETA_ERR_UNSUPPORTED;
   }
@@ -938,4 +957,22 @@ extern "C" eta_status_t eta_prefill(const eta_dims_t* dims, const eta_bf16_t* Q,
     case 8: return launch_prefill<8>(mq, mk, mv, prm, (int)ctas, s);
   }
   return ETA_ERR_UNSUPPORTED;
+}
+
+extern "C" eta_status_t eta_set_prefill_kernel(eta_prefill_kernel_t kernel) {
+  if (kernel != ETA_PREFILL_AUTO && kernel != ETA_PREFILL_ONE_TILE &&
+      kernel != ETA_PREFILL_TWO_TILE)
+    return ETA_ERR_INVALID_ARG;
+  g_prefill_kernel.store((int)kernel);
+  return ETA_OK;
+}
+
+extern "C" eta_prefill_kernel_t eta_get_prefill_kernel(void) {
+  return static_cast<eta_prefill_kernel_t>(g_prefill_kernel.load());
+}
+
+extern "C" int32_t eta_prefill_kernel_for(const eta_dims_t* dims, float T) {
+  if (check_dims(dims, /*rows_in_grid_y=*/false) != ETA_OK) return -1;
+  if (!(T >= 0.f) || isinf(T) || dims->d != 128 || dims->T_max % pf::TILE != 0) return -1;
+  return prefill_two_tile(dims, T == 0.f) ? ETA_PREFILL_TWO_TILE : ETA_PREFILL_ONE_TILE;
 }

@@ -95,6 +95,27 @@ def test_argument_validation_without_gpu():
     assert lib.eta_decode_launches(ctypes.byref(dims)) in (2, 3)
 
 
+def test_prefill_kernel_selection_host_only():
+    assert L.eta_get_prefill_kernel() == "auto"
+    dims = L.Dims.of(4, 16, 4, 128, 64, 8192)
+    for k in ("one_tile", "two_tile"):
+        L.eta_set_prefill_kernel(k)
+        assert L.eta_get_prefill_kernel() == k
+        assert L.eta_prefill_kernel_for(dims, 0.0) == k
+        assert L.eta_prefill_kernel_for(dims, 0.05) == k
+    L.eta_set_prefill_kernel("auto")
+    with pytest.raises(L.EtaError):
+        L.eta_set_prefill_kernel(5)
+    assert L.eta_get_prefill_kernel() == "auto"
+    # shapes eta_prefill refuses are refused by the query too
+    for bad in (L.Dims.of(4, 16, 4, 64, 64, 8192), L.Dims.of(4, 16, 4, 128, 64, 8256),
+                L.Dims.of(4, 16, 5, 128, 64, 8192)):
+        with pytest.raises(L.EtaError):
+            L.eta_prefill_kernel_for(bad, 0.0)
+    with pytest.raises(L.EtaError):
+        L.eta_prefill_kernel_for(dims, -1.0)
+
+
 def test_engine_selection_host_only():
     assert L.eta_get_decode_engine() == "auto"
     L.eta_set_decode_engine("fma")

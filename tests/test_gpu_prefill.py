@@ -13,6 +13,14 @@ from oracle import eta_oracle as O
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True, params=["one_tile", "two_tile"])
+def prefill_kernel(request):
+    """Every case runs through both prefill kernels."""
+    L.eta_set_prefill_kernel(request.param)
+    yield request.param
+    L.eta_set_prefill_kernel("auto")
+
+
 def run_case(B, Hq, Hkv, T_max, lengths, T_gate, seed, q_gain=1.0, tau_mu=0.5):
     g = torch.Generator().manual_seed(seed)
     d = 128
@@ -129,3 +137,17 @@ def test_prefill_fullsize_sampled_rows():
             checked += 1
         e = np.stack(errs)
         assert checked >= 24 and e.max() <= 1e-2 and e.mean() <= 1e-3, (checked, e.max(), e.mean())
+
+
+def test_prefill_auto_kernel_choice(prefill_kernel):
+    """The automatic choice: the two-tile kernel once its tile pairs exceed half the SM
+    count (hard gate) or twice the SM count (soft gate)."""
+    L.eta_set_prefill_kernel("auto")
+    n = torch.cuda.get_device_properties(0).multi_processor_count
+    for B, Hq, T in [(1, 16, 1024), (1, 16, 2048), (1, 16, 4096), (2, 16, 4096), (4, 16, 8192)]:
+        pairs = B * Hq * ((T // 128 + 1) // 2)
+        dims = L.Dims.of(B, Hq, 4, 128, 64, T)
+        assert L.eta_prefill_kernel_for(dims, 0.0) == ("two_tile" if pairs > n // 2 else "one_tile")
+        assert L.eta_prefill_kernel_for(dims, 0.05) == ("two_tile" if pairs > 2 * n else "one_tile")
+    # the prefill benchmark's configuration takes the two-tile kernel with both gates
+    assert L.eta_prefill_kernel_for(L.Dims.of(4, 16, 4, 128, 64, 8192), 0.05) == "two_tile"

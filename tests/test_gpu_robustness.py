@@ -99,8 +99,17 @@ def test_fused_step_cache_past_lengths_poisoned():
     print(compare_step(gpu, tau, sc, o, lse, q64, K64, V64, Lr, w.blk, scale, 0.0, w.G))
 
 
+@pytest.mark.parametrize("kernel", ["one_tile", "two_tile"])
 @pytest.mark.parametrize("T_gate", [0.0, 0.05])
-def test_prefill_past_lengths_poisoned(T_gate):
+def test_prefill_past_lengths_poisoned(T_gate, kernel):
+    L.eta_set_prefill_kernel(kernel)
+    try:
+        _prefill_past_lengths_poisoned(T_gate)
+    finally:
+        L.eta_set_prefill_kernel("auto")
+
+
+def _prefill_past_lengths_poisoned(T_gate):
     B, Hq, Hkv, T_max, d = 2, 8, 2, 384, 128
     gen = torch.Generator().manual_seed(303)
     q = torch.randn(B, Hq, T_max, d, generator=gen).to(torch.bfloat16)

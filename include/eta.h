@@ -51,7 +51,8 @@ typedef enum {
   ETA_ERR_WORKSPACE = 3,       /* workspace NULL or smaller than the query says */
   ETA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed */
   ETA_ERR_DEVICE_TIMEOUT = 5,  /* returned by eta_status_from_device() */
-  ETA_ERR_NONFINITE = 6        /* returned by eta_status_from_device() */
+  ETA_ERR_NONFINITE = 6,       /* returned by eta_status_from_device() */
+  ETA_ERR_DEVICE_BOUNDS = 7    /* returned by eta_status_from_device(): checked build */
 } eta_status_t;
 
 /* Bits OR-ed into *dev_status by the kernels. */
@@ -59,6 +60,12 @@ typedef enum {
 #define ETA_DEVSTAT_NONFINITE_Q 0x2  /* a query element was NaN or Inf */
 #define ETA_DEVSTAT_BAD_BLOCK 0x4    /* a block index out of range or an empty block */
 #define ETA_DEVSTAT_BAD_LENGTH 0x8   /* lengths[b] < 0 or > T_max (clamped) */
+/* Checked build only (libeta_checked.so, compiled with -DETA_CHECKED): an index that
+   a kernel computed for a global load or store fell outside its buffer; that access
+   was skipped, the outputs are invalid, and the first such event of each source file
+   is printed (device printf) with its file and line.  A library defect, never an
+   input error: the host-side checks refuse every input that could cause one. */
+#define ETA_DEVSTAT_BOUNDS 0x10
 
 typedef struct {
   int32_t B;      /* batch rows (decode queries) */
@@ -404,6 +411,23 @@ eta_status_t eta_calibrate_const_tau(const float* bounds, const uint8_t* valid,
  */
 eta_status_t eta_selftest_wait_timeout(uint32_t wait_limit, const int32_t* never_set,
                                        int32_t* dev_status, void* stream);
+
+/*
+ * eta_build_checked -- 1 in the checked build (libeta_checked.so: every global access
+ * whose index a kernel computes is range-checked first, see ETA_DEVSTAT_BOUNDS), 0 in
+ * the release build (libeta.so).  Both builds export the same entry points and
+ * compute the same outputs; the checked one is a debugging aid (compute-sanitizer's
+ * memcheck is not assumed to be available).
+ *
+ * eta_selftest_bounds -- diagnostic of the checked build: launches one thread that
+ * runs the range check on (index, extent) without any memory access.  The checked
+ * build ORs ETA_DEVSTAT_BOUNDS into *dev_status (device memory) when index lies
+ * outside [0, extent); the release build compiles the check away and writes nothing.
+ * extent < 0 or dev_status NULL: ETA_ERR_INVALID_ARG.
+ */
+int32_t eta_build_checked(void);
+eta_status_t eta_selftest_bounds(int64_t index, int64_t extent, int32_t* dev_status,
+                                 void* stream);
 
 /* Maps a device status word (read back by the caller) to a status code. */
 eta_status_t eta_status_from_device(int32_t dev_status);

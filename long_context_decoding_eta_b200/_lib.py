@@ -3,7 +3,10 @@ function per entry point with the same name.  Argument marshalling only: torch
 tensors are turned into device pointers, and every non-OK status raises.
 
 The library must be built (python -m long_context_decoding_eta_b200.build); there
-is no fallback of any kind when it is missing.
+is no fallback of any kind when it is missing.  With ETA_CHECKED=1 in the
+environment the range-checked build (libeta_checked.so, `build --checked`) is
+loaded instead: same entry points, same outputs, every computed global index
+checked on the device (include/eta.h, ETA_DEVSTAT_BOUNDS).
 """
 from __future__ import annotations
 
@@ -14,17 +17,20 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libeta.so")
+LIB_PATH = os.path.join(
+    _HERE, "libeta_checked.so" if os.environ.get("ETA_CHECKED") == "1" else "libeta.so")
 
 ETA_OK = 0
 STATUS_NAMES = {0: "ok", 1: "invalid argument", 2: "unsupported shape",
                 3: "workspace missing or too small", 4: "CUDA error",
-                5: "device wait timed out", 6: "non-finite query"}
+                5: "device wait timed out", 6: "non-finite query",
+                7: "out-of-range index (checked build)"}
 BOUND = {"exact": 0, "prob": 1, "prob_dim": 2}
 CENT = {"f32": 0, "bf16": 1}
 PRUNE = {"skip": 0, "floor": 1}
 TAIL_BLOCK = -1
 DEVSTAT_TIMEOUT, DEVSTAT_NONFINITE_Q, DEVSTAT_BAD_BLOCK, DEVSTAT_BAD_LENGTH = 1, 2, 4, 8
+DEVSTAT_BOUNDS = 0x10
 
 EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size",
            "eta_screen", "eta_decode_workspace_size", "eta_decode", "eta_dense_decode",
@@ -33,7 +39,8 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_decode_static_max_workspace", "eta_selftest_wait_timeout", "eta_prefill",
            "eta_decode_step_workspace_size", "eta_decode_step", "eta_lse_merge",
            "eta_append_and_predict_tau", "eta_screen_launches", "eta_decode_launches",
-           "eta_set_prefill_kernel", "eta_get_prefill_kernel", "eta_prefill_kernel_for")
+           "eta_set_prefill_kernel", "eta_get_prefill_kernel", "eta_prefill_kernel_for",
+           "eta_build_checked", "eta_selftest_bounds")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 PREFILL_KERNEL = {"auto": 0, "one_tile": 1, "two_tile": 2}
 
@@ -121,6 +128,10 @@ def lib() -> C.CDLL:
     L.eta_get_prefill_kernel.restype = I32
     L.eta_prefill_kernel_for.argtypes = [DIMS, F32]
     L.eta_prefill_kernel_for.restype = I32
+    L.eta_build_checked.argtypes = []
+    L.eta_build_checked.restype = I32
+    L.eta_selftest_bounds.argtypes = [C.c_int64, C.c_int64, P, P]
+    L.eta_selftest_bounds.restype = I32
     for name in ("eta_build_block_meta", "eta_predict_tau", "eta_screen", "eta_decode",
                  "eta_dense_decode", "eta_calibrate_const_tau", "eta_status_from_device"):
         getattr(L, name).restype = I32
@@ -312,6 +323,17 @@ def eta_prefill_kernel_for(dims: Dims, T: float) -> str:
     if v < 0:
         raise EtaError("eta_prefill_kernel_for", 1)
     return {k: n for n, k in PREFILL_KERNEL.items()}[v]
+
+
+def eta_build_checked() -> bool:
+    """True when the loaded library is the range-checked build."""
+    return bool(lib().eta_build_checked())
+
+
+def eta_selftest_bounds(index: int, extent: int, dev_status, stream=None) -> None:
+    """Runs the checked build's range check on (index, extent) (see include/eta.h)."""
+    _check("eta_selftest_bounds", lib().eta_selftest_bounds(
+        int(index), int(extent), _p(dev_status), _stream(stream)))
 
 
 def eta_selftest_wait_timeout(wait_limit: int, never_set, dev_status, stream=None) -> None:

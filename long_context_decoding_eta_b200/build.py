@@ -1,9 +1,12 @@
 """Builds libeta.so (the ETA C-ABI library) in-tree for sm_100a with nvcc.
 
-    python -m long_context_decoding_eta_b200.build [--verbose]
+    python -m long_context_decoding_eta_b200.build [--verbose] [--checked]
 
 Objects are compiled in parallel into `_build/` next to this file and linked
 into `long_context_decoding_eta_b200/libeta.so`.  Rebuilds only what changed.
+`--checked` builds the range-checked debugging variant instead (-DETA_CHECKED,
+objects in `_build_checked/`, library `libeta_checked.so`), which the binding
+loads when the environment sets ETA_CHECKED=1.
 """
 from __future__ import annotations
 
@@ -18,6 +21,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libeta.so")
+BUILD_CHECKED = os.path.join(HERE, "_build_checked")
+LIB_CHECKED = os.path.join(HERE, "libeta_checked.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -38,12 +43,13 @@ def _headers_mtime():
     return max(os.path.getmtime(h) for h in hs)
 
 
-def _compile(src: str, verbose: bool, extra=()):
+def _compile(src: str, verbose: bool, checked: bool = False):
     path = os.path.join(CSRC, src)
-    obj = os.path.join(BUILD, src + ".o")
+    obj = os.path.join(BUILD_CHECKED if checked else BUILD, src + ".o")
     if (os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(path)
-            and os.path.getmtime(obj) >= _headers_mtime() and not extra):
+            and os.path.getmtime(obj) >= _headers_mtime()):
         return obj, ""
+    extra = ["-DETA_CHECKED"] if checked else []
     cmd = [NVCC, *ARCH, *CUFLAGS, *extra, "-c", path, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -53,11 +59,13 @@ def _compile(src: str, verbose: bool, extra=()):
     return obj, p.stdout + p.stderr
 
 
-def build(verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose: bool = False, checked: bool = False) -> str:
+    """Builds libeta.so, or libeta_checked.so with checked=True; returns its path."""
+    lib_path = LIB_CHECKED if checked else LIB
+    os.makedirs(BUILD_CHECKED if checked else BUILD, exist_ok=True)
     cu, cpp = _sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        futs = [ex.submit(_compile, s, verbose) for s in cu + cpp]
+        futs = [ex.submit(_compile, s, verbose, checked) for s in cu + cpp]
         objs = []
         for f in futs:
             obj, log = f.result()
@@ -65,17 +73,18 @@ def build(verbose: bool = False) -> str:
             if verbose and log:
                 print(log)
     newest = max(os.path.getmtime(o) for o in objs)
-    if not os.path.exists(LIB) or os.path.getmtime(LIB) < newest:
-        cmd = [NVCC, *ARCH, "-shared", "-o", LIB, *objs, "-lcudart"]
+    if not os.path.exists(lib_path) or os.path.getmtime(lib_path) < newest:
+        cmd = [NVCC, *ARCH, "-shared", "-o", lib_path, *objs, "-lcudart"]
         p = subprocess.run(cmd, capture_output=True, text=True)
         if p.returncode != 0:
             raise RuntimeError(f"link failed:\n{p.stdout}\n{p.stderr}")
-    return LIB
+    return lib_path
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--checked", action="store_true")
     a = ap.parse_args()
-    print(build(a.verbose))
+    print(build(a.verbose, a.checked))
     sys.exit(0)

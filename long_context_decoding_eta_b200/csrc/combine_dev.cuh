@@ -25,6 +25,7 @@ struct CombineParams {
   const float* part_ml;
   float* o;
   float* lse;
+  int32_t* status;   // the checked build's range reports (may be NULL)
 };
 
 constexpr int kCombineMaxPairs = 256;   // (head, slot) pairs staged in shared memory
@@ -43,15 +44,18 @@ ETA_DEV float ld_part(const float* p) {
 }
 
 // Called by D threads (thread = dim dd) that `sync` synchronizes.  Slot s of pair r
-// and head h lives at ((p0 + s) + r) * G + h.  On return O[h] holds this dim's
-// un-normalized merged output, sc.M[h] / sc.L[h] the merged max and sum
+// and head h lives at ((p0 + s) + r) * G + h, of n_slots slots.  On return O[h] holds
+// this dim's un-normalized merged output, sc.M[h] / sc.L[h] the merged max and sum
 // (-inf / 0 when ns = 0).  CG: the partials were written by other CTAs of the
 // same grid (L2-coherent loads).
 template <int D, int G, bool CG, typename Sync>
 ETA_DEV void combine_merge(const float* part_ml, const float* part_o, int r, int p0, int ns,
-                           int dd, CombineScratch<G>& sc, float (&O)[G], Sync sync) {
+                           int dd, CombineScratch<G>& sc, float (&O)[G], Sync sync,
+                           long long n_slots, int32_t* status) {
 #pragma unroll
   for (int h = 0; h < G; ++h) O[h] = 0.f;
+  // (checked build) the pair's slots lie inside the workspace; uniform over the callers
+  if (!ETA_RANGE_IN_BOUNDS((long long)p0 + r, (long long)p0 + r + ns, n_slots, status)) ns = 0;
   if (ns > 0) {
     const int np = G * ns;                 // pair k = slot * G + h
     if (np <= kCombineMaxPairs) {

@@ -20,12 +20,13 @@ struct CompactScratch {
 
 // All NT threads of the CTA call this (it synchronises the CTA).  union_words and
 // head_mask: [R][NW] and [B * Hq][NW]; writes union_idx[r * NB ...], union_cnt[r]
-// and, if given, head_cnt of the pair's G query heads.
+// and, if given, head_cnt of the pair's G query heads.  status: the checked build's
+// range reports (may be NULL).
 template <int NT>
 ETA_DEV void compact_row(int r, int Hq, int Hkv, int G, int NB, int NW,
                          const uint32_t* union_words, const uint32_t* head_mask,
                          int32_t* union_idx, int32_t* union_cnt, int32_t* head_cnt,
-                         CompactScratch<NT>& cs) {
+                         CompactScratch<NT>& cs, int32_t* status) {
   static_assert(NT % 32 == 0 && NT <= 1024, "NT");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int carry = 0;
@@ -53,9 +54,9 @@ ETA_DEV void compact_row(int r, int Hq, int Hkv, int G, int NB, int NW,
     __syncthreads();
     for (int i = warp; i < NT && base + i < NW; i += NT / 32) {
       const uint32_t wd = cs.wbuf[i];
-      if ((wd >> lane) & 1u)
-        union_idx[(size_t)r * NB + cs.woff[i] + __popc(wd & ((1u << lane) - 1u))] =
-            (base + i) * 32 + lane;
+      const int pos = cs.woff[i] + __popc(wd & ((1u << lane) - 1u));
+      if (((wd >> lane) & 1u) && ETA_IN_BOUNDS(pos, NB, status))
+        union_idx[(size_t)r * NB + pos] = (base + i) * 32 + lane;
     }
     carry += total;
     __syncthreads();

@@ -47,6 +47,8 @@ struct StageInfo {
 
 struct DecodeParams {
   int Hq, Hkv, T_max, NB, blk;
+  int R;               // (row, KV head) pairs
+
   float scale, invT;   // invT < 0 selects the hard gate
   const eta_bf16_t* q;
   const float* tau;
@@ -137,14 +139,26 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_kernel(const DecodeP
   if (warp == NCW) {
     if (lane != 0) return;
     int r = p.cta_row[blockIdx.x];
+    bool ok = true;
+    if (!ETA_IN_BOUNDS(r, p.R, p.status)) {   // checked build: give up like a lost wait
+      r = 0;
+      ok = false;
+    }
     int roff = p.row_off[r], rend = p.row_off[r + 1];
     int it = 0;
-    bool ok = true;
     for (int pos = a; pos < e && ok; ++pos) {
       while (pos >= rend) {
+        if (!ETA_IN_BOUNDS(r + 2, p.R + 1, p.status)) {
+          ok = false;
+          break;
+        }
         ++r;
         roff = rend;
         rend = p.row_off[r + 1];
+      }
+      if (!ok || (!DENSE && !ETA_IN_BOUNDS(pos - roff, p.NB, p.status))) {
+        ok = false;
+        break;
       }
       const int b = r / p.Hkv;
       const int len = min(max(p.lengths[b], 0), p.T_max);
@@ -212,7 +226,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1) decode_kernel(const DecodeP
     }
     named_bar_sync(1, NCW * 32);
     const size_t slot = (size_t)blockIdx.x + row;
-    for (int idx = threadIdx.x; idx < G * D; idx += NCW * 32) {
+    const bool slot_ok = ETA_IN_BOUNDS(slot, (long long)gridDim.x + p.R, p.status);
+    for (int idx = threadIdx.x; idx < G * D && slot_ok; idx += NCW * 32) {
       const int h = idx / D, dd = idx % D;
       float M = -INFINITY;
 #pragma unroll
@@ -421,7 +436,9 @@ __global__ void __launch_bounds__(D) combine_kernel(const CombineParams p) {
   __shared__ int s_nfloor;
   const int r = blockIdx.x, b = r / p.Hkv, g = r % p.Hkv;
   const int dd = threadIdx.x;
-  const int off = p.row_off[r], c = p.row_off[r + 1] - off;
+  const int off = p.row_off[r];
+  int c = p.row_off[r + 1] - off;
+  if (!ETA_IN_BOUNDS(c, p.NB + 1, p.status)) c = 0;   // checked build: a pair's list fits its row
   const int chunk = p.plan[1];
   float fv = 0.f;
   int nfloor = 0;
@@ -450,7 +467,8 @@ __global__ void __launch_bounds__(D) combine_kernel(const CombineParams p) {
   const int p0 = c > 0 ? off / chunk : 0;
   const int ns = c > 0 ? (off + c - 1) / chunk - p0 + 1 : 0;
   float O[G];
-  combine_merge<D, G, false>(p.part_ml, p.part_o, r, p0, ns, dd, sc, O, [] { __syncthreads(); });
+  combine_merge<D, G, false>(p.part_ml, p.part_o, r, p0, ns, dd, sc, O, [] { __syncthreads(); },
+                             (long long)p.P + gridDim.x, p.status);
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     float M = sc.M[h], L = sc.L[h], Oh = O[h];
@@ -643,6 +661,7 @@ eta_status_t run_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float
   prm.q = q; prm.tau = tau; prm.K = K; prm.V = V; prm.lengths = lengths;
   prm.union_idx = union_idx; prm.row_off = row_off; prm.cta_row = cta_row; prm.plan = plan;
   prm.part_o = part_o; prm.part_ml = part_ml; prm.status = dev_status;
+  prm.R = R;
   st = use_tc(dims) ? launch_tc<DENSE>(dims, prm, q, K, V, P, plan_in, union_cnt, s)
                     : launch_decode<DENSE>(dims, prm, P, s);
   if (st != ETA_OK) return st;
@@ -652,6 +671,7 @@ eta_status_t run_decode(const eta_dims_t* dims, const eta_bf16_t* q, const float
   cp.P = P; cp.floor_mode = (!DENSE && prune == ETA_PRUNE_FLOOR) ? 1 : 0;
   cp.row_off = row_off; cp.plan = plan; cp.union_idx = union_idx; cp.lengths = lengths;
   cp.cnt = cnt; cp.vsum = vsum; cp.part_o = part_o; cp.part_ml = part_ml; cp.o = o; cp.lse = lse;
+  cp.status = dev_status;
   return launch_combine(dims, cp, s);
 }
 

@@ -349,13 +349,18 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       int r = (LOCAL || PLAN_IN) ? cta_row[0] : cta_row[blockIdx.x];
+      bool ok = true;
+      if (!ETA_IN_BOUNDS(r, p.R, p.status)) {   // checked build: give up like a lost wait
+        r = 0;
+        ok = false;
+      }
       int roff = row_off[r], rend = row_off[r + 1];
       int it = 0;
-      bool ok = true;
       int pend_row = -1, pend_t0 = 0, pend_nv = 0;   // a lone sub-tile waiting for a partner
       auto emit = [&](int row, int t0a, int nva, int t0b, int nvb, int flags) -> bool {
         const int s = it % NSTAGE;
         const uint32_t ph = (uint32_t)(it / NSTAGE) & 1u;
+        if (!flags && !ETA_IN_BOUNDS(row, p.R, p.status)) return false;
         if (!mbar_wait(&ms->empty[s], ph ^ 1u, abort_flag)) return false;
         ms->info[s] = TcStage{row, {t0a, t0b}, {nva, nvb}, flags, {0, 0}};
         unsigned char* st = smem + s * STAGE_BYTES;
@@ -402,12 +407,16 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
       // are emitted, so its L2 latency overlaps the wait for a free stage.
       auto fetch = [&](int pos, int& rr, int& ro, int& re) -> int {
         while (pos >= re) {
+          if (!ETA_IN_BOUNDS(rr + 2, p.R + 1, p.status)) {
+            rows_ok = false;
+            return 0;
+          }
           ++rr;
           ro = re;
           re = row_off[rr + 1];
         }
         if (DENSE) return pos - ro;
-        if (!row_ready(rr)) {
+        if (!row_ready(rr) || !ETA_IN_BOUNDS(pos - ro, p.NB, p.status)) {
           rows_ok = false;
           return 0;
         }
@@ -566,8 +575,9 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
         named_bar_sync(1, NWARP_SM * 32);
       } else {
         const size_t slot = (size_t)blockIdx.x + row;
+        const bool slot_ok = ETA_IN_BOUNDS(slot, (long long)gridDim.x + p.R, p.status);
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < G && slot_ok; ++h) {
           p.part_o[(slot * G + h) * D + t] = o_acc[h];
           if (t == 0) {
             float L = 0.f;
@@ -596,7 +606,8 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
             CombineScratch<G>& cs = *reinterpret_cast<CombineScratch<G>*>(&fs->cs);
             float O[G];
             combine_merge<D, G, true>(p.part_ml, p.part_o, row, p0, ns, t, cs, O,
-                                      [] { named_bar_sync(1, NWARP_SM * 32); });
+                                      [] { named_bar_sync(1, NWARP_SM * 32); },
+                                      (long long)gridDim.x + p.R, p.status);
             const int b = row / p.Hkv, g = row % p.Hkv;
 #pragma unroll
             for (int h = 0; h < G; ++h)

@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
 
 #include "../../include/eta.h"
 
@@ -37,6 +38,39 @@ ETA_DEV float bf16_to_f(uint16_t h) { return __uint_as_float(((uint32_t)h) << 16
 ETA_DEV void set_status(int32_t* st, int32_t bits) {
   if (st) atomicOr(st, bits);
 }
+
+// Checked build (-DETA_CHECKED): every global load or store whose index a kernel
+// computes from its inputs or its schedule is guarded by ETA_IN_BOUNDS(i, n, status),
+// false when i lies outside [0, n): ETA_DEVSTAT_BOUNDS is then OR-ed into the status
+// word (when the call has one), the first such event of the source file is printed
+// with its file and line, and the caller skips the access.  In the release build the
+// guard is the constant true and generates no code.
+#ifdef ETA_CHECKED
+static __device__ int g_bounds_reported = 0;
+
+static __device__ __noinline__ bool in_bounds_report(long long i, long long n, int32_t* st,
+                                                     const char* file, int line) {
+  set_status(st, ETA_DEVSTAT_BOUNDS);
+  if (atomicExch(&g_bounds_reported, 1) == 0)
+    printf("eta checked build: index %lld outside [0, %lld) at %s:%d\n", i, n, file, line);
+  return false;
+}
+
+ETA_DEV bool in_bounds(long long i, long long n, int32_t* st, const char* file, int line) {
+  return (i >= 0 && i < n) ? true : in_bounds_report(i, n, st, file, line);
+}
+#define ETA_IN_BOUNDS(i, n, st) \
+  eta::in_bounds((long long)(i), (long long)(n), (st), __FILE__, __LINE__)
+// The half-open index range [lo, hi) lies inside [0, n) (true when it is empty).
+#define ETA_RANGE_IN_BOUNDS(lo, hi, n, st) \
+  ((long long)(hi) <= (long long)(lo) ||    \
+   (ETA_IN_BOUNDS(lo, n, st) && ETA_IN_BOUNDS((long long)(hi) - 1, n, st)))
+constexpr bool kChecked = true;
+#else
+#define ETA_IN_BOUNDS(i, n, st) true
+#define ETA_RANGE_IN_BOUNDS(lo, hi, n, st) true
+constexpr bool kChecked = false;
+#endif
 
 ETA_DEV uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -37,6 +37,7 @@ extern "C" eta_status_t eta_calibrate_const_tau(const float* bounds, const uint8
 }
 
 extern "C" eta_status_t eta_status_from_device(int32_t dev_status) {
+  if (dev_status & ETA_DEVSTAT_BOUNDS) return ETA_ERR_DEVICE_BOUNDS;
   if (dev_status & ETA_DEVSTAT_TIMEOUT) return ETA_ERR_DEVICE_TIMEOUT;
   if (dev_status & ETA_DEVSTAT_NONFINITE_Q) return ETA_ERR_NONFINITE;
   if (dev_status & (ETA_DEVSTAT_BAD_BLOCK | ETA_DEVSTAT_BAD_LENGTH)) return ETA_ERR_INVALID_ARG;
@@ -52,6 +53,7 @@ extern "C" const char* eta_status_string(eta_status_t s) {
     case ETA_ERR_CUDA: return "CUDA error";
     case ETA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case ETA_ERR_NONFINITE: return "non-finite query";
+    case ETA_ERR_DEVICE_BOUNDS: return "out-of-range index (checked build)";
   }
   return "unknown status";
 }

@@ -35,6 +35,9 @@ meta_build_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restr
   if (jj >= nblk) return;
   const int j = blk_begin + jj;
   const int n = min(max(len - j * blk, 0), blk);
+  // the block's metadata slot and the tokens its keys come from
+  if (!ETA_IN_BOUNDS(j, NB, status) || !ETA_RANGE_IN_BOUNDS(j * blk, j * blk + n, T_max, status))
+    return;
   const size_t rowj = (size_t)r * NB + j;
   const eta_bf16_t* kb = K + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;
 
@@ -154,7 +157,7 @@ meta_tail_kernel(int Hkv, int T_max, int blk, int NB, const eta_bf16_t* __restri
   ETA_PDL_ENTRY();
   __shared__ TailScratch<D, CF> sc;
   meta_tail_block<D, CF, kMetaWarps>(blockIdx.x, Hkv, T_max, blk, NB, K, V, lengths, cent, rmax,
-                                     var, cnt, vsum, vardim, sc, threadIdx.x >> 5,
+                                     var, cnt, vsum, vardim, nullptr, sc, threadIdx.x >> 5,
                                      [] { __syncthreads(); });
 }
 

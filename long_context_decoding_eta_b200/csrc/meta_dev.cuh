@@ -49,7 +49,8 @@ ETA_DEV void store_centroid(void* cent, size_t idx, float c) {
 // kMetaWarps chunks ("virtual warps") whose partial sums are combined in chunk
 // order, the order meta_build_kernel uses, so a tail refresh and a full rebuild of
 // the same block give bit-identical metadata.  NWARP real warps (local index wid)
-// run the chunks in turns; `sync` synchronizes them; returns synchronized.
+// run the chunks in turns; `sync` synchronizes them; returns synchronized.  status:
+// the checked build's range reports (may be NULL).
 template <int D, int CF>
 struct TailScratch {
   using Acc = typename std::conditional<CF == 1, double, float>::type;
@@ -65,8 +66,8 @@ ETA_DEV void meta_tail_block(int r, int Hkv, int T_max, int blk, int NB,
                              const int32_t* __restrict__ lengths, void* __restrict__ cent,
                              float* __restrict__ rmax, float* __restrict__ var,
                              int32_t* __restrict__ cnt, float* __restrict__ vsum,
-                             float* __restrict__ vardim, TailScratch<D, CF>& sc, int wid,
-                             Sync sync) {
+                             float* __restrict__ vardim, int32_t* status,
+                             TailScratch<D, CF>& sc, int wid, Sync sync) {
   constexpr int DPL = D / 32;
   using Acc = typename TailScratch<D, CF>::Acc;
   const int warp = wid, lane = threadIdx.x & 31;
@@ -75,6 +76,9 @@ ETA_DEV void meta_tail_block(int r, int Hkv, int T_max, int blk, int NB,
   if (len == 0) return;                      // uniform over the callers
   const int j = (len - 1) / blk;
   const int n = min(len - j * blk, blk);
+  // (checked build) the tail block's slot and tokens; uniform over the callers
+  if (!ETA_IN_BOUNDS(j, NB, status) || !ETA_RANGE_IN_BOUNDS(j * blk, j * blk + n, T_max, status))
+    return;
   const int per = (blk + kMetaWarps - 1) / kMetaWarps;
   const size_t rowj = (size_t)r * NB + j;
   const eta_bf16_t* kb = K + ((size_t)r * T_max + (size_t)j * blk) * D + lane * DPL;

@@ -204,7 +204,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       int j = 0;
       for (; j < nkv && ok; ++j) {
         const int s = j % NKV;
-        if (!mbar_wait(&ms->kv_empty[s], ((uint32_t)(j / NKV) & 1u) ^ 1u, abort_flag)) {
+        // (checked build) the key tile lies inside the cache row; a refused copy ends
+        // the CTA like a lost wait, after the copies already issued
+        if (!ETA_IN_BOUNDS((j + 1) * TILE - 1, p.T_max, p.status) ||
+            !mbar_wait(&ms->kv_empty[s], ((uint32_t)(j / NKV) & 1u) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
@@ -588,7 +591,10 @@ prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       int j = 0;
       for (; j < nkv && ok; ++j) {
         const int s = j % NKV;
-        if (!mbar_wait(&ms->kv_empty[s], ((uint32_t)(j / NKV) & 1u) ^ 1u, abort_flag)) {
+        // (checked build) the key tile lies inside the cache row; a refused copy ends
+        // the CTA like a lost wait, after the copies already issued
+        if (!ETA_IN_BOUNDS((j + 1) * TILE - 1, p.T_max, p.status) ||
+            !mbar_wait(&ms->kv_empty[s], ((uint32_t)(j / NKV) & 1u) ^ 1u, abort_flag)) {
           ok = false;
           break;
         }

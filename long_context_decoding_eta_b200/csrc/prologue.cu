@@ -32,7 +32,7 @@ prologue_kernel(int Hq, int Hkv, int T_max, int blk, int NB, const eta_bf16_t* _
   const int b = blockIdx.x, g = blockIdx.y, r = b * Hkv + g;
   if (warp < kMetaWarps) {
     meta_tail_block<D, CF, kMetaWarps>(r, Hkv, T_max, blk, NB, K, V, lengths, cent, rmax, var,
-                                       cnt, vsum, vardim, sc, warp,
+                                       cnt, vsum, vardim, status, sc, warp,
                                        [] { named_bar_sync(1, kMetaWarps * 32); });
   } else if (tau_const) {
     const int lt = threadIdx.x - kMetaWarps * 32;

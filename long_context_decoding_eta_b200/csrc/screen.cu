@@ -148,11 +148,12 @@ screen_vec_kernel(int Hq, int Hkv, int NB, int NW, const eta_bf16_t* __restrict_
 __global__ void __launch_bounds__(kCompactThreads)
 compact_kernel(int Hq, int Hkv, int G, int NB, int NW, const uint32_t* __restrict__ union_words,
                const uint32_t* __restrict__ head_mask, int32_t* __restrict__ union_idx,
-               int32_t* __restrict__ union_cnt, int32_t* __restrict__ head_cnt) {
+               int32_t* __restrict__ union_cnt, int32_t* __restrict__ head_cnt,
+               int32_t* status) {
   ETA_PDL_ENTRY();
   __shared__ CompactScratch<kCompactThreads> cs;
   compact_row<kCompactThreads>(blockIdx.x, Hq, Hkv, G, NB, NW, union_words, head_mask, union_idx,
-                               union_cnt, head_cnt, cs);
+                               union_cnt, head_cnt, cs, status);
 }
 
 // Small batches: one CTA per (row, KV head) pair screens the whole row and compacts
@@ -207,6 +208,8 @@ screen_row_kernel(const __grid_constant__ CUtensorMap tmC, int Hq, int Hkv, int 
     unsigned char* st = smem + buf * C::SB;
     const int j0 = grp * kScreenGroupBlocks;
     const uint32_t nb4 = (uint32_t)min(kScreenGroupBlocks, NB - j0) * 4u;
+    // (checked build) a group starts inside the row; a skipped copy ends in a timeout
+    if (!ETA_RANGE_IN_BOUNDS(j0, j0 + (int)(nb4 / 4u), NB, status)) return;
     mbar_arrive_expect_tx(&full[buf], (uint32_t)C::CENT + nb4 * (pv ? 3u : 2u));
     tc::tma_load_2d(st, &tmC, j0, r * D, &full[buf]);
     const size_t rj = (size_t)r * NB + j0;
@@ -267,7 +270,7 @@ screen_row_kernel(const __grid_constant__ CUtensorMap tmC, int Hq, int Hkv, int 
   if (!ok && lane == 0) mbar_wait(&full[warp], (uint32_t)round & 1u, nullptr);
   __syncthreads();
   compact_row<C::NT>(r, Hq, Hkv, G, NB, NW, union_words, head_mask, union_idx, union_cnt,
-                     head_cnt, cs);
+                     head_cnt, cs, status);
 }
 
 template <int D, int CF, bool VD>
@@ -429,5 +432,5 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   if (st != ETA_OK) return st;
   return launch_k(compact_kernel, dim3(R), dim3(kCompactThreads), 0, s, dims->Hq, dims->Hkv, G,
                   NB, NW, (const uint32_t*)uw, (const uint32_t*)head_mask, union_idx, union_cnt,
-                  head_cnt);
+                  head_cnt, dev_status);
 }

@@ -110,10 +110,9 @@ ETA_DEV void compact_row(const StepParams& sp, int r) {
     const int nw = min(32, sp.NW - base);
     for (int i = 0; i < nw; ++i) {
       const uint32_t wd = __shfl_sync(0xffffffffu, word, i);
-      const int off = __shfl_sync(0xffffffffu, excl, i);
-      if ((wd >> lane) & 1u)
-        sp.union_idx[(size_t)r * sp.NB + off + __popc(wd & ((1u << lane) - 1u))] =
-            (base + i) * 32 + lane;
+      const int pos = __shfl_sync(0xffffffffu, excl, i) + __popc(wd & ((1u << lane) - 1u));
+      if (((wd >> lane) & 1u) && ETA_IN_BOUNDS(pos, sp.NB, sp.status))
+        sp.union_idx[(size_t)r * sp.NB + pos] = (base + i) * 32 + lane;
     }
     carry += __shfl_sync(0xffffffffu, incl, 31);
   }
@@ -238,7 +237,8 @@ step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
       if (warp < 4) {
         if (sp.update_tail)
           meta_tail_block<D, CF, 4>(r, sp.Hkv, sp.T_max, sp.blk, sp.NB, sp.K, sp.V, sp.lengths,
-                                    sp.cent, sp.rmax, sp.var, sp.cnt, nullptr, sp.vardim, *tail,
+                                    sp.cent, sp.rmax, sp.var, sp.cnt, nullptr, sp.vardim,
+                                    sp.status, *tail,
                                     warp, [] { named_bar_sync(1, 128); });
       } else if (sp.tau_const) {
         const int lt = threadIdx.x - 128;
@@ -566,6 +566,8 @@ extern "C" eta_status_t eta_decode_step(
   tp.part_o = reinterpret_cast<float*>(w + L.part_o);
   tp.part_ml = reinterpret_cast<float*>(w + L.part_ml);
   tp.status = dev_status;
+  tp.R = R;
+  tp.counts = nullptr; tp.row_off_g = nullptr; tp.plan_g = nullptr;   // the plan is per CTA
 
   CUtensorMap mk, mv, mq, mc;
   const uint64_t kv_rows = (uint64_t)dims->B * dims->Hkv * dims->T_max;

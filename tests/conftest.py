@@ -24,9 +24,10 @@ def pytest_collection_modifyitems(config, items):
 
 @pytest.fixture(scope="session", autouse=True)
 def _built_library():
-    """Builds libeta.so in-tree once per session (nvcc cross-compiles without a GPU)."""
+    """Builds libeta.so in-tree once per session (nvcc cross-compiles without a GPU);
+    libeta_checked.so instead when ETA_CHECKED=1 selects the range-checked build."""
     from long_context_decoding_eta_b200 import build
-    build.build()
+    build.build(checked=os.environ.get("ETA_CHECKED") == "1")
     yield
 
 

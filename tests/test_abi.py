@@ -123,3 +123,35 @@ def test_engine_selection_host_only():
     L.eta_set_decode_engine("auto")
     with pytest.raises(L.EtaError):
         L.eta_set_decode_engine(7)
+
+
+def test_checked_build_loads_with_the_same_entry_points():
+    """The range-checked build (-DETA_CHECKED) links, exports every declared entry
+    point and says it is the checked one; the release build says it is not."""
+    import subprocess
+    import sys
+    from long_context_decoding_eta_b200 import build
+    path = build.build(checked=True)
+    assert path.endswith("libeta_checked.so")
+    assert L.eta_build_checked() is False
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from long_context_decoding_eta_b200 import _lib as L\n"
+            "lib = L.lib()\n"
+            "assert L.LIB_PATH.endswith('libeta_checked.so'), L.LIB_PATH\n"
+            "missing = [n for n in %r if not hasattr(lib, n)]\n"
+            "assert not missing, missing\n"
+            "print('checked', L.eta_build_checked())\n") % (ROOT, declared_functions())
+    env = dict(os.environ, ETA_CHECKED="1")
+    p = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert p.returncode == 0, p.stderr
+    assert "checked True" in p.stdout
+
+
+def test_device_status_mapping_of_the_bounds_bit():
+    assert L.eta_status_from_device(L.DEVSTAT_BOUNDS) == 7
+    assert L.eta_status_from_device(L.DEVSTAT_BOUNDS | L.DEVSTAT_TIMEOUT) == 7
+    assert "checked build" in L.eta_status_string(7)
+    # argument checks run on the host: nothing is launched
+    assert L.lib().eta_selftest_bounds(0, -1, ctypes.c_void_p(16), None) == 1
+    assert L.lib().eta_selftest_bounds(0, 4, None, None) == 1

@@ -77,6 +77,9 @@ typedef struct {
 } eta_dims_t;
 
 typedef enum { ETA_BOUND_EXACT = 0, ETA_BOUND_PROB = 1, ETA_BOUND_PROB_DIM = 2 } eta_bound_t;
+/* Compute engine of the decode and of the screen (eta_set_decode_engine,
+   eta_set_screen_engine). */
+typedef enum { ETA_ENGINE_AUTO = 0, ETA_ENGINE_TCGEN05 = 1, ETA_ENGINE_FMA = 2 } eta_engine_t;
 /* Storage of the block centroids.  ETA_CENT_BF16 halves the bytes the screen reads;
    the centroid is then rounded to bf16 (nearest even) before rmax and var are
    measured against it, so the geometric bound stays exact for what is stored. */
@@ -156,12 +159,26 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  *   bounds_out fp32   [B, Hq, NB] or NULL (calibration, near-tie logging)
  *   head_cnt   int32  [B, Hq] or NULL: popcount of the head's admit mask
  * ws/ws_bytes: scratch of at least eta_screen_workspace_size(dims) bytes.
+ * Two forms compute the q . cent products (both tested against the float64 oracle;
+ * their fp32 sums differ in order, so they agree up to rounding, i.e. near-ties):
+ *   tensor cores (bf16 centroids, d = 128, ETA_BOUND_EXACT or _PROB, NB % 8 == 0,
+ *     every pointer 16-byte aligned): a 128-block group's products as one
+ *     tcgen05.mma (M = 128 blocks, N = 16, K = d) from TMA-staged tiles;
+ *   CUDA cores: fp32 FMA chains.
+ * eta_set_screen_engine (process-wide) chooses: ETA_ENGINE_TCGEN05 the tensor cores
+ * wherever they apply, ETA_ENGINE_FMA the CUDA cores always, ETA_ENGINE_AUTO (the
+ * default) the tensor cores where this library measures them faster: when the
+ * (row, KV head) pairs fit one per SM and rows have at most 32 groups of 128
+ * blocks.  The one-launch step follows the same choice.
  * Kernel launches: one (screening and compaction together, one CTA per (row, KV
- * head) pair: batches of at most two CTAs per SM whose rows fit two rounds of the
- * CTA's group buffers, NB a multiple of 8 for bf16 centroids or 4 for fp32) or two
- * (screening, then compaction); eta_screen_launches says which.
- * dev_status (may be NULL): ETA_DEVSTAT_TIMEOUT if the one-launch form's bounded wait
- * for a staged group tile ran out (the outputs are then incomplete).
+ * head) pair: the tensor-core form when the pairs fit one per SM and rows have at
+ * most 32 groups of 128 blocks; the CUDA-core form for batches of at most two CTAs
+ * per SM whose rows fit two rounds of the CTA's group buffers, NB a multiple of 8
+ * for bf16 centroids or 4 for fp32) or two (screening, then compaction);
+ * eta_screen_launches says which.
+ * dev_status (may be NULL): ETA_DEVSTAT_TIMEOUT if a one-launch or tensor-core
+ * form's bounded wait for a staged group tile ran out (the outputs are then
+ * incomplete).
  */
 /*
  * eta_append_and_predict_tau -- eta_build_block_meta(..., ETA_TAIL_BLOCK, ...) and
@@ -183,10 +200,16 @@ eta_status_t eta_append_and_predict_tau(const eta_dims_t* dims, const eta_bf16_t
 
 size_t eta_screen_workspace_size(const eta_dims_t* dims);
 /* Kernel launches eta_screen makes on the current device for these dims and centroid
- * format when every pointer argument is 16-byte aligned (1 or 2; 2 without a
- * device), or -1 for invalid dims.  A packaging query with no counterpart in the
- * pages; host only, launches nothing. */
+ * format with the exact or variance bound, under the current screen engine, when
+ * every pointer argument is 16-byte aligned (1 or 2; 2 without a device), or -1 for
+ * invalid dims.  A packaging query with no counterpart in the pages; host only,
+ * launches nothing. */
 int32_t eta_screen_launches(const eta_dims_t* dims, eta_cent_format_t cent_format);
+/* Screen engine (process-wide; see eta_screen): ETA_ENGINE_TCGEN05 takes the tensor
+ * cores wherever they apply, ETA_ENGINE_AUTO where they measured faster,
+ * ETA_ENGINE_FMA always the CUDA cores.  ETA_ERR_INVALID_ARG for an unknown value. */
+eta_status_t eta_set_screen_engine(eta_engine_t engine);
+eta_engine_t eta_get_screen_engine(void);
 eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
                         eta_cent_format_t cent_format, const void* cent, const float* rmax,
                         const float* var, const float* vardim,
@@ -337,7 +360,6 @@ eta_status_t eta_dense_decode(const eta_dims_t* dims, const eta_bf16_t* q,
  *   ETA_ENGINE_AUTO    -- the default: the engine this library measures fastest
  * eta_set_decode_engine returns ETA_ERR_INVALID_ARG for an unknown value.
  */
-typedef enum { ETA_ENGINE_AUTO = 0, ETA_ENGINE_TCGEN05 = 1, ETA_ENGINE_FMA = 2 } eta_engine_t;
 eta_status_t eta_set_decode_engine(eta_engine_t engine);
 eta_engine_t eta_get_decode_engine(void);
 

@@ -40,7 +40,8 @@ EXPORTS = ("eta_build_block_meta", "eta_predict_tau", "eta_screen_workspace_size
            "eta_decode_step_workspace_size", "eta_decode_step", "eta_lse_merge",
            "eta_append_and_predict_tau", "eta_screen_launches", "eta_decode_launches",
            "eta_set_prefill_kernel", "eta_get_prefill_kernel", "eta_prefill_kernel_for",
-           "eta_build_checked", "eta_selftest_bounds")
+           "eta_build_checked", "eta_selftest_bounds", "eta_set_screen_engine",
+           "eta_get_screen_engine")
 ENGINE = {"auto": 0, "tcgen05": 1, "fma": 2}
 PREFILL_KERNEL = {"auto": 0, "one_tile": 1, "two_tile": 2}
 
@@ -128,6 +129,10 @@ def lib() -> C.CDLL:
     L.eta_get_prefill_kernel.restype = I32
     L.eta_prefill_kernel_for.argtypes = [DIMS, F32]
     L.eta_prefill_kernel_for.restype = I32
+    L.eta_set_screen_engine.argtypes = [I32]
+    L.eta_set_screen_engine.restype = I32
+    L.eta_get_screen_engine.argtypes = []
+    L.eta_get_screen_engine.restype = I32
     L.eta_build_checked.argtypes = []
     L.eta_build_checked.restype = I32
     L.eta_selftest_bounds.argtypes = [C.c_int64, C.c_int64, P, P]
@@ -302,6 +307,17 @@ def eta_set_decode_engine(engine) -> None:
 
 def eta_get_decode_engine() -> str:
     v = int(lib().eta_get_decode_engine())
+    return {k: n for n, k in ENGINE.items()}.get(v, str(v))
+
+
+def eta_set_screen_engine(engine) -> None:
+    """engine: "auto" | "tcgen05" | "fma" (or the integer value)."""
+    _check("eta_set_screen_engine", lib().eta_set_screen_engine(
+        ENGINE[engine] if isinstance(engine, str) else int(engine)))
+
+
+def eta_get_screen_engine() -> str:
+    v = int(lib().eta_get_screen_engine())
     return {k: n for n, k in ENGINE.items()}.get(v, str(v))
 
 

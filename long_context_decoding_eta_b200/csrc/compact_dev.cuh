@@ -18,15 +18,15 @@ struct CompactScratch {
   int wsum[NT / 32];
 };
 
-// All NT threads of the CTA call this (it synchronises the CTA).  union_words and
-// head_mask: [R][NW] and [B * Hq][NW]; writes union_idx[r * NB ...], union_cnt[r]
-// and, if given, head_cnt of the pair's G query heads.  status: the checked build's
-// range reports (may be NULL).
-template <int NT>
+// Threads 0 .. NT-1 of the CTA call this; `sync` synchronises exactly them.
+// union_words and head_mask: [R][NW] and [B * Hq][NW]; writes union_idx[r * NB ...],
+// union_cnt[r] and, if given, head_cnt of the pair's G query heads.  status: the
+// checked build's range reports (may be NULL).
+template <int NT, typename Sync>
 ETA_DEV void compact_row(int r, int Hq, int Hkv, int G, int NB, int NW,
                          const uint32_t* union_words, const uint32_t* head_mask,
                          int32_t* union_idx, int32_t* union_cnt, int32_t* head_cnt,
-                         CompactScratch<NT>& cs, int32_t* status) {
+                         CompactScratch<NT>& cs, int32_t* status, Sync sync) {
   static_assert(NT % 32 == 0 && NT <= 1024, "NT");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int carry = 0;
@@ -41,7 +41,7 @@ ETA_DEV void compact_row(int r, int Hq, int Hkv, int G, int NB, int NW,
       if (lane >= o) incl += y;
     }
     if (lane == 31) cs.wsum[warp] = incl;
-    __syncthreads();
+    sync();
     int wpre = 0, total = 0;
 #pragma unroll
     for (int i = 0; i < NT / 32; ++i) {
@@ -51,7 +51,7 @@ ETA_DEV void compact_row(int r, int Hq, int Hkv, int G, int NB, int NW,
     }
     cs.wbuf[tid] = word;
     cs.woff[tid] = carry + wpre + incl - c;
-    __syncthreads();
+    sync();
     for (int i = warp; i < NT && base + i < NW; i += NT / 32) {
       const uint32_t wd = cs.wbuf[i];
       const int pos = cs.woff[i] + __popc(wd & ((1u << lane) - 1u));
@@ -59,7 +59,7 @@ ETA_DEV void compact_row(int r, int Hq, int Hkv, int G, int NB, int NW,
         union_idx[(size_t)r * NB + pos] = (base + i) * 32 + lane;
     }
     carry += total;
-    __syncthreads();
+    sync();
   }
   if (tid == 0) union_cnt[r] = carry;
   if (head_cnt) {

@@ -84,6 +84,8 @@ struct FuseItem {
 };
 struct FuseSmem {
   uint64_t bfull[kFuseStages], bempty[kFuseStages];
+  uint64_t bacc_full[2], bacc_free[2], bfin;   // tensor-core screening's accumulators
+  uint32_t btmem;                               // and their TMEM columns
   FuseItem item[kFuseStages];
   CombineScratch<8> cs;   // sized for the largest group
   int last;

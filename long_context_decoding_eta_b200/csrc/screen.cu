@@ -16,6 +16,7 @@
 //   list of admitted block indices (popcount prefix over words, lane = bit).
 // screen_row_kernel (small batches): screening from TMA-staged group tiles and the
 //   compaction of its row in one launch.
+#include <atomic>
 #include <type_traits>
 
 #include "eta_common.cuh"
@@ -23,6 +24,7 @@
 #include "compact_dev.cuh"
 #include "decode_tc.cuh"   // tc::tma_load_2d
 #include "screen_dev.cuh"
+#include "screen_tc.cuh"
 #include "tma_host.h"
 
 namespace eta {
@@ -153,7 +155,7 @@ compact_kernel(int Hq, int Hkv, int G, int NB, int NW, const uint32_t* __restric
   ETA_PDL_ENTRY();
   __shared__ CompactScratch<kCompactThreads> cs;
   compact_row<kCompactThreads>(blockIdx.x, Hq, Hkv, G, NB, NW, union_words, head_mask, union_idx,
-                               union_cnt, head_cnt, cs, status);
+                               union_cnt, head_cnt, cs, status, [] { __syncthreads(); });
 }
 
 // Small batches: one CTA per (row, KV head) pair screens the whole row and compacts
@@ -270,7 +272,7 @@ screen_row_kernel(const __grid_constant__ CUtensorMap tmC, int Hq, int Hkv, int 
   if (!ok && lane == 0) mbar_wait(&full[warp], (uint32_t)round & 1u, nullptr);
   __syncthreads();
   compact_row<C::NT>(r, Hq, Hkv, G, NB, NW, union_words, head_mask, union_idx, union_cnt,
-                     head_cnt, cs, status);
+                     head_cnt, cs, status, [] { __syncthreads(); });
 }
 
 template <int D, int CF, bool VD>
@@ -333,9 +335,105 @@ static bool row_screen_fits(int R, int NB) {
          NB % (CF == 1 ? 8 : 4) == 0;
 }
 
+// ---------------------------------------------------------------- tensor-core screen
+std::atomic<int> g_screen_engine{ETA_ENGINE_AUTO};
+
+// One launch (a CTA per row, the row's compaction included) when every row gets its
+// own SM and rows are short; otherwise the (row, group) items in equal contiguous
+// shares over one CTA per SM, and compact_kernel after.
+constexpr int kTcRowsMaxGroups = 32;
+inline bool tc_screen_rows(int R, int NB) {
+  const int ngrp = (NB + stc::GB - 1) / stc::GB;
+  return R <= sm_count() && ngrp <= kTcRowsMaxGroups;
+}
+
+// ETA_ENGINE_AUTO takes the tensor cores where they measured faster on one B200: the
+// one-launch form (128K / B = 16: 23.5 vs 27.7 us for screen + compaction; the
+// one-launch step at B = 8, 32K: 76.6 vs 82.4 us per step).  For larger batches the
+// CUDA-core screen streams the dimension-major centroids a little faster (128K /
+// B = 64: 42.1 vs 46.0 us; the tensor-core form's 128-byte TMA rows of a 4 KB-strided
+// layout stay near 3.7 us of DRAM latency with 5 or 6 stages in flight).
+bool tc_screen_applies(const eta_dims_t* d, int cent_format, int bound) {
+  const int e = g_screen_engine.load();
+  if (e == ETA_ENGINE_FMA || cent_format != ETA_CENT_BF16 || d->d != 128 ||
+      bound == ETA_BOUND_PROB_DIM || num_blocks(d) % 8 != 0)
+    return false;
+  return e == ETA_ENGINE_TCGEN05 || tc_screen_rows(d->B * d->Hkv, num_blocks(d));
+}
+
+template <int G>
+static eta_status_t launch_screen_tc(bool rows, const CUtensorMap& mc, const CUtensorMap& mq,
+                                     const stc::Params& prm, int grid, cudaStream_t s) {
+  if (rows) {
+    if (!set_smem_once<stc::screen_tc_kernel<G, true>>(stc::SMEM_BYTES)) return ETA_ERR_CUDA;
+    return launch_k(stc::screen_tc_kernel<G, true>, dim3(grid), dim3(stc::NT), stc::SMEM_BYTES,
+                    s, mc, mq, prm);
+  }
+  if (!set_smem_once<stc::screen_tc_kernel<G, false>>(stc::SMEM_BYTES)) return ETA_ERR_CUDA;
+  return launch_k(stc::screen_tc_kernel<G, false>, dim3(grid), dim3(stc::NT), stc::SMEM_BYTES, s,
+                  mc, mq, prm);
+}
+
+// eta_screen on the tensor cores (tc_screen_applies).  Pointers are 16-byte aligned.
+static eta_status_t run_screen_tc(const eta_dims_t* dims, const eta_bf16_t* q, const float* tau,
+                                  const void* cent, const float* rmax, const float* var,
+                                  const int32_t* cnt, int bound, float z, float scale,
+                                  uint32_t* head_mask, uint32_t* uw, int32_t* union_idx,
+                                  int32_t* union_cnt, float* bounds_out, int32_t* head_cnt,
+                                  int32_t* dev_status, cudaStream_t s) {
+  const int NB = num_blocks(dims), NW = num_words(dims);
+  const int R = dims->B * dims->Hkv, G = dims->Hq / dims->Hkv;
+  CUtensorMap mc, mq;
+  if (!make_map_bf16_swz(&mc, cent, NB, (uint64_t)R * stc::D, (uint64_t)NB * 2, stc::D) ||
+      !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16))
+    return ETA_ERR_CUDA;
+  stc::Params prm;
+  prm.Hq = dims->Hq; prm.Hkv = dims->Hkv; prm.NB = NB; prm.NW = NW;
+  prm.ngrp = (NB + stc::GB - 1) / stc::GB;
+  prm.items = R * prm.ngrp;
+  prm.prob = bound == ETA_BOUND_PROB ? 1 : 0;
+  prm.z = z; prm.scale = scale;
+  prm.q = q; prm.tau = tau; prm.rmax = rmax; prm.var = var; prm.cnt = cnt;
+  prm.head_mask = head_mask; prm.union_words = uw; prm.bounds_out = bounds_out;
+  prm.union_idx = union_idx; prm.union_cnt = union_cnt; prm.head_cnt = head_cnt;
+  prm.status = dev_status;
+  const bool rows = tc_screen_rows(R, NB);
+  int grid;
+  if (rows) {
+    prm.chunk = prm.ngrp;
+    grid = R;
+  } else {
+    const int n = std::max(sm_count(), 1);
+    prm.chunk = (prm.items + n - 1) / n;
+    grid = (prm.items + prm.chunk - 1) / prm.chunk;
+  }
+  eta_status_t st = ETA_ERR_UNSUPPORTED;
+  switch (G) {
+    case 1: st = launch_screen_tc<1>(rows, mc, mq, prm, grid, s); break;
+    case 2: st = launch_screen_tc<2>(rows, mc, mq, prm, grid, s); break;
+    case 4: st = launch_screen_tc<4>(rows, mc, mq, prm, grid, s); break;
+    case 8: st = launch_screen_tc<8>(rows, mc, mq, prm, grid, s); break;
+  }
+  if (st != ETA_OK || rows) return st;
+  return launch_k(compact_kernel, dim3(R), dim3(kCompactThreads), 0, s, dims->Hq, dims->Hkv, G,
+                  NB, NW, (const uint32_t*)uw, (const uint32_t*)head_mask, union_idx, union_cnt,
+                  head_cnt, dev_status);
+}
+
 }  // namespace eta
 
 using namespace eta;
+
+extern "C" eta_status_t eta_set_screen_engine(eta_engine_t engine) {
+  if (engine != ETA_ENGINE_AUTO && engine != ETA_ENGINE_TCGEN05 && engine != ETA_ENGINE_FMA)
+    return ETA_ERR_INVALID_ARG;
+  g_screen_engine.store((int)engine);
+  return ETA_OK;
+}
+
+extern "C" eta_engine_t eta_get_screen_engine(void) {
+  return static_cast<eta_engine_t>(g_screen_engine.load());
+}
 
 extern "C" size_t eta_screen_workspace_size(const eta_dims_t* dims) {
   if (check_dims(dims) != ETA_OK) return 0;
@@ -346,6 +444,7 @@ extern "C" int32_t eta_screen_launches(const eta_dims_t* dims, eta_cent_format_t
   if (check_dims(dims) != ETA_OK) return -1;
   const int NB = num_blocks(dims), R = dims->B * dims->Hkv;
   const bool bf = cent_format == ETA_CENT_BF16;
+  if (tc_screen_applies(dims, cent_format, ETA_BOUND_EXACT)) return tc_screen_rows(R, NB) ? 1 : 2;
   if (NB % 4 != 0) return 2;
   bool row;
   if (dims->d == 128) row = bf ? row_screen_fits<128, 1>(R, NB) : row_screen_fits<128, 0>(R, NB);
@@ -381,6 +480,9 @@ extern "C" eta_status_t eta_screen(const eta_dims_t* dims, const eta_bf16_t* q, 
   const bool vec = (NB % VW == 0) && aligned16(cent) && aligned16(rmax) && aligned16(cnt) &&
                    (!var || aligned16(var)) && (!vardim || aligned16(vardim)) &&
                    (!bounds_out || aligned16(bounds_out));
+  if (vec && aligned16(q) && tc_screen_applies(dims, cent_format, bound))
+    return run_screen_tc(dims, q, tau, cent, rmax, var, cnt, (int)bound, z, scale, head_mask, uw,
+                         union_idx, union_cnt, bounds_out, head_cnt, dev_status, s);
   bool row = vec;
   if (row) {
     if (dims->d == 128) row = bf ? row_screen_fits<128, 1>(R, NB) : row_screen_fits<128, 0>(R, NB);

@@ -18,8 +18,10 @@
 //      waits for a group's row to be released and stages the group with TMA into a
 //      shared-memory ring: the [d x 128] centroid tile (tensor copy), the rmax / var /
 //      cnt slices and the G query rows (bulk copies).  Up to five warps (no more than
-//      the ring has stages) screen the staged groups (head words, union word).
-//      The screening warps also count each row's admitted blocks.
+//      the ring has stages) screen the staged groups (head words, union word); where
+//      eta_screen takes the tensor cores (tc_screen_applies) the step does too:
+//      warp 5 issues each group's q . c product (screen_tc.cuh) and warps 0-3 read
+//      it from TMEM.  The screening warps also count each row's admitted blocks.
 //   -  grid barrier; then warps compact the rows' union lists (and write o = 0,
 //      lse = -inf for a row with nothing admitted), flagging each row as it is done;
 //      every CTA lays out the CTA shares in its own shared memory (prefix sum of the
@@ -40,6 +42,7 @@
 #include "eta_host.h"
 #include "meta_dev.cuh"
 #include "screen_dev.cuh"
+#include "screen_tc.cuh"
 #include "tau_dev.cuh"
 #include "tma_host.h"
 
@@ -199,7 +202,171 @@ ETA_DEV void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-template <int G, int CF, bool VD>
+// Phase B on the tensor cores (bf16 centroids, not the per-dimension bound): the
+// groups pass in order through a ring of screen_tc stages; warp 5 issues each group's
+// q . c product into one of two TMEM accumulators and warps 0-3 turn it into the
+// bound, the admit words and the row's admitted count (stc::issue_mma and
+// stc::epilogue, the arithmetic of the standalone tensor-core screen).
+constexpr int kTcFit = tc::SM_P / (stc::TILE + stc::META);
+constexpr int kTcStages = kTcFit < tc::kFuseStages ? kTcFit : tc::kFuseStages;
+constexpr int kTcMeta = kTcStages * stc::TILE;         // the stages' metadata slots
+static_assert(kTcStages >= 2, "two tensor-core screening stages must fit");
+static_assert(kTcMeta + kTcStages * stc::META <= tc::SM_P, "screening ring in the decode ring");
+
+template <int G>
+ETA_DEV void phase_b_tc(unsigned char* smem, tc::FuseSmem* fs, const StepParams& sp,
+                        const CUtensorMap* tmC, const CUtensorMap* tmQ, int32_t* adm_now,
+                        int tok_released) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int items = sp.R * sp.ngroups;
+  const uint32_t tmem = fs->btmem;
+  if (warp == tc::NWARP_SM) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane != 0) return;
+    bool ok = true;
+    int k = 0, cur_r = -1, nvalid = 0;
+    float ts[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int batch = atomicAdd(sp.sync + kSyncItems, kGrab);
+    while (ok && batch < items) {
+      const int next = atomicAdd(sp.sync + kSyncItems, kGrab);   // in flight meanwhile
+      const int end = min(batch + kGrab, items);
+      for (int it = batch; it < end; ++it) {
+        const int r = it / sp.ngroups, grp = it % sp.ngroups;
+        const int b = r / sp.Hkv, g = r % sp.Hkv;
+        const size_t qhead0 = (size_t)b * sp.Hq + (size_t)g * G;
+        if (r != cur_r) {
+          // the row's tail metadata and thresholds are released by its prologue
+          if (!wait_flag_thread(sp.ready + r, tok_released, sp)) { ok = false; break; }
+          fence_proxy_async_global();       // TMA reads what the release published
+          cur_r = r;
+          const int len = min(max(sp.lengths[b], 0), sp.T_max);
+          nvalid = (len + sp.blk - 1) / sp.blk;
+#pragma unroll
+          for (int h = 0; h < G; ++h) ts[h] = __ldcg(sp.tau + qhead0 + h);
+        }
+        const int s = k % kTcStages;
+        if (!mbar_wait(&fs->bempty[s], ((uint32_t)(k / kTcStages) & 1u) ^ 1u, &fs->abort)) {
+          ok = false;
+          break;
+        }
+        tc::FuseItem& rec = fs->item[s];
+        rec.r = r; rec.grp = grp; rec.nvalid = nvalid; rec.flags = 0;
+#pragma unroll
+        for (int h = 0; h < G; ++h) rec.ts[h] = ts[h];
+        unsigned char* st = smem + s * stc::TILE;
+        unsigned char* mt = smem + kTcMeta + s * stc::META;
+        const int j0 = grp * stc::GB;
+        const uint32_t nb4 = (uint32_t)min(stc::GB, sp.NB - j0) * 4u;
+        const bool pv = sp.bound == ETA_BOUND_PROB;
+        mbar_arrive_expect_tx(&fs->bfull[s], (uint32_t)(2 * stc::CENT_HALF + 2 * stc::Q_HALF) +
+                                                 nb4 * (pv ? 3u : 2u));
+        tc::tma_load_2d(st + stc::OFF_C0, tmC, j0, r * D, &fs->bfull[s]);
+        tc::tma_load_2d(st + stc::OFF_C1, tmC, j0 + 64, r * D, &fs->bfull[s]);
+        const int qrow = b * sp.Hq + g * G;
+        tc::tma_load_2d(st + stc::OFF_Q0, tmQ, 0, qrow, &fs->bfull[s]);
+        tc::tma_load_2d(st + stc::OFF_Q1, tmQ, 64, qrow, &fs->bfull[s]);
+        const size_t rj = (size_t)r * sp.NB + j0;
+        bulk_g2s(mt + stc::M_RMAX, sp.rmax + rj, nb4, &fs->bfull[s]);
+        if (pv) bulk_g2s(mt + stc::M_VAR, sp.var + rj, nb4, &fs->bfull[s]);
+        bulk_g2s(mt + stc::M_CNT, sp.cnt + rj, nb4, &fs->bfull[s]);
+        ++k;
+      }
+      batch = next;
+    }
+    if (ok) {
+      // one end marker: the MMA warp and the epilogue warps read every stage in order
+      const int s = k % kTcStages;
+      if (mbar_wait(&fs->bempty[s], ((uint32_t)(k / kTcStages) & 1u) ^ 1u, &fs->abort)) {
+        fs->item[s].flags = 1;
+        mbar_arrive(&fs->bfull[s]);
+      } else {
+        ok = false;
+      }
+    }
+    if (!ok) {
+      fail(sp);
+      set_abort(fs);
+      // every copy issued lands before the ring is reused or the CTA exits
+      for (int kk = max(0, k - kTcStages); kk < k; ++kk)
+        mbar_wait(&fs->bfull[kk % kTcStages], (uint32_t)(kk / kTcStages) & 1u, nullptr);
+    }
+  } else if (warp == tc::NWARP_SM + 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane != 0) return;
+    bool ok = true;
+    for (int k = 0;; ++k) {
+      const int s = k % kTcStages, b = k & 1;
+      if (!mbar_wait(&fs->bfull[s], (uint32_t)(k / kTcStages) & 1u, &fs->abort)) {
+        ok = false;
+        break;
+      }
+      if (fs->item[s].flags) break;
+      if (!mbar_wait(&fs->bacc_free[b], ((uint32_t)(k >> 1) & 1u) ^ 1u, &fs->abort)) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      stc::issue_mma(tmem + b * stc::kAccCols, smem + s * stc::TILE);
+      tc::mma_commit(&fs->bacc_full[b]);
+    }
+    if (!ok) {
+      fail(sp);
+      set_abort(fs);
+    }
+    tc::mma_commit(&fs->bfin);             // every MMA issued completes before TMEM is freed
+    mbar_wait(&fs->bfin, 0, nullptr);
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 0-3)
+    const uint32_t lane_sel = (uint32_t)(warp * 32) << 16;
+    int cur_r = -1;
+    float qn[G], ts[G];
+    for (int k = 0;; ++k) {
+      const int s = k % kTcStages, b = k & 1;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&fs->bfull[s],
+                                                         (uint32_t)(k / kTcStages) & 1u,
+                                                         &fs->abort));
+      if (!got) {
+        if (lane == 0) { fail(sp); set_abort(fs); }
+        break;
+      }
+      const tc::FuseItem rec = fs->item[s];
+      __syncwarp();
+      if (rec.flags) {
+        if (lane == 0) mbar_arrive(&fs->bempty[s]);
+        break;
+      }
+      const int r = rec.r, bb = r / sp.Hkv, g = r % sp.Hkv;
+      const size_t qhead0 = (size_t)bb * sp.Hq + (size_t)g * G;
+      if (r != cur_r) {
+        stc::query_norms_staged<G>(smem + s * stc::TILE, qn);
+        cur_r = r;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&fs->bacc_full[b], (uint32_t)(k >> 1) & 1u,
+                                             &fs->abort))) {
+        if (lane == 0) { fail(sp); set_abort(fs); }
+        break;
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) ts[h] = rec.ts[h];
+      tc::tc_fence_after();
+      float dot[16];
+      tc::tmem_ld16(tmem + b * stc::kAccCols + lane_sel, dot);
+      tc::tc_fence_before();
+      const stc::BlockMeta bm = stc::block_meta(smem + kTcMeta + s * stc::META,
+                                                sp.bound == ETA_BOUND_PROB, sp.z, sp.NB, rec.grp);
+      __syncwarp();
+      if (lane == 0) {                      // accumulator and stage are no longer read
+        mbar_arrive(&fs->bacc_free[b]);
+        mbar_arrive(&fs->bempty[s]);
+      }
+      const int adm = stc::epilogue<G>(dot, bm, sp.scale, sp.NB, sp.NW, rec.grp, r, qhead0, qn,
+                                       ts, rec.nvalid, sp.head_mask, sp.union_words, nullptr);
+      if (lane == 0 && adm) atomicAdd(adm_now + r, adm);
+    }
+  }
+}
+
+template <int G, int CF, bool VD, bool TCS>
 __global__ void __launch_bounds__(tc::NT, 1)
 step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
             const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmC,
@@ -211,9 +378,16 @@ step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
   tc::FuseSmem* fs = reinterpret_cast<tc::FuseSmem*>(smem + tc::SM_FUSE);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < PB::NSB; ++s) {
+    for (int s = 0; s < (TCS ? kTcStages : PB::NSB); ++s) {
       mbar_init(&fs->bfull[s], 1);
-      mbar_init(&fs->bempty[s], 1);
+      mbar_init(&fs->bempty[s], TCS ? tc::NWARP_SM : 1);   // TCS: the epilogue warps release
+    }
+    if constexpr (TCS) {
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&fs->bacc_full[b], 1);
+        mbar_init(&fs->bacc_free[b], tc::NWARP_SM);
+      }
+      mbar_init(&fs->bfin, 1);
     }
     fs->abort = 0;
     // the barrier generation cannot move before every CTA has arrived, so all CTAs
@@ -221,7 +395,16 @@ step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
     fs->gen0 = ld_acquire_gpu(sp.sync + kSyncGen);
     fence_mbar_init();
   }
+  if constexpr (TCS) {
+    // phase B's accumulators (freed before phase C allocates its own; no relinquish)
+    if (warp == tc::NWARP_SM + 1)
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&fs->btmem)),
+                   "r"(32));
+    tc::tc_fence_before();
+  }
   __syncthreads();
+  if constexpr (TCS) tc::tc_fence_after();
   const int gen0 = fs->gen0;
   const int tok_released = 2 * gen0 + 1, tok_compacted = 2 * gen0 + 2;
   int32_t* adm_now = sp.adm_cnt + (gen0 & 1) * sp.R;
@@ -262,7 +445,18 @@ step_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUt
   // ---------------------------------------------------------------- B: screening
   // warp 4 (one thread) stages groups with TMA; warps 0-3 and 5 screen them
   const int items = sp.R * sp.ngroups;
-  if (warp == tc::NWARP_SM) {
+  if constexpr (TCS) {
+    phase_b_tc<G>(smem, fs, sp, &tmC, &tmQ, adm_now, tok_released);
+    // every accumulator has been read (the MMA warp waited for its last MMA)
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == tc::NWARP_SM + 1) {
+      __syncwarp();
+      tc::tc_fence_after();
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(fs->btmem),
+                   "r"(32));
+    }
+  } else if (warp == tc::NWARP_SM) {
     if (lane == 0) {
       bool ok = true;
       int k = 0, cur_r = -1, nvalid = 0;
@@ -451,12 +645,12 @@ inline StepWs step_ws(const eta_dims_t* d, int P) {
   return w;
 }
 
-template <int G, int CF, bool VD>
+template <int G, int CF, bool VD, bool TCS>
 eta_status_t launch_step(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq,
                          const CUtensorMap& mc, const StepParams& sp,
                          const tc::TcParams& tp, int P, cudaStream_t s) {
-  auto kern = step_kernel<G, CF, VD>;
-  if (!set_smem_once<step_kernel<G, CF, VD>>(tc::FUSED_SMEM_BYTES)) return ETA_ERR_CUDA;
+  auto kern = step_kernel<G, CF, VD, TCS>;
+  if (!set_smem_once<step_kernel<G, CF, VD, TCS>>(tc::FUSED_SMEM_BYTES)) return ETA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(P);
   cfg.blockDim = dim3(tc::NT);
@@ -472,15 +666,15 @@ eta_status_t launch_step(const CUtensorMap& mk, const CUtensorMap& mv, const CUt
              : ETA_ERR_CUDA;
 }
 
-template <int CF, bool VD>
+template <int CF, bool VD, bool TCS = false>
 eta_status_t dispatch_g(int G, const CUtensorMap& mk, const CUtensorMap& mv,
                         const CUtensorMap& mq, const CUtensorMap& mc, const StepParams& sp,
                         const tc::TcParams& tp, int P, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_step<1, CF, VD>(mk, mv, mq, mc, sp, tp, P, s);
-    case 2: return launch_step<2, CF, VD>(mk, mv, mq, mc, sp, tp, P, s);
-    case 4: return launch_step<4, CF, VD>(mk, mv, mq, mc, sp, tp, P, s);
-    case 8: return launch_step<8, CF, VD>(mk, mv, mq, mc, sp, tp, P, s);
+    case 1: return launch_step<1, CF, VD, TCS>(mk, mv, mq, mc, sp, tp, P, s);
+    case 2: return launch_step<2, CF, VD, TCS>(mk, mv, mq, mc, sp, tp, P, s);
+    case 4: return launch_step<4, CF, VD, TCS>(mk, mv, mq, mc, sp, tp, P, s);
+    case 8: return launch_step<8, CF, VD, TCS>(mk, mv, mq, mc, sp, tp, P, s);
   }
   return ETA_ERR_UNSUPPORTED;
 }
@@ -574,13 +768,18 @@ extern "C" eta_status_t eta_decode_step(
   const bool bf = cent_format == ETA_CENT_BF16, vd = bound == ETA_BOUND_PROB_DIM;
   const uint64_t meta_rows = (uint64_t)R * dims->d;     // [R * d, NB], dimension-major
   const uint32_t box = kScreenGroupBlocks;
+  // the screening takes the tensor cores exactly when eta_screen would
+  const bool tcs = tc_screen_applies(dims, (int)cent_format, (int)bound);
   if (!make_map(&mk, K, kv_rows, 64) || !make_map(&mv, V, kv_rows, 64) ||
-      !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16) ||
-      !make_map_plain(&mc, cent, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                      NB, meta_rows, (uint64_t)NB * (bf ? 2 : 4), box, 128))
+      !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16))
+    return ETA_ERR_CUDA;
+  if (tcs ? !make_map_bf16_swz(&mc, cent, NB, meta_rows, (uint64_t)NB * 2, stc::D)
+          : !make_map_plain(&mc, cent, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                            NB, meta_rows, (uint64_t)NB * (bf ? 2 : 4), box, 128))
     return ETA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (tcs) return fused::dispatch_g<1, false, true>(G, mk, mv, mq, mc, sp, tp, P, s);
   if (bf) return vd ? fused::dispatch_g<1, true>(G, mk, mv, mq, mc, sp, tp, P, s)
                     : fused::dispatch_g<1, false>(G, mk, mv, mq, mc, sp, tp, P, s);
   return vd ? fused::dispatch_g<0, true>(G, mk, mv, mq, mc, sp, tp, P, s)

@@ -1,6 +1,7 @@
 // Host-side TMA tensor maps: the bf16 [rows, 128] views the tcgen05 kernels load
-// (K, V, queries; box of 64 columns x box_rows rows with 128-byte swizzle) and plain
-// 2-D views (the fused step's metadata tiles).  The encoder is the driver's
+// (K, V, queries; box of 64 columns x box_rows rows with 128-byte swizzle), the
+// swizzled bf16 centroid view of the tensor-core screen, and plain 2-D views (the
+// CUDA-core screens' metadata tiles).  The encoder is the driver's
 // cuTensorMapEncodeTiled, looked up once through the runtime.
 #pragma once
 
@@ -31,6 +32,23 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t b
   if (!fn) return false;
   cuuint64_t gdim[2] = {128, rows};
   cuuint64_t gstride[1] = {128 * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// 2-D view of a bf16 tensor, `cols` x `rows` elements, row stride `row_bytes` (a
+// multiple of 16); box 64 columns (128 bytes) x box_rows rows with 128-byte swizzle.
+// Out-of-range elements of a box read as zero.
+inline bool make_map_bf16_swz(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                              uint64_t row_bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {cols, rows};
+  cuuint64_t gstride[1] = {row_bytes};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,

@@ -116,6 +116,20 @@ def test_prefill_kernel_selection_host_only():
         L.eta_prefill_kernel_for(dims, -1.0)
 
 
+def test_screen_engine_selection_host_only():
+    assert L.eta_get_screen_engine() == "auto"
+    for e in ("tcgen05", "fma", "auto"):
+        L.eta_set_screen_engine(e)
+        assert L.eta_get_screen_engine() == e
+    with pytest.raises(L.EtaError):
+        L.eta_set_screen_engine(9)
+    # without a device the launch-count query reports the two-launch form
+    dims = L.Dims.of(4, 16, 4, 128, 64, 8192)
+    L.eta_set_screen_engine("tcgen05")
+    assert L.eta_screen_launches(dims, "bf16") == 2
+    L.eta_set_screen_engine("auto")
+
+
 def test_engine_selection_host_only():
     assert L.eta_get_decode_engine() == "auto"
     L.eta_set_decode_engine("fma")

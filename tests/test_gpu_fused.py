@@ -109,19 +109,37 @@ def test_probabilistic_bound_blk128():
     fused_vs_separate(synth.EXTREME512K.with_(B=2, ctx=16384, seed=403), cent_format="bf16")
 
 
+@pytest.mark.parametrize("screen_engine", ["auto", "fma"])
+@pytest.mark.parametrize("bound", ["exact", "prob"])
+def test_bf16_screening_forms(screen_engine, bound):
+    """bf16 centroids with the exact and the variance bound: the step screens on the
+    tensor cores when eta_screen does (the default) and on the CUDA cores when the
+    screen engine says so; either way it writes the separate calls' bits.  A
+    multi-group row with a partial last group (NB = 144)."""
+    from long_context_decoding_eta_b200 import _lib as L
+    w = synth.MID.with_(B=5, ctx=9216, needles=3, q_scale=3.0, density=0.35, seed=420)
+    L.eta_set_screen_engine(screen_engine)
+    try:
+        fused_vs_separate(w, bound=bound, z=2.0, cent_format="bf16")
+    finally:
+        L.eta_set_screen_engine("auto")
+
+
 def test_const_tau():
     w = synth.MID.with_(B=2, ctx=8192, seed=404)
     fused_vs_separate(w, tau_const=np.linspace(1.6, 2.2, w.Hq))
 
 
+@pytest.mark.parametrize("cent_format", ["f32", "bf16"])
 @pytest.mark.parametrize("G,blk", [(1, 64), (2, 128), (8, 64), (4, 128)])
-def test_shapes_ragged_lengths(G, blk):
-    """Rows that are full, empty, one token long and ragged."""
+def test_shapes_ragged_lengths(G, blk, cent_format):
+    """Rows that are full, empty, one token long and ragged (bf16 centroids: the
+    screening on the tensor cores in both the step and the separate calls)."""
     w = synth.Workload("fused-shape", B=4, Hq=2 * G, Hkv=2, d=128, ctx=3072, blk=blk,
                        n_clusters=16, seg=200, needles=2, gate_T=0.0, density=0.4,
                        density_kind="head", seed=410 + G + blk)
     lengths = torch.tensor([3072, 0, 1, 2000], dtype=torch.int32)
-    sep, fus, *_ = fused_vs_separate(w, lengths=lengths)
+    sep, fus, *_ = fused_vs_separate(w, lengths=lengths, cent_format=cent_format)
     # the empty row got its token; a row whose union is empty reads o = 0, lse = -inf
     cnt = fus.union_cnt.cpu().numpy()
     for b, g in zip(*np.nonzero(cnt == 0)):

@@ -21,11 +21,15 @@ DEV = "cuda"
 
 @pytest.fixture(autouse=True, params=["fma", "tcgen05"])
 def engine(request):
-    """Every parity test runs on both decode engines."""
+    """Every parity test runs on both engines: the CUDA-core decode with the CUDA-core
+    screen, and the tensor-core decode with the tensor-core screen where it applies
+    (bf16 centroids, d = 128, not the per-dimension bound)."""
     from long_context_decoding_eta_b200 import _lib as L
     L.eta_set_decode_engine(request.param)
+    L.eta_set_screen_engine(request.param)
     yield request.param
     L.eta_set_decode_engine("auto")
+    L.eta_set_screen_engine("auto")
 
 
 def make(w, lengths=None, seed=None):
@@ -325,6 +329,77 @@ def test_bf16_screen_of_long_rows(d, G, Hkv, bound, engine):
                        blk=64, n_clusters=32, seg=(384, 640), needles=2, gate_T=0.0,
                        density=0.3, density_kind="head", q_scale=2.0, seed=320 + d + G)
     dims = L.Dims.of(w.B, w.Hq, w.Hkv, w.d, w.blk, w.T_max)
-    assert L.eta_screen_launches(dims, "bf16") == 2
+    if engine == "fma" or d == 64:
+        assert L.eta_screen_launches(dims, "bf16") == 2
+    elif bound != "prob_dim":
+        # the tensor-core screen: a CTA per pair with its compaction (13 groups per row)
+        assert L.eta_screen_launches(dims, "bf16") == 1
     lengths = torch.tensor([w.ctx, w.ctx - 7000], dtype=torch.int32)
     full_parity(w, lengths=lengths, bound=bound, z=2.0, cent_format="bf16")
+
+
+@pytest.mark.parametrize("B,Hkv,G,ctx,bound", [(3, 2, 4, 9216, "exact"), (2, 1, 8, 40960, "prob"),
+                                              (40, 4, 1, 8192, "exact"), (37, 4, 2, 4096, "prob"),
+                                              (20, 8, 4, 6144, "exact")])
+def test_tensor_core_screen_against_cuda_core_screen(B, Hkv, G, ctx, bound, engine):
+    """eta_screen on the tensor cores (one launch with a CTA per pair for small
+    batches, or (row, group) items over one CTA per SM and the compaction after)
+    against the CUDA-core screen on the same inputs: the bounds agree to fp32
+    rounding, the admit words bit for bit except blocks whose bound lies within
+    1e-5 (relative) of tau, the union lists and counts follow the words.  Ragged
+    rows, a partial last group, G = 1/2/4/8, the exact and the variance bound."""
+    from long_context_decoding_eta_b200 import _lib as L
+    if engine == "fma":
+        pytest.skip("one comparison of the two screens is enough")
+    w = synth.Workload("tc-screen", B=B, Hq=G * Hkv, Hkv=Hkv, d=128, ctx=ctx, blk=64,
+                       n_clusters=24, seg=(200, 500), needles=2, gate_T=0.0, density=0.35,
+                       density_kind="union", q_scale=2.0, seed=600 + B + G)
+    lens = [(ctx - 977 * i) if i % 3 else ctx for i in range(B)]
+    lens = [max(x, 1) for x in lens]
+    g = to_dev(make(w, lengths=torch.tensor(lens, dtype=torch.int32)))
+    dec = EtaDecoder(g["K"], g["V"], g["lengths"], w.Hq, w.blk, bound=bound, z=2.0, T=0.0,
+                     cent_format="bf16")
+    dims = dec.dims
+    R, NB = B * Hkv, dec.NB
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    assert L.eta_screen_launches(dims, "bf16") == (1 if R <= n_sm and (NB + 127) // 128 <= 32
+                                                   else 2)
+    dec.build_meta()
+    q = g["q"]
+    bias = torch.zeros(w.Hq, device=DEV)
+    dec.predict_tau(q, g["W"], bias)
+    out = {}
+    for eng in ("tcgen05", "fma"):
+        L.eta_set_screen_engine(eng)
+        bnd = torch.empty(B, w.Hq, NB, device=DEV)
+        dec.screen(q, bounds=bnd)
+        if eng == "tcgen05":
+            # threshold offset for ~35% union, from the tensor-core bounds
+            m = (bnd - dec.tau[..., None]).view(B, Hkv, G, NB).amax(2).flatten()
+            off = float(torch.quantile(m.float()[::3], 0.65))
+            dec.tau += off
+            dec.screen(q, bounds=bnd)
+        torch.cuda.synchronize()
+        dec.check_status()
+        out[eng] = dict(b=bnd.clone(), hm=dec.head_mask.clone(), uc=dec.union_cnt.clone(),
+                        ui=dec.union_idx.clone())
+    L.eta_set_screen_engine("auto")
+    t, f = out["tcgen05"], out["fma"]
+    valid = dec.cnt.view(B, Hkv, 1, NB).expand(B, Hkv, G, NB).reshape(B, w.Hq, NB) > 0
+    db = (t["b"] - f["b"]).abs()[valid]
+    assert float(db.max()) <= 1e-4 * max(1.0, float(f["b"][valid].abs().max()))
+    tau = dec.tau[..., None]
+    near = ((f["b"] - tau).abs() <= 1e-5 * torch.clamp(tau.abs(), min=1.0)) & valid
+    mt, mf = unpack_mask(t["hm"], NB), unpack_mask(f["hm"], NB)
+    diff = (mt != mf)
+    assert not np.any(diff & ~near.cpu().numpy()), int(np.sum(diff & ~near.cpu().numpy()))
+    # union lists follow the words
+    ut = mt.reshape(B, Hkv, G, NB).any(2)
+    cnt_t = t["uc"].cpu().numpy()
+    assert np.array_equal(cnt_t, ut.sum(-1))
+    ui = t["ui"].cpu().numpy()
+    for b in range(B):
+        for k in range(Hkv):
+            assert np.array_equal(ui[b, k, :cnt_t[b, k]], np.nonzero(ut[b, k])[0])
+    adm = float(ut.mean())
+    assert 0.05 < adm < 0.95, adm

@@ -220,16 +220,19 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
-      int i = 0;
+      int i = 0, cur_r = -1;
+      float tsv[G];                       // the current row's thresholds
       for (; i < n_local && ok; ++i) {
         const int it = a + i, r = it / p.ngrp, grp = it % p.ngrp;
         const int s = i % NSTAGE;
         const int j0 = grp * GB;
         const int nb = min(GB, p.NB - j0);
         const int qrow = (r / p.Hkv) * p.Hq + (r % p.Hkv) * G;
-        float tsv[G];                     // loaded before the wait: its latency overlaps it
+        if (r != cur_r) {                 // loaded before the wait: its latency overlaps it
 #pragma unroll
-        for (int h = 0; h < G; ++h) tsv[h] = p.tau[qrow + h];
+          for (int h = 0; h < G; ++h) tsv[h] = p.tau[qrow + h];
+          cur_r = r;
+        }
         // (checked build) the group's metadata slices lie inside the row
         if (!ETA_RANGE_IN_BOUNDS(j0, j0 + nb, p.NB, p.status) ||
             !mbar_wait(&ms->empty[s], ((uint32_t)(i / NSTAGE) & 1u) ^ 1u, abort_flag)) {

@@ -348,11 +348,11 @@ inline bool tc_screen_rows(int R, int NB) {
 }
 
 // ETA_ENGINE_AUTO takes the tensor cores where they measured faster on one B200: the
-// one-launch form (128K / B = 16: 23.5 vs 27.7 us for screen + compaction; the
+// one-launch form (128K / B = 16: 21.4 vs 27.7 us for screen + compaction; the
 // one-launch step at B = 8, 32K: 76.6 vs 82.4 us per step).  For larger batches the
-// CUDA-core screen is a little faster (128K / B = 64: 42.1 vs 46.0 us): each tensor-
-// core CTA takes ~0.96 us per 128-block group (its single epilogue chain) after a
-// ~4 us start-up, where the CUDA-core kernel's thousands of warps start at once.
+// CUDA-core screen is a little faster (128K / B = 64: 42.1 vs 45.8 us): each tensor-
+// core CTA pays a ~4 us start-up before its first group lands, where the CUDA-core
+// kernel's thousands of warps start at once.
 bool tc_screen_applies(const eta_dims_t* d, int cent_format, int bound) {
   const int e = g_screen_engine.load();
   if (e == ETA_ENGINE_FMA || cent_format != ETA_CENT_BF16 || d->d != 128 ||

@@ -15,7 +15,8 @@
 // every screening form that takes this path (eta_screen and the one-launch step)
 // shares these functions and writes identical bits.
 //
-// Epilogue: four warps, thread t = block t of the group (= TMEM lane): one tcgen05.ld
+// Epilogue: four warps (the standalone kernel runs two such groups on alternate
+// groups), thread t = block t of the group (= TMEM lane): one tcgen05.ld
 // of the 16 accumulator columns and the block's rmax / var / cnt from the stage
 // (after which the stage and the accumulator are released), then per head the
 // bound, the admit bit and a ballot into the 32-bit admit word of the warp's 32
@@ -136,7 +137,10 @@ ETA_DEV int epilogue(const float (&dot)[16], BlockMeta bm, float scale, int NB, 
 
 // ------------------------------------------------------------------ standalone kernel
 constexpr int NSTAGE = 6;
-constexpr int NT = 6 * 32;          // warps 0-3 epilogue, 4 TMA producer, 5 MMA issuer
+// warps 0-7 epilogue (two groups of four taking alternate items, one TMEM accumulator
+// each), warp 8 TMA producer, warp 9 MMA issuer
+constexpr int NT = 10 * 32;
+constexpr int kWarpTma = 8, kWarpMma = 9;
 
 struct Params {
   int Hq, Hkv, NB, NW, ngrp, items, chunk, prob;
@@ -204,7 +208,7 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
     ms->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&ms->tmem_base)),
                  "r"(32));
@@ -216,7 +220,7 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
   const uint32_t tmem = ms->tmem_base;
   ETA_PDL_ENTRY();
 
-  if (warp == 4) {
+  if (warp == kWarpTma) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
@@ -263,7 +267,7 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
           mbar_wait(&ms->full[k % NSTAGE], (uint32_t)(k / NSTAGE) & 1u, nullptr);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = true;
@@ -287,15 +291,18 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
       mbar_wait(&ms->fin, 0, nullptr);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 0-3)
-    const uint32_t lane_sel = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------------------ epilogue (warps 0-7)
+    // group eg = warp / 4 takes the items i with i % 2 == eg, i.e. accumulator eg;
+    // warp w reads TMEM lanes 32 (w % 4) .. + 31
+    const int eg = warp >> 2;
+    const uint32_t lane_sel = (uint32_t)((warp & 3) * 32) << 16;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
     };
     int cur_r = -1;
     bool ok = true;
     float qn[G], ts[G];                     // every warp holds the row's norms itself
-    for (int i = 0; i < n_local; ++i) {
+    for (int i = eg; i < n_local; i += 2) {
       const int it = a + i, r = it / p.ngrp, grp = it % p.ngrp;
       const int s = i % NSTAGE, b = i & 1;
       const size_t qhead0 = (size_t)(r / p.Hkv) * p.Hq + (size_t)(r % p.Hkv) * G;
@@ -342,7 +349,7 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
                        [] { named_bar_sync(1, 128); });
     }
   }
-  if (warp == 5) {
+  if (warp == kWarpMma) {
     __syncwarp();
     tc::tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(32));

@@ -176,12 +176,11 @@ static_assert(sizeof(CompactScratch<128>) <= TILE, "compaction scratch");
 
 // Items are (row, group) pairs in row-major order; CTA c screens items
 // [c * chunk, min((c + 1) * chunk, items)) in order, so its in-flight tiles are
-// neighbouring 256-byte strips of the same dimension-major centroid rows (items
-// dealt round-robin over the CTAs met twice the DRAM latency: 6.1 vs 3.7 us from
-// copy issue to data).  ROWS (chunk = groups per row, one CTA per row): the CTA then
-// compacts its row's union list as compact_kernel does.  A row change costs no
-// global round trip: the norms come from the staged query rows, the thresholds
-// from the stage's record.
+// neighbouring 256-byte strips of the same dimension-major centroid rows (items dealt
+// round-robin over the CTAs measured slower: 54 vs 46 us at 128K, B = 64).  ROWS
+// (chunk = groups per row, one CTA per row): the CTA then compacts its row's union
+// list as compact_kernel does.  A row change costs no global round trip: the norms
+// come from the staged query rows, the thresholds from the stage's record.
 template <int G, bool ROWS>
 __global__ void __launch_bounds__(NT, 1)
 screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmQ,

@@ -355,7 +355,7 @@ eta_status_t eta_dense_decode(const eta_dims_t* dims, const eta_bf16_t* q,
  * against the float64 oracle):
  *   ETA_ENGINE_TCGEN05 -- q.k and p.v on the tensor cores (tcgen05.mma, TMEM
  *                         accumulators, TMA tensor copies with 128-byte swizzle);
- *                         d = 128 only (other d fall back to the FMA engine)
+ *                         d = 128 and d = 64
  *   ETA_ENGINE_FMA     -- q.k and p.v on the CUDA cores in fp32 (1-D TMA bulk copies)
  *   ETA_ENGINE_AUTO    -- the default: the engine this library measures fastest
  * eta_set_decode_engine returns ETA_ERR_INVALID_ARG for an unknown value.

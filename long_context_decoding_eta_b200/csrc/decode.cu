@@ -557,7 +557,7 @@ inline bool use_tc(const eta_dims_t* d) {
   const bool fits = (uint64_t)d->B * d->Hkv * d->T_max < (1ull << 31);
   // AUTO and TCGEN05: the tensor-core engine wherever it applies (measured ~1.6x the
   // FMA engine's bandwidth on the 128K / B = 64 workload)
-  return d->d == 128 && fits;
+  return (d->d == 128 || d->d == 64) && fits;
 }
 
 // Whether the tensor-core sparse decode plans its shares in the kernel.  Measured on
@@ -569,19 +569,20 @@ inline bool plan_in_kernel(const eta_dims_t* d) {
   return use_tc(d) && R >= kPlanInMinRows && R <= tc::kFusedMaxRows;
 }
 
-template <int G, bool DENSE>
+template <int G, bool DENSE, int DD>
 eta_status_t launch_tc_t(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq,
                          const tc::TcParams& prm, int P, bool plan_in, cudaStream_t s) {
   if constexpr (!DENSE) {
     if (plan_in) {
-      auto kern = tc::decode_tc_kernel<G, false, true>;
-      if (!set_smem_once<tc::decode_tc_kernel<G, false, true>>(tc::FUSED_SMEM_BYTES))
+      auto kern = tc::decode_tc_kernel<G, false, true, DD>;
+      if (!set_smem_once<tc::decode_tc_kernel<G, false, true, DD>>(tc::FUSED_SMEM_BYTES))
         return ETA_ERR_CUDA;
       return launch_k(kern, dim3(P), dim3(tc::NT), tc::FUSED_SMEM_BYTES, s, mk, mv, mq, prm);
     }
   }
-  auto kern = tc::decode_tc_kernel<G, DENSE>;
-  if (!set_smem_once<tc::decode_tc_kernel<G, DENSE>>(tc::SMEM_BYTES)) return ETA_ERR_CUDA;
+  auto kern = tc::decode_tc_kernel<G, DENSE, false, DD>;
+  if (!set_smem_once<tc::decode_tc_kernel<G, DENSE, false, DD>>(tc::SMEM_BYTES))
+    return ETA_ERR_CUDA;
   return launch_k(kern, dim3(P), dim3(tc::NT), tc::SMEM_BYTES, s, mk, mv, mq, prm);
 }
 
@@ -593,8 +594,9 @@ eta_status_t launch_tc(const eta_dims_t* dims, const DecodeParams& d, const eta_
                        const int32_t* counts, cudaStream_t s) {
   CUtensorMap mk, mv, mq;
   const uint64_t kv_rows = (uint64_t)dims->B * dims->Hkv * dims->T_max;
-  if (!make_map(&mk, K, kv_rows, 64) || !make_map(&mv, V, kv_rows, 64) ||
-      !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16))
+  const uint64_t dcols = (uint64_t)dims->d;
+  if (!make_map(&mk, K, kv_rows, 64, dcols) || !make_map(&mv, V, kv_rows, 64, dcols) ||
+      !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16, dcols))
     return ETA_ERR_CUDA;
   tc::TcParams prm;
   prm.Hq = d.Hq; prm.Hkv = d.Hkv; prm.T_max = d.T_max; prm.NB = d.NB; prm.blk = d.blk;
@@ -605,11 +607,16 @@ eta_status_t launch_tc(const eta_dims_t* dims, const DecodeParams& d, const eta_
   prm.counts = counts;
   prm.row_off_g = const_cast<int32_t*>(d.row_off);   // the workspace
   prm.plan_g = const_cast<int32_t*>(d.plan);
+  const bool d64 = dims->d == 64;
   switch (dims->Hq / dims->Hkv) {
-    case 1: return launch_tc_t<1, DENSE>(mk, mv, mq, prm, P, plan_in, s);
-    case 2: return launch_tc_t<2, DENSE>(mk, mv, mq, prm, P, plan_in, s);
-    case 4: return launch_tc_t<4, DENSE>(mk, mv, mq, prm, P, plan_in, s);
-    case 8: return launch_tc_t<8, DENSE>(mk, mv, mq, prm, P, plan_in, s);
+    case 1: return d64 ? launch_tc_t<1, DENSE, 64>(mk, mv, mq, prm, P, plan_in, s)
+                       : launch_tc_t<1, DENSE, 128>(mk, mv, mq, prm, P, plan_in, s);
+    case 2: return d64 ? launch_tc_t<2, DENSE, 64>(mk, mv, mq, prm, P, plan_in, s)
+                       : launch_tc_t<2, DENSE, 128>(mk, mv, mq, prm, P, plan_in, s);
+    case 4: return d64 ? launch_tc_t<4, DENSE, 64>(mk, mv, mq, prm, P, plan_in, s)
+                       : launch_tc_t<4, DENSE, 128>(mk, mv, mq, prm, P, plan_in, s);
+    case 8: return d64 ? launch_tc_t<8, DENSE, 64>(mk, mv, mq, prm, P, plan_in, s)
+                       : launch_tc_t<8, DENSE, 128>(mk, mv, mq, prm, P, plan_in, s);
   }
   return ETA_ERR_UNSUPPORTED;
 }

@@ -260,10 +260,16 @@ ETA_DEV void plan_local(const int32_t* counts, int R, int NB, int* row_off, Fuse
 // PLAN_IN (with PDL_IN, sparse): no plan launch; every CTA lays the shares out itself
 // (plan_local, from the admitted counts) and CTA 0 publishes row_off and the plan
 // for the combine launch.
-template <int G, bool DENSE, bool LOCAL, bool FLAGS, bool PDL_IN = false, bool PLAN_IN = false>
+// DD (head dimension) 128, or 64: then one 64-dim box per K/V sub-tile and for the
+// query rows, QK^T in 4 steps of 16 dims, and P V still M = 128 (the V tile's upper
+// 64-dim half stays zero, so those accumulator rows are zero and not written out).
+template <int G, bool DENSE, bool LOCAL, bool FLAGS, bool PDL_IN = false, bool PLAN_IN = false,
+          int DD = 128>
 ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const CUtensorMap* tmV,
                             const CUtensorMap* tmQ, const TcParams& p, const FuseCtx& fx) {
   static_assert(G >= 1 && G <= 8, "G");
+  static_assert(DD == 128 || (DD == 64 && !LOCAL), "d = 64 in the standalone decode");
+  constexpr int NHALF = DD / 64;   // 64-dim boxes per K/V sub-tile and per query tile
   static_assert(!(LOCAL && DENSE), "the in-kernel merge is for the sparse decode");
   static_assert(!FLAGS || LOCAL, "flags come with the local plan");
   static_assert(!PLAN_IN || (PDL_IN && !DENSE && !LOCAL), "plan in the standalone sparse decode");
@@ -370,17 +376,20 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
           mbar_arrive(&ms->full[s]);
         } else {
           const int nsub = nvb > 0 ? 2 : 1;
-          mbar_arrive_expect_tx(&ms->full[s], (uint32_t)(nsub * 4 * SUB_HALF + 2 * QHALF));
+          mbar_arrive_expect_tx(&ms->full[s],
+                                (uint32_t)(NHALF * (nsub * 2 * SUB_HALF + QHALF)));
           const int b = row / p.Hkv, g = row % p.Hkv;
           const int qrow = b * p.Hq + g * G;
           tma_load_2d(st + OFF_Q0, tmQ, 0, qrow, &ms->full[s]);
-          tma_load_2d(st + OFF_Q1, tmQ, 64, qrow, &ms->full[s]);
+          if constexpr (NHALF == 2) tma_load_2d(st + OFF_Q1, tmQ, 64, qrow, &ms->full[s]);
           for (int u = 0; u < nsub; ++u) {
             const int y = row * p.T_max + (u == 0 ? t0a : t0b);
             tma_load_2d(st + OFF_K0 + u * SUB_HALF, tmK, 0, y, &ms->full[s]);
-            tma_load_2d(st + OFF_K1 + u * SUB_HALF, tmK, 64, y, &ms->full[s]);
             tma_load_2d(st + OFF_V0 + u * SUB_HALF, tmV, 0, y, &ms->full[s]);
-            tma_load_2d(st + OFF_V1 + u * SUB_HALF, tmV, 64, y, &ms->full[s]);
+            if constexpr (NHALF == 2) {
+              tma_load_2d(st + OFF_K1 + u * SUB_HALF, tmK, 64, y, &ms->full[s]);
+              tma_load_2d(st + OFF_V1 + u * SUB_HALF, tmV, 64, y, &ms->full[s]);
+            }
           }
         }
         ++it;
@@ -496,7 +505,7 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
         tc_fence_after();
         unsigned char* st = smem + s * STAGE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < DD / 16; ++kk) {
           const uint32_t koff = (uint32_t)(kk & 3) * 32;
           const uint32_t ka = smem_u32(st + (kk < 4 ? OFF_K0 : OFF_K1)) + koff;
           const uint32_t qb = smem_u32(st + (kk < 4 ? OFF_Q0 : OFF_Q1)) + koff;
@@ -580,7 +589,7 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
         const bool slot_ok = ETA_IN_BOUNDS(slot, (long long)gridDim.x + p.R, p.status);
 #pragma unroll
         for (int h = 0; h < G && slot_ok; ++h) {
-          p.part_o[(slot * G + h) * D + t] = o_acc[h];
+          if (t < DD) p.part_o[(slot * G + h) * DD + t] = o_acc[h];
           if (t == 0) {
             float L = 0.f;
 #pragma unroll
@@ -733,14 +742,15 @@ ETA_DEV void decode_tc_body(unsigned char* smem, const CUtensorMap* tmK, const C
   }
 }
 
-template <int G, bool DENSE, bool PLAN_IN = false>
+template <int G, bool DENSE, bool PLAN_IN = false, int DD = 128>
 __global__ void __launch_bounds__(NT, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmQ, const TcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  decode_tc_body<G, DENSE, false, false, true, PLAN_IN>(smem, &tmK, &tmV, &tmQ, p, FuseCtx{});
+  decode_tc_body<G, DENSE, false, false, true, PLAN_IN, DD>(smem, &tmK, &tmV, &tmQ, p,
+                                                             FuseCtx{});
 }
 
 }  // namespace tc

@@ -1,4 +1,4 @@
-// Host-side TMA tensor maps: the bf16 [rows, 128] views the tcgen05 kernels load
+// Host-side TMA tensor maps: the bf16 [rows, d] views the tcgen05 kernels load
 // (K, V, queries; box of 64 columns x box_rows rows with 128-byte swizzle), the
 // swizzled bf16 centroid view of the tensor-core screen, and plain 2-D views (the
 // CUDA-core screens' metadata tiles).  The encoder is the driver's
@@ -26,12 +26,13 @@ inline EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// 2-D view [rows, 128] of a bf16 tensor (row stride 256 bytes).
-inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+// 2-D view [rows, cols] of a bf16 tensor (cols 128 or 64; row stride 2 cols bytes).
+inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows,
+                     uint64_t cols = 128) {
   EncodeTiledFn fn = encode_tiled();
   if (!fn) return false;
-  cuuint64_t gdim[2] = {128, rows};
-  cuuint64_t gstride[1] = {128 * 2};
+  cuuint64_t gdim[2] = {cols, rows};
+  cuuint64_t gstride[1] = {cols * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box,

@@ -117,6 +117,25 @@ def test_long_128k_b64_union16(engine, cent):
     print(rep, dens)
 
 
+@pytest.mark.parametrize("engine", ["auto", "fma"])
+def test_d64_b32_ctx64k_union16(engine):
+    """Head dimension 64 at a realistic size (B = 32, 16 / 4 heads, 64K context, 128
+    (row, KV head) pairs): the tensor-core decode (one 64-dim box per sub-tile, P V
+    over a zero upper half) with its in-kernel share plan, and the CUDA-core engine,
+    against the oracle on sampled rows."""
+    w = synth.LONG128K.with_(d=64, B=32, ctx=65536)
+    from long_context_decoding_eta_b200 import _lib as L
+    dims = L.Dims.of(w.B, w.Hq, w.Hkv, w.d, w.blk, w.T_max)
+    L.eta_set_decode_engine(engine)
+    try:
+        assert L.eta_decode_launches(dims) == (2 if engine != "fma" else 3)
+    finally:
+        L.eta_set_decode_engine("auto")
+    rep, dens = run_fullsize(w, rows=[0, 17, 31], engine=engine, cent_format="bf16")
+    assert 0.01 < dens < 0.6, dens
+    print(rep, dens)
+
+
 @pytest.mark.parametrize("density,kind", [(0.38, "head"), (0.51, "union")])
 def test_long_128k_b64_trained_operating_points(density, kind):
     """The 128K configuration at the pages' trained operating point: about 38% of

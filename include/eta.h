@@ -161,9 +161,9 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  * ws/ws_bytes: scratch of at least eta_screen_workspace_size(dims) bytes.
  * Two forms compute the q . cent products (both tested against the float64 oracle;
  * their fp32 sums differ in order, so they agree up to rounding, i.e. near-ties):
- *   tensor cores (bf16 centroids, d = 128, ETA_BOUND_EXACT or _PROB, NB % 8 == 0,
- *     every pointer 16-byte aligned): a 128-block group's products as one
- *     tcgen05.mma (M = 128 blocks, N = 16, K = d) from TMA-staged tiles;
+ *   tensor cores (bf16 centroids, d = 128 or 64, ETA_BOUND_EXACT or _PROB,
+ *     NB % 8 == 0, every pointer 16-byte aligned): a 128-block group's products as
+ *     one tcgen05.mma (M = 128 blocks, N = 16, K = d) from TMA-staged tiles;
  *   CUDA cores: fp32 FMA chains.
  * eta_set_screen_engine (process-wide) chooses: ETA_ENGINE_TCGEN05 the tensor cores
  * wherever they apply, ETA_ENGINE_FMA the CUDA cores always, ETA_ENGINE_AUTO (the

@@ -37,7 +37,7 @@ inline eta_status_t check_dims(const eta_dims_t* d, bool rows_in_grid_y = true) 
 }
 
 // Whether the block screening of these dims takes the tensor-core form
-// (screen_tc.cuh): bf16 centroids, d = 128, not the per-dimension bound, NB a
+// (screen_tc.cuh): bf16 centroids, d = 128 or 64, not the per-dimension bound, NB a
 // multiple of 8 (the centroid rows' TMA stride), and the process-wide screen engine
 // (eta_set_screen_engine): ETA_ENGINE_TCGEN05 wherever that applies, ETA_ENGINE_AUTO
 // only in the sizes where it measured faster, ETA_ENGINE_FMA never.  eta_screen and

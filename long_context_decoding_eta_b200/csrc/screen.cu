@@ -355,23 +355,24 @@ inline bool tc_screen_rows(int R, int NB) {
 // kernel's thousands of warps start at once.
 bool tc_screen_applies(const eta_dims_t* d, int cent_format, int bound) {
   const int e = g_screen_engine.load();
-  if (e == ETA_ENGINE_FMA || cent_format != ETA_CENT_BF16 || d->d != 128 ||
+  if (e == ETA_ENGINE_FMA || cent_format != ETA_CENT_BF16 || (d->d != 128 && d->d != 64) ||
       bound == ETA_BOUND_PROB_DIM || num_blocks(d) % 8 != 0)
     return false;
   return e == ETA_ENGINE_TCGEN05 || tc_screen_rows(d->B * d->Hkv, num_blocks(d));
 }
 
-template <int G>
+template <int D, int G>
 static eta_status_t launch_screen_tc(bool rows, const CUtensorMap& mc, const CUtensorMap& mq,
                                      const stc::Params& prm, int grid, cudaStream_t s) {
+  constexpr int SM = stc::Ring<D>::SMEM_BYTES;
   if (rows) {
-    if (!set_smem_once<stc::screen_tc_kernel<G, true>>(stc::SMEM_BYTES)) return ETA_ERR_CUDA;
-    return launch_k(stc::screen_tc_kernel<G, true>, dim3(grid), dim3(stc::NT), stc::SMEM_BYTES,
-                    s, mc, mq, prm);
+    if (!set_smem_once<stc::screen_tc_kernel<D, G, true>>(SM)) return ETA_ERR_CUDA;
+    return launch_k(stc::screen_tc_kernel<D, G, true>, dim3(grid), dim3(stc::NT), SM, s, mc, mq,
+                    prm);
   }
-  if (!set_smem_once<stc::screen_tc_kernel<G, false>>(stc::SMEM_BYTES)) return ETA_ERR_CUDA;
-  return launch_k(stc::screen_tc_kernel<G, false>, dim3(grid), dim3(stc::NT), stc::SMEM_BYTES, s,
-                  mc, mq, prm);
+  if (!set_smem_once<stc::screen_tc_kernel<D, G, false>>(SM)) return ETA_ERR_CUDA;
+  return launch_k(stc::screen_tc_kernel<D, G, false>, dim3(grid), dim3(stc::NT), SM, s, mc, mq,
+                  prm);
 }
 
 // eta_screen on the tensor cores (tc_screen_applies).  Pointers are 16-byte aligned.
@@ -384,8 +385,9 @@ static eta_status_t run_screen_tc(const eta_dims_t* dims, const eta_bf16_t* q, c
   const int NB = num_blocks(dims), NW = num_words(dims);
   const int R = dims->B * dims->Hkv, G = dims->Hq / dims->Hkv;
   CUtensorMap mc, mq;
-  if (!make_map_bf16_swz(&mc, cent, NB, (uint64_t)R * stc::D, (uint64_t)NB * 2, stc::D) ||
-      !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16))
+  const int D = dims->d;
+  if (!make_map_bf16_swz(&mc, cent, NB, (uint64_t)R * D, (uint64_t)NB * 2, (uint32_t)D) ||
+      !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16, (uint64_t)D))
     return ETA_ERR_CUDA;
   stc::Params prm;
   prm.Hq = dims->Hq; prm.Hkv = dims->Hkv; prm.NB = NB; prm.NW = NW;
@@ -408,11 +410,16 @@ static eta_status_t run_screen_tc(const eta_dims_t* dims, const eta_bf16_t* q, c
     grid = (prm.items + prm.chunk - 1) / prm.chunk;
   }
   eta_status_t st = ETA_ERR_UNSUPPORTED;
+  const bool d64 = D == 64;
   switch (G) {
-    case 1: st = launch_screen_tc<1>(rows, mc, mq, prm, grid, s); break;
-    case 2: st = launch_screen_tc<2>(rows, mc, mq, prm, grid, s); break;
-    case 4: st = launch_screen_tc<4>(rows, mc, mq, prm, grid, s); break;
-    case 8: st = launch_screen_tc<8>(rows, mc, mq, prm, grid, s); break;
+    case 1: st = d64 ? launch_screen_tc<64, 1>(rows, mc, mq, prm, grid, s)
+                     : launch_screen_tc<128, 1>(rows, mc, mq, prm, grid, s); break;
+    case 2: st = d64 ? launch_screen_tc<64, 2>(rows, mc, mq, prm, grid, s)
+                     : launch_screen_tc<128, 2>(rows, mc, mq, prm, grid, s); break;
+    case 4: st = d64 ? launch_screen_tc<64, 4>(rows, mc, mq, prm, grid, s)
+                     : launch_screen_tc<128, 4>(rows, mc, mq, prm, grid, s); break;
+    case 8: st = d64 ? launch_screen_tc<64, 8>(rows, mc, mq, prm, grid, s)
+                     : launch_screen_tc<128, 8>(rows, mc, mq, prm, grid, s); break;
   }
   if (st != ETA_OK || rows) return st;
   return launch_k(compact_kernel, dim3(R), dim3(kCompactThreads), 0, s, dims->Hq, dims->Hkv, G,

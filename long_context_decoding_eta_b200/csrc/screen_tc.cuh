@@ -1,4 +1,4 @@
-// Block screening on the 5th-generation tensor cores: bf16 centroids, d = 128, the
+// Block screening on the 5th-generation tensor cores: bf16 centroids, d = 128 or 64, the
 // exact (Cauchy-Schwarz) and the variance bound (arXiv 2609.20888 abstract: blocks
 // screened "in O(1) time using cached geometric-probabilistic bounds"; evolve.pub
 // review FAQ: a block whose best possible score falls below the threshold is
@@ -8,7 +8,7 @@
 //   D[128 blocks][16] = C^T[128 blocks][d] x Q^T[d][16]
 // (tcgen05.mma kind::f16, bf16 x bf16 products are exact in fp32, fp32 sums in TMEM),
 // the group's G heads in the first G of the 16 columns.  The centroid tile arrives
-// by two TMA tensor copies (128 dims x 64 blocks each, 128-byte swizzle) and is read
+// by two TMA tensor copies (d dims x 64 blocks each, 128-byte swizzle) and is read
 // by the tensor core MN-major (blocks contiguous), the 16 query rows K-major, as the
 // decode reads V and Q.  The fp32 accumulation order differs from the CUDA-core
 // screen's, so the two agree up to fp32 rounding (near-ties), not bit for bit;
@@ -31,32 +31,42 @@
 namespace eta {
 namespace stc {
 
-constexpr int D = 128;
 constexpr int GB = kScreenGroupBlocks;             // blocks per group (128)
-constexpr int CENT_HALF = D * 64 * 2;               // [d rows][64 blocks] bf16: 16 KB
 constexpr int Q_HALF = 16 * 64 * 2;                 // [16 heads][64 dims] bf16: 2 KB
 // A ring stage is a tile (the swizzled centroid and query boxes, 1024-byte aligned)
 // plus a metadata slot (the group's rmax, var and cnt slices); the slots of all
 // stages sit together after the tiles, so that no stage pads its tile to 1 KB.
-constexpr int OFF_C0 = 0, OFF_C1 = CENT_HALF;
-constexpr int OFF_Q0 = 2 * CENT_HALF, OFF_Q1 = OFF_Q0 + Q_HALF;
-constexpr int TILE = 2 * CENT_HALF + 2 * Q_HALF;   // 36 KB
+// D = 128: two 16 KB centroid boxes and two query boxes (36 KB); D = 64: two 8 KB
+// centroid boxes and one query box (18 KB).
+template <int D>
+struct Tile {
+  static_assert(D == 128 || D == 64, "d");
+  static constexpr int CENT_HALF = D * 64 * 2;      // [d rows][64 blocks] bf16
+  static constexpr int NQ = D / 64;                  // 64-dim query boxes
+  static constexpr int OFF_C0 = 0, OFF_C1 = CENT_HALF;
+  static constexpr int OFF_Q0 = 2 * CENT_HALF, OFF_Q1 = OFF_Q0 + Q_HALF;
+  static constexpr int BYTES = 2 * CENT_HALF + NQ * Q_HALF;
+  static_assert(BYTES % 1024 == 0, "swizzled tiles stay 1024-byte aligned");
+};
 constexpr int M_RMAX = 0, M_VAR = 4 * GB, M_CNT = 8 * GB;
 constexpr int META = 12 * GB;                       // 1.5 KB
-static_assert(TILE % 1024 == 0, "swizzled tiles stay 1024-byte aligned");
 // kind::f16, D fp32, bf16 operands, M = 128, N = 16; A (centroids) MN-major, B (q) K-major
 constexpr uint32_t kIdesc = tc::kIdescBase | (1u << 15);
 constexpr int kAccCols = 16;
 
-// The group's q . c products into TMEM columns [d_tmem, d_tmem + 16): K = d in 8
-// steps of 16 dims, in order.  `st` is a stage tile laid out as above (1024-aligned).
+// The group's q . c products into TMEM columns [d_tmem, d_tmem + 16): K = d in
+// d / 16 steps of 16 dims, in order.  `st` is a stage tile laid out as Tile<D>
+// (1024-aligned).
+template <int D>
 ETA_DEV void issue_mma(uint32_t d_tmem, const unsigned char* st) {
-  const uint32_t c0 = smem_u32(st + OFF_C0);
+  using T = Tile<D>;
+  const uint32_t c0 = smem_u32(st + T::OFF_C0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    // A: 16 dims (rows of 128 B) per step; the second 64 blocks 16 KB further on
-    const uint64_t da = tc::smem_desc(c0 + kk * 2048, CENT_HALF, 1024, tc::kSwizzle128);
-    const uint32_t qb = smem_u32(st + (kk < 4 ? OFF_Q0 : OFF_Q1)) + (uint32_t)(kk & 3) * 32;
+    // A: 16 dims (rows of 128 B) per step; the second 64 blocks one box further on
+    const uint64_t da = tc::smem_desc(c0 + kk * 2048, T::CENT_HALF, 1024, tc::kSwizzle128);
+    const uint32_t qb =
+        smem_u32(st + (kk < 4 ? T::OFF_Q0 : T::OFF_Q1)) + (uint32_t)(kk & 3) * 32;
     const uint64_t db = tc::smem_desc(qb, 16, 1024, tc::kSwizzle128);
     tc::mma_f16(d_tmem, da, db, kIdesc, kk > 0 ? 1u : 0u);
   }
@@ -67,8 +77,9 @@ ETA_DEV void issue_mma(uint32_t d_tmem, const unsigned char* st) {
 // c ^ (h % 8)), by one warp into every lane's registers, so that a row change costs
 // no global-memory round trip.  The fmaf order of query_norm (lane k sums dims k,
 // k + 32, ...), then a butterfly sum.
-template <int G>
+template <int D, int G>
 ETA_DEV void query_norms_staged(const unsigned char* st, float (&qn)[G]) {
+  using T = Tile<D>;
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int h = 0; h < G; ++h) {
@@ -76,7 +87,7 @@ ETA_DEV void query_norms_staged(const unsigned char* st, float (&qn)[G]) {
 #pragma unroll
     for (int i = 0; i < D / 32; ++i) {
       const int k = lane + 32 * i, kk = k & 63;
-      const unsigned char* row = st + (k < 64 ? OFF_Q0 : OFF_Q1) + h * 128;
+      const unsigned char* row = st + (k < 64 ? T::OFF_Q0 : T::OFF_Q1) + h * 128;
       const uint16_t bits =
           *reinterpret_cast<const uint16_t*>(row + (((kk >> 3) ^ (h & 7)) << 4) + (kk & 7) * 2);
       const float x = bf16_to_f(bits);
@@ -94,6 +105,7 @@ struct BlockMeta {
   float rad;
   int n;
 };
+template <int D>
 ETA_DEV BlockMeta block_meta(const unsigned char* ms, bool prob, float z, int NB, int grp) {
   const int t = threadIdx.x & 127;
   BlockMeta m{0.f, 0};
@@ -167,12 +179,15 @@ struct Misc {
   uint32_t tmem_base;
   int abort_flag;
 };
-constexpr int OFF_META = NSTAGE * TILE;
-constexpr int OFF_MISC = OFF_META + NSTAGE * META;
-constexpr int SMEM_BYTES = OFF_MISC + (int)sizeof(Misc) + 1024;   // + alignment slack
-static_assert(SMEM_BYTES <= 227 * 1024, "screen_tc shared memory");
-// ROWS: the compaction's scratch reuses the first tile once every item is screened
-static_assert(sizeof(CompactScratch<128>) <= TILE, "compaction scratch");
+template <int D>
+struct Ring {
+  static constexpr int OFF_META = NSTAGE * Tile<D>::BYTES;
+  static constexpr int OFF_MISC = OFF_META + NSTAGE * META;
+  static constexpr int SMEM_BYTES = OFF_MISC + (int)sizeof(Misc) + 1024;   // + align slack
+  static_assert(SMEM_BYTES <= 227 * 1024, "screen_tc shared memory");
+  // ROWS: the compaction's scratch reuses the first tile once every item is screened
+  static_assert(sizeof(CompactScratch<128>) <= Tile<D>::BYTES, "compaction scratch");
+};
 
 // Items are (row, group) pairs in row-major order; CTA c screens items
 // [c * chunk, min((c + 1) * chunk, items)) in order, so its in-flight tiles are
@@ -181,14 +196,16 @@ static_assert(sizeof(CompactScratch<128>) <= TILE, "compaction scratch");
 // (chunk = groups per row, one CTA per row): the CTA then compacts its row's union
 // list as compact_kernel does.  A row change costs no global round trip: the norms
 // come from the staged query rows, the thresholds from the stage's record.
-template <int G, bool ROWS>
+template <int D, int G, bool ROWS>
 __global__ void __launch_bounds__(NT, 1)
 screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmQ,
                  const Params p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Misc* ms = reinterpret_cast<Misc*>(smem + OFF_MISC);
+  using T = Tile<D>;
+  using RG = Ring<D>;
+  Misc* ms = reinterpret_cast<Misc*>(smem + RG::OFF_MISC);
   volatile int* abort_flag = &ms->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int a = blockIdx.x * p.chunk;
@@ -244,15 +261,14 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) ms->ts[s][h] = tsv[h];   // published by the arrive below
-        unsigned char* st = smem + s * TILE;
-        unsigned char* mt = smem + OFF_META + s * META;
+        unsigned char* st = smem + s * T::BYTES;
+        unsigned char* mt = smem + RG::OFF_META + s * META;
         const uint32_t nb4 = (uint32_t)nb * 4u;
-        mbar_arrive_expect_tx(&ms->full[s], (uint32_t)(2 * CENT_HALF + 2 * Q_HALF) +
-                                                nb4 * (p.prob ? 3u : 2u));
-        tc::tma_load_2d(st + OFF_C0, &tmC, j0, r * D, &ms->full[s]);
-        tc::tma_load_2d(st + OFF_C1, &tmC, j0 + 64, r * D, &ms->full[s]);
-        tc::tma_load_2d(st + OFF_Q0, &tmQ, 0, qrow, &ms->full[s]);
-        tc::tma_load_2d(st + OFF_Q1, &tmQ, 64, qrow, &ms->full[s]);
+        mbar_arrive_expect_tx(&ms->full[s], (uint32_t)T::BYTES + nb4 * (p.prob ? 3u : 2u));
+        tc::tma_load_2d(st + T::OFF_C0, &tmC, j0, r * D, &ms->full[s]);
+        tc::tma_load_2d(st + T::OFF_C1, &tmC, j0 + 64, r * D, &ms->full[s]);
+        tc::tma_load_2d(st + T::OFF_Q0, &tmQ, 0, qrow, &ms->full[s]);
+        if constexpr (T::NQ == 2) tc::tma_load_2d(st + T::OFF_Q1, &tmQ, 64, qrow, &ms->full[s]);
         const size_t rj = (size_t)r * p.NB + j0;
         bulk_g2s(mt + M_RMAX, p.rmax + rj, nb4, &ms->full[s]);
         if (p.prob) bulk_g2s(mt + M_VAR, p.var + rj, nb4, &ms->full[s]);
@@ -278,7 +294,7 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
           break;
         }
         tc::tc_fence_after();
-        issue_mma(tmem + b * kAccCols, smem + s * TILE);
+        issue_mma<D>(tmem + b * kAccCols, smem + s * T::BYTES);
         tc::mma_commit(&ms->acc_full[b]);
       }
       if (!ok) {
@@ -310,7 +326,7 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
         break;
       }
       if (r != cur_r) {
-        query_norms_staged<G>(smem + s * TILE, qn);
+        query_norms_staged<D, G>(smem + s * T::BYTES, qn);
 #pragma unroll
         for (int h = 0; h < G; ++h) ts[h] = ms->ts[s][h];
         cur_r = r;
@@ -323,7 +339,8 @@ screen_tc_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant_
       float dot[16];
       tc::tmem_ld16(tmem + b * kAccCols + lane_sel, dot);
       tc::tc_fence_before();
-      const BlockMeta bm = block_meta(smem + OFF_META + s * META, p.prob != 0, p.z, p.NB, grp);
+      const BlockMeta bm =
+          block_meta<D>(smem + RG::OFF_META + s * META, p.prob != 0, p.z, p.NB, grp);
       __syncwarp();
       if (lane == 0) {                      // accumulator and stage are no longer read
         mbar_arrive(&ms->acc_free[b]);

@@ -207,9 +207,10 @@ ETA_DEV void fence_proxy_async_global() {
 // q . c product into one of two TMEM accumulators and warps 0-3 turn it into the
 // bound, the admit words and the row's admitted count (stc::issue_mma and
 // stc::epilogue, the arithmetic of the standalone tensor-core screen).
-constexpr int kTcFit = tc::SM_P / (stc::TILE + stc::META);
+using TcTile = stc::Tile<128>;
+constexpr int kTcFit = tc::SM_P / (TcTile::BYTES + stc::META);
 constexpr int kTcStages = kTcFit < tc::kFuseStages ? kTcFit : tc::kFuseStages;
-constexpr int kTcMeta = kTcStages * stc::TILE;         // the stages' metadata slots
+constexpr int kTcMeta = kTcStages * TcTile::BYTES;     // the stages' metadata slots
 static_assert(kTcStages >= 2, "two tensor-core screening stages must fit");
 static_assert(kTcMeta + kTcStages * stc::META <= tc::SM_P, "screening ring in the decode ring");
 
@@ -253,18 +254,17 @@ ETA_DEV void phase_b_tc(unsigned char* smem, tc::FuseSmem* fs, const StepParams&
         rec.r = r; rec.grp = grp; rec.nvalid = nvalid; rec.flags = 0;
 #pragma unroll
         for (int h = 0; h < G; ++h) rec.ts[h] = ts[h];
-        unsigned char* st = smem + s * stc::TILE;
+        unsigned char* st = smem + s * TcTile::BYTES;
         unsigned char* mt = smem + kTcMeta + s * stc::META;
         const int j0 = grp * stc::GB;
         const uint32_t nb4 = (uint32_t)min(stc::GB, sp.NB - j0) * 4u;
         const bool pv = sp.bound == ETA_BOUND_PROB;
-        mbar_arrive_expect_tx(&fs->bfull[s], (uint32_t)(2 * stc::CENT_HALF + 2 * stc::Q_HALF) +
-                                                 nb4 * (pv ? 3u : 2u));
-        tc::tma_load_2d(st + stc::OFF_C0, tmC, j0, r * D, &fs->bfull[s]);
-        tc::tma_load_2d(st + stc::OFF_C1, tmC, j0 + 64, r * D, &fs->bfull[s]);
+        mbar_arrive_expect_tx(&fs->bfull[s], (uint32_t)TcTile::BYTES + nb4 * (pv ? 3u : 2u));
+        tc::tma_load_2d(st + TcTile::OFF_C0, tmC, j0, r * D, &fs->bfull[s]);
+        tc::tma_load_2d(st + TcTile::OFF_C1, tmC, j0 + 64, r * D, &fs->bfull[s]);
         const int qrow = b * sp.Hq + g * G;
-        tc::tma_load_2d(st + stc::OFF_Q0, tmQ, 0, qrow, &fs->bfull[s]);
-        tc::tma_load_2d(st + stc::OFF_Q1, tmQ, 64, qrow, &fs->bfull[s]);
+        tc::tma_load_2d(st + TcTile::OFF_Q0, tmQ, 0, qrow, &fs->bfull[s]);
+        tc::tma_load_2d(st + TcTile::OFF_Q1, tmQ, 64, qrow, &fs->bfull[s]);
         const size_t rj = (size_t)r * sp.NB + j0;
         bulk_g2s(mt + stc::M_RMAX, sp.rmax + rj, nb4, &fs->bfull[s]);
         if (pv) bulk_g2s(mt + stc::M_VAR, sp.var + rj, nb4, &fs->bfull[s]);
@@ -306,7 +306,7 @@ ETA_DEV void phase_b_tc(unsigned char* smem, tc::FuseSmem* fs, const StepParams&
         break;
       }
       tc::tc_fence_after();
-      stc::issue_mma(tmem + b * stc::kAccCols, smem + s * stc::TILE);
+      stc::issue_mma<D>(tmem + b * stc::kAccCols, smem + s * TcTile::BYTES);
       tc::mma_commit(&fs->bacc_full[b]);
     }
     if (!ok) {
@@ -338,7 +338,7 @@ ETA_DEV void phase_b_tc(unsigned char* smem, tc::FuseSmem* fs, const StepParams&
       const int r = rec.r, bb = r / sp.Hkv, g = r % sp.Hkv;
       const size_t qhead0 = (size_t)bb * sp.Hq + (size_t)g * G;
       if (r != cur_r) {
-        stc::query_norms_staged<G>(smem + s * stc::TILE, qn);
+        stc::query_norms_staged<D, G>(smem + s * TcTile::BYTES, qn);
         cur_r = r;
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&fs->bacc_full[b], (uint32_t)(k >> 1) & 1u,
@@ -352,7 +352,7 @@ ETA_DEV void phase_b_tc(unsigned char* smem, tc::FuseSmem* fs, const StepParams&
       float dot[16];
       tc::tmem_ld16(tmem + b * stc::kAccCols + lane_sel, dot);
       tc::tc_fence_before();
-      const stc::BlockMeta bm = stc::block_meta(smem + kTcMeta + s * stc::META,
+      const stc::BlockMeta bm = stc::block_meta<D>(smem + kTcMeta + s * stc::META,
                                                 sp.bound == ETA_BOUND_PROB, sp.z, sp.NB, rec.grp);
       __syncwarp();
       if (lane == 0) {                      // accumulator and stage are no longer read
@@ -773,7 +773,7 @@ extern "C" eta_status_t eta_decode_step(
   if (!make_map(&mk, K, kv_rows, 64) || !make_map(&mv, V, kv_rows, 64) ||
       !make_map(&mq, q, (uint64_t)dims->B * dims->Hq, 16))
     return ETA_ERR_CUDA;
-  if (tcs ? !make_map_bf16_swz(&mc, cent, NB, meta_rows, (uint64_t)NB * 2, stc::D)
+  if (tcs ? !make_map_bf16_swz(&mc, cent, NB, meta_rows, (uint64_t)NB * 2, 128)
           : !make_map_plain(&mc, cent, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                             NB, meta_rows, (uint64_t)NB * (bf ? 2 : 4), box, 128))

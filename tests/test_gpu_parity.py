@@ -329,19 +329,24 @@ def test_bf16_screen_of_long_rows(d, G, Hkv, bound, engine):
                        blk=64, n_clusters=32, seg=(384, 640), needles=2, gate_T=0.0,
                        density=0.3, density_kind="head", q_scale=2.0, seed=320 + d + G)
     dims = L.Dims.of(w.B, w.Hq, w.Hkv, w.d, w.blk, w.T_max)
-    if engine == "fma" or d == 64:
+    if engine == "fma":
         assert L.eta_screen_launches(dims, "bf16") == 2
     elif bound != "prob_dim":
-        # the tensor-core screen: a CTA per pair with its compaction (13 groups per row)
+        # the tensor-core screen: a CTA per pair with its compaction (13 or 21 groups
+        # per row)
         assert L.eta_screen_launches(dims, "bf16") == 1
     lengths = torch.tensor([w.ctx, w.ctx - 7000], dtype=torch.int32)
     full_parity(w, lengths=lengths, bound=bound, z=2.0, cent_format="bf16")
 
 
-@pytest.mark.parametrize("B,Hkv,G,ctx,bound", [(3, 2, 4, 9216, "exact"), (2, 1, 8, 40960, "prob"),
-                                              (40, 4, 1, 8192, "exact"), (37, 4, 2, 4096, "prob"),
-                                              (20, 8, 4, 6144, "exact")])
-def test_tensor_core_screen_against_cuda_core_screen(B, Hkv, G, ctx, bound, engine):
+@pytest.mark.parametrize("B,Hkv,G,ctx,bound,d", [(3, 2, 4, 9216, "exact", 128),
+                                                (2, 1, 8, 40960, "prob", 128),
+                                                (40, 4, 1, 8192, "exact", 128),
+                                                (37, 4, 2, 4096, "prob", 128),
+                                                (20, 8, 4, 6144, "exact", 128),
+                                                (6, 2, 4, 9216, "prob", 64),
+                                                (40, 4, 2, 8192, "exact", 64)])
+def test_tensor_core_screen_against_cuda_core_screen(B, Hkv, G, ctx, bound, d, engine):
     """eta_screen on the tensor cores (one launch with a CTA per pair for small
     batches, or (row, group) items over one CTA per SM and the compaction after)
     against the CUDA-core screen on the same inputs: the bounds agree to fp32
@@ -351,7 +356,7 @@ def test_tensor_core_screen_against_cuda_core_screen(B, Hkv, G, ctx, bound, engi
     from long_context_decoding_eta_b200 import _lib as L
     if engine == "fma":
         pytest.skip("one comparison of the two screens is enough")
-    w = synth.Workload("tc-screen", B=B, Hq=G * Hkv, Hkv=Hkv, d=128, ctx=ctx, blk=64,
+    w = synth.Workload("tc-screen", B=B, Hq=G * Hkv, Hkv=Hkv, d=d, ctx=ctx, blk=64,
                        n_clusters=24, seg=(200, 500), needles=2, gate_T=0.0, density=0.35,
                        density_kind="union", q_scale=2.0, seed=600 + B + G)
     lens = [(ctx - 977 * i) if i % 3 else ctx for i in range(B)]

@@ -167,8 +167,8 @@ eta_status_t eta_predict_tau(const eta_dims_t* dims, const eta_bf16_t* q, const 
  *   CUDA cores: fp32 FMA chains.
  * eta_set_screen_engine (process-wide) chooses: ETA_ENGINE_TCGEN05 the tensor cores
  * wherever they apply, ETA_ENGINE_FMA the CUDA cores always, ETA_ENGINE_AUTO (the
- * default) the tensor cores where this library measures them faster: when the
- * (row, KV head) pairs fit one per SM and rows have at most 32 groups of 128
+ * default) the tensor cores where this library measures them faster: d = 128 when
+ * the (row, KV head) pairs fit one per SM and rows have at most 32 groups of 128
  * blocks.  The one-launch step follows the same choice.
  * Kernel launches: one (screening and compaction together, one CTA per (row, KV
  * head) pair: the tensor-core form when the pairs fit one per SM and rows have at

@@ -40,7 +40,7 @@ inline eta_status_t check_dims(const eta_dims_t* d, bool rows_in_grid_y = true) 
 // (screen_tc.cuh): bf16 centroids, d = 128 or 64, not the per-dimension bound, NB a
 // multiple of 8 (the centroid rows' TMA stride), and the process-wide screen engine
 // (eta_set_screen_engine): ETA_ENGINE_TCGEN05 wherever that applies, ETA_ENGINE_AUTO
-// only in the sizes where it measured faster, ETA_ENGINE_FMA never.  eta_screen and
+// only where it measured faster (d = 128, the one-launch form), ETA_ENGINE_FMA never.  eta_screen and
 // the one-launch step decide alike, so that both write the same bits.  Defined in
 // screen.cu.
 bool tc_screen_applies(const eta_dims_t* d, int cent_format, int bound);

@@ -348,17 +348,20 @@ inline bool tc_screen_rows(int R, int NB) {
 }
 
 // ETA_ENGINE_AUTO takes the tensor cores where they measured faster on one B200: the
-// one-launch form (128K / B = 16: 21.4 vs 27.7 us for screen + compaction; the
-// one-launch step at B = 8, 32K: 76.6 vs 82.4 us per step).  For larger batches the
-// CUDA-core screen is a little faster (128K / B = 64: 42.1 vs 45.8 us): each tensor-
-// core CTA pays a ~4 us start-up before its first group lands, where the CUDA-core
-// kernel's thousands of warps start at once.
+// one-launch form at d = 128 (128K / B = 16: 21.4 vs 27.7 us for screen + compaction;
+// the one-launch step at B = 8, 32K: 76.6 vs 82.4 us per step).  For larger batches
+// the CUDA-core screen is a little faster (128K / B = 64: 42.1 vs 45.8 us): each
+// tensor-core CTA pays a ~4 us start-up before its first group lands, where the
+// CUDA-core kernel's thousands of warps start at once.  At d = 64 the CUDA-core
+// one-launch screen has half the arithmetic and stays ahead (20.4 vs 16.4 us at
+// 128K / B = 16).
 bool tc_screen_applies(const eta_dims_t* d, int cent_format, int bound) {
   const int e = g_screen_engine.load();
   if (e == ETA_ENGINE_FMA || cent_format != ETA_CENT_BF16 || (d->d != 128 && d->d != 64) ||
       bound == ETA_BOUND_PROB_DIM || num_blocks(d) % 8 != 0)
     return false;
-  return e == ETA_ENGINE_TCGEN05 || tc_screen_rows(d->B * d->Hkv, num_blocks(d));
+  return e == ETA_ENGINE_TCGEN05 ||
+         (d->d == 128 && tc_screen_rows(d->B * d->Hkv, num_blocks(d)));
 }
 
 template <int D, int G>

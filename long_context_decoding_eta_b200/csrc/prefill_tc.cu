@@ -345,6 +345,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             sv[c] = y;
             pm[c & 7] = fmaxf(pm[c & 7], y);
           }
+        } else if (hard) {
+          // every key of an earlier tile precedes every query of this one; the hard
+          // gate as a 1.0 / 0.0 flag (set.ge) and one packed multiply per two scores
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            float g0, g1;
+            asm("set.ge.f32.f32 %0, %1, %2;" : "=f"(g0) : "f"(sv[c]), "f"(tau_raw));
+            asm("set.ge.f32.f32 %0, %1, %2;" : "=f"(g1) : "f"(sv[c + 1]), "f"(tau_raw));
+            const float2 y = __fmul2_rn(make_float2(sv[c], sv[c + 1]), make_float2(g0, g1));
+            sv[c] = y.x;
+            sv[c + 1] = y.y;
+            pm[c & 7] = fmaxf(pm[c & 7], y.x);
+            pm[(c + 1) & 7] = fmaxf(pm[(c + 1) & 7], y.y);
+          }
         } else {
           // every key of an earlier tile precedes every query of this one
 #pragma unroll

@@ -356,8 +356,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             const float2 y = __fmul2_rn(make_float2(sv[c], sv[c + 1]), make_float2(g0, g1));
             sv[c] = y.x;
             sv[c + 1] = y.y;
-            pm[c & 7] = fmaxf(pm[c & 7], y.x);
-            pm[(c + 1) & 7] = fmaxf(pm[(c + 1) & 7], y.y);
+            pm[(c >> 1) & 7] = fmax3(pm[(c >> 1) & 7], y.x, y.y);
           }
         } else {
           // every key of an earlier tile precedes every query of this one
